@@ -101,6 +101,42 @@ def test_on_grid_weights_recovered_exactly(symmetric, g, act_order):
     assert np.array_equal(What, W.view(np.float16).astype(np.float32))
 
 
+@pytest.mark.parametrize("symmetric", [False, True])
+def test_exact_ties_round_to_even(symmetric):
+    # weights exactly half-way between two grid points: W'/sc = j + 0.5 exactly, so
+    # rint must return the even integer -- independent of the (often odd) zero point
+    rng = np.random.default_rng(31 + symmetric)
+    N, K, g = 16, 64, 32
+    G = K // g
+    sc = 2.0 ** -7
+    W = np.zeros((N, K))
+    expect = np.zeros((N, K), bool)
+    for n in range(N):
+        for gg in range(G):
+            ks = np.arange(gg * g, (gg + 1) * g)
+            if symmetric:
+                z = 8
+                W[n, ks[0]], W[n, ks[1]] = -7 * sc, 7 * sc          # absmax = 7 sc
+                lo, hi = -7, 6
+            else:
+                z = int(rng.integers(1, 15))
+                W[n, ks[0]], W[n, ks[1]] = -z * sc, (15 - z) * sc   # range = 15 sc
+                lo, hi = -z, 14 - z
+            j = rng.integers(lo, hi + 1, size=g - 2)
+            W[n, ks[2:]] = (j + 0.5) * sc
+            expect[n, ks[2:]] = True
+    Wb = f16bits(W)
+    assert np.array_equal(Wb.view(np.float16).astype(np.float64), W)
+    q, scales, zeros = oracle.quantize_weights(Wb, None, g, symmetric)
+    assert np.all(oracle.f16_to_f32(scales) == sc)
+    z = np.full((G, N), 8.0) if symmetric else oracle.f16_to_f32(zeros)
+    zk = z[np.arange(K) // g, :].T
+    d = q.astype(np.float64) - zk           # the rounded integer rint(W'/sc)
+    half = W / sc
+    assert np.all(np.abs(d[expect] - half[expect]) == 0.5)
+    assert np.all(d[expect] % 2 == 0)
+
+
 def test_hand_worked_group():
     vals = {}
     for line in open(os.path.join(GOLDEN, "quant_hand_example.txt")):
