@@ -1,0 +1,492 @@
+"""Benchmark of the W4A16 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one decode token (M=1) through the linear projections of a 32-block
+Llama-7B-shaped stack (per block: qkv 4096->12288, o 4096->4096, gate_up 4096->22016,
+down 11008->4096): 128 w4a16_gemm calls on weights quantised by w4_quantize_pack
+(asymmetric INT4, group 128, fp16 scales and zero points, AWQ s_inv applied to the
+activations in-kernel).  The 3.4 GB of packed weights per step are far larger than L2.
+The timed steps are replayed from a CUDA graph.  The metric is effective weight GB/s: algorithmic bytes of packed codes +
+scales + zeros per step / time.  Extra keys report the decode sweep M in {1..16}, the
+prefill GEMM at M=4096 (TFLOPS) and the quantiser.
+
+--impl reference times the CPU oracle (the plain C restatement of the method) on a
+bounded sample of the same workload.  Under torchrun (N > 1) every rank runs an
+independent replica (the path has no exchange step); the value is all ranks' bytes over
+the slowest rank's time.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_weight_only_w4_b200 import workloads  # noqa: E402
+
+METRIC = "W4A16 GEMM: weight GB/s & %HBM peak at M=1; TFLOPS & %TC peak at M=4096"
+DECODE_CFG = 2
+PREFILL_CFG = 4
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def workload_desc(wl, M):
+    shapes = ", ".join(f"{l.name} {l.K}x{l.N}" for l in wl.layers)
+    return f"{wl.name} M={M} ({shapes}); asymmetric INT4 g128, fp16 scales+zeros, AWQ s_inv"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples; only samples stamped inside the timed
+    region [mark_start, mark_end] are summarised."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.5)  # let the sampler come up before the timed region
+        except Exception:
+            self.proc = None
+
+    def mark_start(self):
+        import datetime
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        import datetime
+        self.t1 = datetime.datetime.now()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        import datetime
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            t = [x.strip() for x in line.split(",")]
+            if len(t) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(t[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(t[1]), float(t[2]), t[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        inside = [r for r in rows if self.t0 and self.t1 and self.t0 <= r[0] <= self.t1]
+        use = inside or rows
+        if not use:
+            return None
+        reasons = set()
+        for r in use:
+            for name, v in zip(self.REASONS, r[3]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in use),
+                "sm_max_mhz": max(r[2] for r in use), "reasons": sorted(reasons),
+                "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if (torch.cuda.is_available() and args.impl == "ours") else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- our arm
+def dev_bits(bits, dtype):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dtype).cuda()
+
+
+N_LAYERS = 32   # transformer blocks of the 7B-shaped stack
+
+
+def prepare_weights(w4, torch, n_layers=N_LAYERS):
+    """Seeded projections of one block, quantised once on the GPU, then stored n_layers
+    times (one copy per block of the stack)."""
+    wl = workloads.workload(DECODE_CFG)
+    projs = []
+    for i, L in enumerate(wl.layers):
+        li = workloads.make_layer(wl, i, M=1)
+        W = dev_bits(li.W.view(np.uint16), torch.float16)
+        s = torch.from_numpy(li.s).cuda()
+        qw, sc, zr = w4.w4_quantize_pack(W, s, li.group_size)
+        projs.append({"li": li, "W": W, "s": s, "s_inv": torch.from_numpy(li.s_inv).cuda(),
+                      "bytes": workloads.effective_weight_bytes(li.N, li.K, li.group_size,
+                                                                False, False)})
+        projs[-1]["copies"] = [(qw, sc, zr)] + [(qw.clone(), sc.clone(), zr.clone())
+                                               for _ in range(n_layers - 1)]
+    torch.cuda.synchronize()
+    step_bytes = n_layers * sum(p["bytes"] for p in projs)
+    return wl, projs, step_bytes
+
+
+def make_acts(wl, projs, M, torch):
+    xs = []
+    for i, pr in enumerate(projs):
+        li = workloads.make_layer(wl, i, M=M, with_weights=False)
+        xs.append(dev_bits(li.X, torch.float16))
+    ys = [torch.empty(M, pr["li"].N, dtype=torch.float16, device="cuda") for pr in projs]
+    return xs, ys
+
+
+def run_decode_steps(w4, projs, xs, ys, steps):
+    """`steps` decode tokens: every block of the stack, every projection."""
+    for _ in range(steps):
+        for layer in range(N_LAYERS):
+            for j, pr in enumerate(projs):
+                qw, sc, zr = pr["copies"][layer]
+                w4.w4a16_gemm(xs[j], qw, sc, zr, 128, s_inv=pr["s_inv"], Y=ys[j])
+
+
+def capture(torch, fn):
+    """Capture fn() into a CUDA graph on a side stream (kernels of a few microseconds are
+    replayed without host launch gaps)."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    return g
+
+
+def time_graph(torch, g, world=1, clocks=None):
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        clocks.mark_start()
+    t0.record()
+    g.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark_end()
+    clk = clocks.stop() if clocks else None
+    barrier(world)
+    return t0.elapsed_time(t1), clk
+
+
+def time_decode(M, steps, warmup, w4, torch, world, wl, projs, step_bytes, clocks=None,
+                per_layer=False):
+    xs, ys = make_acts(wl, projs, M, torch)
+    run_decode_steps(w4, projs, xs, ys, warmup)          # untimed warm-up steps
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    g = capture(torch, lambda: run_decode_steps(w4, projs, xs, ys, steps))
+    torch.cuda.synchronize()
+    total_ms, clk = time_graph(torch, g, world, clocks)
+    w4.w4_check_device_error()
+    del g
+    out = {"total_ms": total_ms, "clocks": clk, "launches": steps * N_LAYERS * len(projs)}
+    if per_layer:
+        rows = []
+        for j, pr in enumerate(projs):
+            def one(j=j, pr=pr):
+                for layer in range(N_LAYERS):
+                    qw, sc, zr = pr["copies"][layer]
+                    w4.w4a16_gemm(xs[j], qw, sc, zr, 128, s_inv=pr["s_inv"], Y=ys[j])
+            gj = capture(torch, one)
+            gj.replay()
+            ms, _ = time_graph(torch, gj)
+            us = ms * 1e3 / N_LAYERS
+            rows.append({"layer": f"{pr['li'].name} {pr['li'].K}x{pr['li'].N}",
+                         "us": round(us, 3), "gbs": round(pr["bytes"] / (us * 1e-6) / 1e9, 1)})
+            del gj
+        out["per_layer"] = rows
+    return out
+
+
+def time_e2e(M, steps, warmup, w4, torch, world, wl, projs):
+    """Same metric through the public call with host buffers: each step copies the four
+    projections' activations host->device (pinned), runs every GEMM of the stack and reads
+    the four results back device->host, all inside the timed region (eager calls)."""
+    xs, ys = make_acts(wl, projs, M, torch)
+    hx = [x.cpu().pin_memory() for x in xs]
+    hy = [torch.empty_like(y, device="cpu").pin_memory() for y in ys]
+
+    def step():
+        for j in range(len(projs)):
+            xs[j].copy_(hx[j], non_blocking=True)
+        run_decode_steps(w4, projs, xs, ys, 1)
+        for j in range(len(projs)):
+            hy[j].copy_(ys[j], non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    h2d = sum(x.numel() * x.element_size() for x in hx)
+    d2h = sum(y.numel() * y.element_size() for y in hy)
+    return ms, h2d, d2h
+
+
+def time_prefill(w4, torch, M=4096, iters=5, warmup=3):
+    wl = workloads.workload(PREFILL_CFG)
+    res = []
+    for i, L in enumerate(wl.layers):
+        li = workloads.make_layer(wl, i, M=M)
+        W = dev_bits(li.W.view(np.uint16), torch.float16)
+        qw, sc, zr = w4.w4_quantize_pack(W, torch.from_numpy(li.s).cuda(), li.group_size)
+        X = dev_bits(li.X, torch.bfloat16)
+        Y = torch.empty(M, li.N, dtype=torch.bfloat16, device="cuda")
+        for _ in range(warmup):
+            w4.w4a16_gemm(X, qw, sc, zr, 128, Y=Y)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            w4.w4a16_gemm(X, qw, sc, zr, 128, Y=Y)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / iters
+        res.append({"layer": f"{L.name} {L.K}x{L.N}", "ms": ms,
+                    "tflops": workloads.gemm_flops(M, li.N, li.K) / ms / 1e9})
+    w4.w4_check_device_error()
+    tot_flop = sum(workloads.gemm_flops(M, L.N, L.K) for L in wl.layers)
+    tot_ms = sum(r["ms"] for r in res)
+    return {"M": M, "layers": res, "tflops": tot_flop / tot_ms / 1e9}
+
+
+def time_quantize(w4, torch, projs, iters=3):
+    l = max(projs, key=lambda x: x["bytes"])
+    li = l["li"]
+    for _ in range(2):
+        w4.w4_quantize_pack(l["W"], l["s"], 128)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        w4.w4_quantize_pack(l["W"], l["s"], 128)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / iters
+    read = li.N * li.K * 2 + li.K * 4
+    return {"layer": f"{li.K}x{li.N}", "ms": ms, "input_gbs": read / ms / 1e6}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(target_s=12.0, rows_per_layer=None):
+    """Time the oracle's online path (X*s_inv, dequantise, fp32 product) for M=1 on a
+    seeded sample of output rows of every decode layer; returns (GB/s of effective weight
+    bytes processed, seconds, description)."""
+    import oracle
+    wl = workloads.workload(DECODE_CFG)
+    rng = np.random.default_rng(0)
+    total_bytes, total_s, n_rows = 0, 0.0, 0
+    rows_per_layer = rows_per_layer or 256
+    for i, L in enumerate(wl.layers):
+        li = workloads.make_layer(wl, i, M=1, with_weights=False)
+        # a fresh seeded sample of rows (weights regenerated only for those rows)
+        ns = np.sort(rng.choice(L.N, size=rows_per_layer, replace=False))
+        Wr = workloads.gen_weights(L.N, L.K, 0, wl.config_id, i)[ns]
+        q, sc, zr = oracle.quantize_weights(Wr.view(np.uint16), li.s, 128)
+        t0 = time.perf_counter()
+        oracle.reference_y(li.X, li.s_inv, q, sc, zr, 128)
+        total_s += time.perf_counter() - t0
+        total_bytes += workloads.effective_weight_bytes(rows_per_layer, L.K, 128, False, False)
+        n_rows += rows_per_layer
+    desc = (f"M=1, {rows_per_layer} seeded output rows of each of the 4 layers "
+            f"({n_rows} rows, {total_bytes / 1e6:.1f} MB effective weights), single thread")
+    return total_bytes / total_s / 1e9, total_s, desc
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    oracle.lib()
+    vals = []
+    desc = ""
+    for _ in range(args.warmup):
+        cpu_oracle_sample(rows_per_layer=64)
+    for _ in range(args.steps):
+        v, s, desc = cpu_oracle_sample(rows_per_layer=256)
+        vals.append(v)
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": workload_desc(workloads.workload(DECODE_CFG), 1),
+                       "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def our_arm(args, world, rank, local):
+    import torch
+    import bit_weight_only_w4_b200 as w4
+    from bit_weight_only_w4_b200 import build as _build
+    if not os.path.exists(w4.LIB_PATH):
+        _build.build()
+    peaks, peak_src = load_peaks()
+    M = 1
+    wl, projs, step_bytes = prepare_weights(w4, torch)
+    clocks = ClockSampler(local)
+    dec = time_decode(M, args.steps, args.warmup, w4, torch, world, wl, projs, step_bytes,
+                      clocks, per_layer=True)
+    t_ms = max_over_ranks(dec["total_ms"], world)
+    value = world * args.steps * step_bytes / (t_ms * 1e-3) / 1e9
+    # dominant kernel = the decode GEMM (every launch of the timed region is one):
+    # achieved = algorithmic bytes per launch / average launch duration on its stream
+    achieved = args.steps * step_bytes / (dec["total_ms"] * 1e-3) / 1e9
+    e2e_ms, h2d, d2h = time_e2e(M, args.steps, args.warmup, w4, torch, world, wl, projs)
+    e2e_val = world * args.steps * step_bytes / (e2e_ms * 1e-3) / 1e9
+
+    extras = {"tokens_per_s_linear_layers": round(1e3 * args.steps / t_ms, 1)}
+    if not args.quick:
+        sweep = {"1": round(value / world, 1)}
+        for m in (2, 4, 8, 16):
+            st = max(3, args.steps // 4)
+            d = time_decode(m, st, args.warmup, w4, torch, world, wl, projs, step_bytes)
+            sweep[str(m)] = round(st * step_bytes / (max_over_ranks(d["total_ms"], world) * 1e-3)
+                                  / 1e9, 1)
+        extras["decode_sweep_gbs_per_gpu"] = sweep
+        pf = time_prefill(w4, torch)
+        pf["frac_of_measured_bf16_burst"] = pf["tflops"] / peaks["bf16_tflops"]
+        pf["frac_of_spec_2250"] = pf["tflops"] / 2250.0
+        extras["prefill_m4096"] = pf
+        extras["quantize_pack"] = time_quantize(w4, torch, projs)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v, sec, desc = cpu_oracle_sample()
+        cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+               "seconds": round(sec, 2)}
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get("bytes_per_launch")
+        except Exception:
+            traffic = None
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(wl, M) + f"; step = 1 token through {N_LAYERS} "
+                   f"blocks x 4 projections ({N_LAYERS * 4} GEMMs)",
+                   "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of packed weights "
+                         "per step (one copy per block)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "peak_source": peak_src, "kernel": "w4a16 decode (stream-K, mma.sync)",
+                     "per_layer": dec["per_layer"]},
+        "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": dec["launches"],
+        "clocks": dec["clocks"],
+        "cpu_baseline": cpu,
+    }
+    line.update(extras)
+    if rank == 0:
+        print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="skip the sweep / prefill extras")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            reference_arm(args, world, rank)
+        else:
+            our_arm(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,1 +1,233 @@
-"""W4A16 for B200: placeholder, replaced by the binding below."""
+"""B200 (sm_100a) W4A16: 4-bit weight-only quantised linear layers with 16-bit activations.
+
+Thin Python binding of the C ABI in include/w4a16.h.  The functions below carry the C
+names and only marshal arguments: PyTorch provides device memory, streams and output
+allocation; every step of the computation runs in the library's CUDA kernels
+(bit_weight_only_w4_b200/_lib/libw4a16.so, built in-tree by
+``python -m bit_weight_only_w4_b200.build``).  There is no CPU fallback: if the library
+is missing or a call fails, an exception is raised.
+
+    qweight, scales, zeros = w4_quantize_pack(W, s, group_size=128)
+    Y = w4a16_gemm(X, qweight, scales, zeros, group_size=128, s_inv=s_inv)
+"""
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libw4a16.so")
+
+W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA, W4_ERR_TIMEOUT, W4_ERR_DEVICE_ARG = range(6)
+W4_F16, W4_BF16, W4_F32 = 0, 1, 2
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+class W4Error(RuntimeError):
+    """A library call returned a status other than W4_OK."""
+
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {w4_status_string(status)}")
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"W4A16 CUDA library not found at {LIB_PATH}; build it with "
+                "`python -m bit_weight_only_w4_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, u64, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                                 ctypes.c_uint64, ctypes.c_size_t)
+        st = ctypes.c_int
+        L.w4_quantize_pack.argtypes = [vp, st, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp]
+        L.w4_quantize_pack.restype = st
+        L.w4a16_gemm.argtypes = [vp, st, i64, i64, i64, vp, vp, vp, vp, i32, vp, vp, st, vp, sz, vp]
+        L.w4a16_gemm.restype = st
+        L.w4a16_workspace_bytes.argtypes = [i64, i64, i64, i32]
+        L.w4a16_workspace_bytes.restype = sz
+        L.w4_unpack_canonical.argtypes = [vp, i64, i64, vp, vp]
+        L.w4_unpack_canonical.restype = st
+        L.w4_check_device_error.argtypes = []
+        L.w4_check_device_error.restype = st
+        L.w4_set_wait_limit_ns.argtypes = [u64]
+        L.w4_set_wait_limit_ns.restype = st
+        L.w4_selftest_expired_wait.argtypes = [vp]
+        L.w4_selftest_expired_wait.restype = st
+        L.w4_status_string.argtypes = [st]
+        L.w4_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- marshalling helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(dt):
+    torch = _torch()
+    if dt == torch.float16:
+        return W4_F16
+    if dt == torch.bfloat16:
+        return W4_BF16
+    if dt == torch.float32:
+        return W4_F32
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status, what):
+    if status != W4_OK:
+        raise W4Error(status, what)
+
+
+def _need_cuda(*tensors):
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("tensors are on different devices")
+    return dev
+
+
+class _DeviceGuard:
+    def __init__(self, device):
+        self.device = device
+
+    def __enter__(self):
+        torch = _torch()
+        self.prev = torch.cuda.current_device()
+        torch.cuda.set_device(self.device)
+
+    def __exit__(self, *exc):
+        _torch().cuda.set_device(self.prev)
+
+
+# ---------------------------------------------------------------- C ABI, same names
+def w4_status_string(status):
+    return lib().w4_status_string(int(status)).decode()
+
+
+def w4a16_workspace_bytes(M, N, K, group_size):
+    return int(lib().w4a16_workspace_bytes(int(M), int(N), int(K), int(group_size)))
+
+
+def w4_quantize_pack(W, s=None, group_size=128, symmetric=False, g_idx=None,
+                     qweight=None, scales=None, zeros=None, stream=None):
+    """AWQ scaling + group-wise RTN INT4 + packing of W [N,K] (fp16/bf16, CUDA).
+
+    Returns (qweight uint32-as-int32 [N*K/8] device layout, scales fp16 [G,N],
+    zeros fp16 [G,N] or None when symmetric)."""
+    torch = _torch()
+    N, K = W.shape
+    G = K // group_size
+    dev = _need_cuda(W, s, g_idx, qweight, scales, zeros)
+    if qweight is None:
+        qweight = torch.empty(N * K // 8, dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty(G, N, dtype=torch.float16, device=dev)
+    if zeros is None and not symmetric:
+        zeros = torch.empty(G, N, dtype=torch.float16, device=dev)
+    if s is not None and s.dtype != torch.float32:
+        raise TypeError("s must be float32")
+    if g_idx is not None and g_idx.dtype != torch.int32:
+        raise TypeError("g_idx must be int32")
+    with _DeviceGuard(dev):
+        st = lib().w4_quantize_pack(_ptr(W), _dtype_code(W.dtype), N, K, _ptr(s), int(group_size),
+                                    int(bool(symmetric)), _ptr(g_idx), _ptr(qweight),
+                                    _ptr(scales), _ptr(zeros), _stream_handle(stream, dev))
+    _check(st, "w4_quantize_pack")
+    return qweight, scales, zeros
+
+
+_ws_cache = {}
+_ws_lock = threading.Lock()
+
+
+def workspace_for(device, nbytes):
+    """A zero-initialised scratch buffer of at least nbytes on `device`, shared by calls
+    on one stream (the kernels leave it zero-filled where that matters)."""
+    torch = _torch()
+    key = torch.device(device).index
+    with _ws_lock:
+        buf = _ws_cache.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+            _ws_cache[key] = buf
+        return buf
+
+
+def w4a16_gemm(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None,
+               out_dtype=None, Y=None, workspace=None, stream=None):
+    """Y[M,N] = (X * s_inv)[M,K] @ dequant(qweight, scales, zeros, g_idx)^T on the GPU."""
+    torch = _torch()
+    M, K = X.shape
+    N = scales.shape[1]
+    dev = _need_cuda(X, qweight, scales, zeros, g_idx, s_inv, Y, workspace)
+    out_dtype = out_dtype or X.dtype
+    if Y is None:
+        Y = torch.empty(M, N, dtype=out_dtype, device=dev)
+    with _DeviceGuard(dev):
+        need = w4a16_workspace_bytes(M, N, K, group_size) if M > 0 else 0
+        if workspace is None and need > 0:
+            workspace = workspace_for(dev, need)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib().w4a16_gemm(_ptr(X), _dtype_code(X.dtype), M, N, K, _ptr(qweight), _ptr(scales),
+                              _ptr(zeros), _ptr(g_idx), int(group_size), _ptr(s_inv), _ptr(Y),
+                              _dtype_code(Y.dtype), _ptr(workspace), ws_bytes,
+                              _stream_handle(stream, dev))
+    _check(st, "w4a16_gemm")
+    return Y
+
+
+def w4_unpack_canonical(qweight, N, K, out=None, stream=None):
+    torch = _torch()
+    dev = _need_cuda(qweight, out)
+    if out is None:
+        out = torch.empty(N, K // 8, dtype=torch.int32, device=dev)
+    with _DeviceGuard(dev):
+        st = lib().w4_unpack_canonical(_ptr(qweight), int(N), int(K), _ptr(out),
+                                       _stream_handle(stream, dev))
+    _check(st, "w4_unpack_canonical")
+    return out
+
+
+def w4_check_device_error():
+    st = lib().w4_check_device_error()
+    _check(st, "w4_check_device_error")
+
+
+def w4_set_wait_limit_ns(ns):
+    _check(lib().w4_set_wait_limit_ns(int(ns)), "w4_set_wait_limit_ns")
+
+
+def w4_selftest_expired_wait(stream=None):
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib().w4_selftest_expired_wait(_stream_handle(stream, dev)), "w4_selftest_expired_wait")

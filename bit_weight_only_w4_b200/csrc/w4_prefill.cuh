@@ -1,0 +1,397 @@
+// w4_prefill.cuh -- compute-bound W4A16 kernel for large M (prefill) on the 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// Prefill multiplies many tokens by every weight and is limited by tensor-core
+// throughput (edgesiliconlab.com article on AWQ vs GPTQ, "The Mathematics of Memory
+// Bandwidth Saturation"); weights are unpacked with AND/OR bit tricks right before the
+// tensor cores and the next tiles are staged while the current ones are multiplied
+// ("Kernel Execution: Marlin vs. ExLlamaV2 INT4 GEMM Micro-Architecture", items 1-3).
+//
+// One CTA computes a 128 (output rows) x 128 (tokens) tile of Y^T = What * X'^T:
+//   warp 0      TMA: activation tile (2-D tensor map, 128B swizzle) + packed weight tiles
+//               (1-D bulk copies) into a 4-stage ring;
+//   warp 1      allocates tensor memory and issues tcgen05.mma (one thread): A = the
+//               dequantised weights (128 x 64 per stage, K-major, 128B swizzle, shared
+//               memory), B = the activations, D = fp32 in tensor memory;
+//   warps 2-5   unpack the packed tile into exact integers q - z (fp16/bf16) in the
+//               swizzled A layout;
+//   warps 6-9   epilogue: after each quantisation group the MMA warp hands over that
+//               group's fp32 partial tile (two tensor-memory buffers, ping-pong); each
+//               thread owns one output row, multiplies the partial by the row's group
+//               scale and adds it to register accumulators; at the end it stores Y.
+// With act-order g_idx the scale is folded into fp16 weights instead and the whole K
+// accumulates in one tensor-memory buffer.
+#pragma once
+#include "w4_common.cuh"
+
+namespace w4p {
+
+constexpr int BN = 128;        // output rows per CTA (MMA M)
+constexpr int BM = 128;        // tokens per CTA (MMA N)
+constexpr int BK = 64;         // input channels per stage (one 128-byte swizzle row)
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kTmemCols = 256; // two fp32 partial buffers of BM columns
+
+constexpr int kABytes = BN * BK * 2;   // 16 KB
+constexpr int kBBytes = BM * BK * 2;   // 16 KB
+constexpr int kPBytes = BN * BK / 2;   // 4 KB packed codes
+constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+
+struct SmemLayout {
+    static constexpr int a = 0;                              // kStages x 16 KB (1024-aligned)
+    static constexpr int b = a + kStages * kABytes;          // kStages x 16 KB
+    static constexpr int pk = b + kStages * kBBytes;         // kStages x 4 KB
+    static constexpr int bars = pk + kStages * kPBytes;      // barriers
+    static constexpr int nbars = 3 * kStages + 4 + 1;
+    static constexpr int tmem_slot = bars + nbars * 8;
+    static constexpr int flags = tmem_slot + 8;
+    static constexpr int bytes = flags + 16 + 1024;          // + alignment slack
+};
+
+struct PrefillParams {
+    const uint32_t* qw;
+    const __half* scales;
+    const __half* zeros;
+    const int32_t* g_idx;
+    void* Y;
+    int M, N, K, group_size, G, out_dtype;
+    int KA;       // K / 64
+    int tiles;    // N / 16
+};
+
+// ---------------------------------------------------------------- tcgen05 wrappers
+W4_DEV void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+W4_DEV void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+W4_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+W4_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+W4_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+W4_DEV void tc_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (fp16 or bf16 in, fp32 out)
+W4_DEV void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                   uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns: thread i of the warp gets its lane's 32 values.
+W4_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major tile whose rows are 128-byte swizzled lines,
+// 8-row groups 1024 bytes apart (the layout TMA writes with 128B swizzle).
+W4_DEV uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
+    d |= (uint64_t)1u << 16;                           // leading byte offset (unused here)
+    d |= (uint64_t)(1024u >> 4) << 32;                 // stride byte offset: 8 rows
+    d |= (uint64_t)1u << 46;                           // descriptor version
+    d |= (uint64_t)2u << 61;                           // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: fp32 accumulator, A/B fp16 (0) or bf16 (1), both K-major,
+// N = BM, M = BN.
+W4_DEV uint32_t mma_idesc(bool bf16) {
+    const uint32_t fmt = bf16 ? 1u : 0u;
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(BM >> 3) << 17) |
+           ((uint32_t)(BN >> 4) << 24);
+}
+
+// byte offset of element (row, k) in a 128B-swizzled K-major tile (k < 64, 2-byte elems)
+W4_DEV uint32_t sw128_off(int row, int k) {
+    return (uint32_t)(row * 128 + ((((k >> 3) ^ (row & 7)) & 7) << 4) + ((k & 7) << 1));
+}
+
+W4_DEV void store_out(const PrefillParams& p, int m, int n, float v) {
+    const size_t idx = (size_t)m * p.N + n;
+    if (p.out_dtype == 2) reinterpret_cast<float*>(p.Y)[idx] = v;
+    else if (p.out_dtype == 1) reinterpret_cast<__nv_bfloat16*>(p.Y)[idx] = __float2bfloat16_rn(v);
+    else reinterpret_cast<__half*>(p.Y)[idx] = __float2half_rn(v);
+}
+
+// bounded wait that also honours the CTA's abort flag
+W4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *abort_flag = 1;
+    return false;
+}
+
+template <bool BF16, bool GIDX>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const PrefillParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    // 1024-byte alignment for the swizzled operand tiles
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    using L = SmemLayout;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::bars);
+    uint64_t* deq = full + kStages;
+    uint64_t* empty = deq + kStages;
+    uint64_t* pfull = empty + kStages;       // [2]
+    uint64_t* pempty = pfull + 2;            // [2]
+    uint64_t* mma_done = pempty + 2;         // [1]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::flags);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN;       // first output row of the tile
+    const int m0 = blockIdx.y * BM;       // first token of the tile
+    const int KT = p.K / BK;              // stages along K
+    const int g = p.group_size;
+    const int ngroups = GIDX ? 1 : p.K / g;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&deq[s], 128);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&pfull[b], 1);
+            mbar_init(&pempty[b], 128);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_x);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const int tiles = min(BN / 16, p.tiles - n0 / 16);
+            const uint32_t bytes = kBBytes + tiles * 512;
+            int issued = 0;
+            for (int kt = 0; kt < KT; ++kt, ++issued) {
+                const int s = kt % kStages, ph = (kt / kStages) & 1;
+                if (kt >= kStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
+                mbar_arrive_expect_tx(&full[s], bytes);
+                tma_load_2d(smem + L::b + s * kBBytes, &tmap_x, kt * BK, m0, &full[s]);
+                for (int t = 0; t < tiles; ++t)
+                    bulk_g2s(smem + L::pk + s * kPBytes + t * 512,
+                             p.qw + ((size_t)(n0 / 16 + t) * p.KA + kt) * 128, 512, &full[s]);
+            }
+            if (*abort_flag)
+                for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+                    (void)mbar_wait(&full[i % kStages], (i / kStages) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = mma_idesc(BF16 && !GIDX);
+            int grp_i = -1, pb = 0;
+            bool ok = true;
+            for (int kt = 0; kt < KT && ok; ++kt) {
+                const int s = kt % kStages, ph = (kt / kStages) & 1;
+                ok = wait_or_abort(&full[s], ph, abort_flag) &&
+                     wait_or_abort(&deq[s], ph, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(smem + L::a + s * kABytes);
+                const uint32_t b_base = smem_u32(smem + L::b + s * kBBytes);
+#pragma unroll
+                for (int j = 0; j < BK / 16; ++j) {
+                    const int kabs = kt * BK + 16 * j;
+                    bool first, last;
+                    if (GIDX) {
+                        first = (kabs == 0);
+                        last = (kabs + 16 == p.K);
+                    } else {
+                        first = (kabs % g) == 0;
+                        last = ((kabs + 16) % g) == 0;
+                    }
+                    if (first) {
+                        ++grp_i;
+                        pb = grp_i & 1;
+                        if (grp_i >= 2) {
+                            ok = wait_or_abort(&pempty[pb], ((grp_i >> 1) - 1) & 1, abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                    }
+                    tc_mma(tmem_base + (uint32_t)(pb * BM), sw128_desc(a_base + 32 * j),
+                           sw128_desc(b_base + 32 * j), idesc, first ? 0u : 1u);
+                    if (last) tc_commit(&pfull[pb]);
+                }
+                if (!ok) break;
+                tc_commit(&empty[s]);
+            }
+            // every MMA this thread issued has finished once mma_done completes
+            tc_commit(mma_done);
+            (void)mbar_wait(mma_done, 0);
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ dequant warps
+        const int dq = warp - 2;                 // handles row tiles 2dq, 2dq+1
+        const int gq = lane >> 2, c = 2 * (lane & 3);
+        for (int kt = 0; kt < KT; ++kt) {
+            const int s = kt % kStages, ph = (kt / kStages) & 1;
+            if (!wait_or_abort(&full[s], ph, abort_flag)) break;
+            unsigned char* a_tile = smem + L::a + s * kABytes;
+            const unsigned char* pk = smem + L::pk + s * kPBytes;
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                const int t = 2 * dq + tt;
+                if (n0 / 16 + t >= p.tiles) continue;
+                const uint4 wq = *reinterpret_cast<const uint4*>(pk + t * 512 + lane * 16);
+                const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+                const int r0 = 16 * t + gq, r1 = r0 + 8;       // rows within the tile
+                const int nr0 = n0 + r0, nr1 = n0 + r1;        // output rows
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int kk = 16 * j + c;                 // column within the stage
+                    const int kabs = kt * BK + kk;
+                    uint32_t af[4];
+                    if constexpr (!GIDX) {
+                        const int grp = kabs / g;
+                        float z0 = 8.0f, z1 = 8.0f;
+                        if (p.zeros) {
+                            z0 = __half2float(__ldg(p.zeros + (size_t)grp * p.N + nr0));
+                            z1 = __half2float(__ldg(p.zeros + (size_t)grp * p.N + nr1));
+                        }
+                        const ZeroConsts zc = BF16 ? zero_consts_bf16(z0, z1) : zero_consts_f16(z0, z1);
+                        unpack_word<BF16>(wv[j], zc, af);
+                    } else {
+                        int gk[4] = {__ldg(p.g_idx + kabs), __ldg(p.g_idx + kabs + 1),
+                                     __ldg(p.g_idx + kabs + 8), __ldg(p.g_idx + kabs + 9)};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (gk[e] < 0 || gk[e] >= p.G) {
+                                atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
+                                gk[e] = 0;
+                            }
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int row = (r & 1) ? nr1 : nr0;
+                            const int kl = (r & 2) ? 2 : 0;
+                            const float qlo = (float)((wv[j] >> (4 * r)) & 0xF);
+                            const float qhi = (float)((wv[j] >> (4 * (r + 4))) & 0xF);
+                            const __half z_lo = p.zeros ? __ldg(p.zeros + (size_t)gk[kl] * p.N + row)
+                                                        : __float2half_rn(8.0f);
+                            const __half z_hi = p.zeros ? __ldg(p.zeros + (size_t)gk[kl + 1] * p.N + row)
+                                                        : __float2half_rn(8.0f);
+                            const __half2 ss = __halves2half2(__ldg(p.scales + (size_t)gk[kl] * p.N + row),
+                                                              __ldg(p.scales + (size_t)gk[kl + 1] * p.N + row));
+                            af[r] = h2_as_u32(__hmul2(
+                                __hsub2(__floats2half2_rn(qlo, qhi), __halves2half2(z_lo, z_hi)), ss));
+                        }
+                    }
+                    *reinterpret_cast<uint32_t*>(a_tile + sw128_off(r0, kk)) = af[0];
+                    *reinterpret_cast<uint32_t*>(a_tile + sw128_off(r1, kk)) = af[1];
+                    *reinterpret_cast<uint32_t*>(a_tile + sw128_off(r0, kk + 8)) = af[2];
+                    *reinterpret_cast<uint32_t*>(a_tile + sw128_off(r1, kk + 8)) = af[3];
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&deq[s]);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue warps
+        const int quad = warp & 3;                 // tensor-memory lanes 32*quad..
+        const int row = 32 * quad + lane;          // output row within the tile
+        const int n = n0 + row;
+        const bool row_ok = n < p.N;
+        float acc[BM];
+#pragma unroll
+        for (int i = 0; i < BM; ++i) acc[i] = 0.0f;
+        bool ok = true;
+        for (int grp_i = 0; grp_i < ngroups && ok; ++grp_i) {
+            const int pb = grp_i & 1;
+            float sc = 1.0f;
+            if (!GIDX && row_ok) sc = __half2float(__ldg(p.scales + (size_t)grp_i * p.N + n));
+            ok = wait_or_abort(&pfull[pb], (grp_i >> 1) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(pb * BM);
+#pragma unroll
+            for (int ch = 0; ch < BM / 32; ++ch) {
+                float v[32];
+                tmem_ld32(taddr + 32 * ch, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[32 * ch + i] = fmaf(sc, v[i], acc[32 * ch + i]);
+            }
+            tc_fence_before();
+            mbar_arrive(&pempty[pb]);
+        }
+        if (ok && row_ok) {
+#pragma unroll
+            for (int i = 0; i < BM; ++i)
+                if (m0 + i < p.M) store_out(p, m0 + i, n, acc[i]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// X'[m,k] = X[m,k] * s_inv[k], rounded to the activation type (for the prefill path,
+// whose activations reach the tensor cores straight from TMA).
+template <bool BF16>
+__global__ void scale_acts_kernel(const void* __restrict__ X, const float* __restrict__ s_inv,
+                                  void* __restrict__ Xp, int M, int K) {
+    const size_t pairs = (size_t)M * K / 2;
+    const uint32_t* xin = reinterpret_cast<const uint32_t*>(X);
+    uint32_t* xout = reinterpret_cast<uint32_t*>(Xp);
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < pairs;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const int k = (int)((2 * i) % K);
+        const float2 v = unpack2<BF16>(xin[i]);
+        const float2 s = *reinterpret_cast<const float2*>(s_inv + k);
+        xout[i] = pack2<BF16>(__fmul_rn(v.x, s.x), __fmul_rn(v.y, s.y));
+    }
+}
+
+}  // namespace w4p

@@ -1,0 +1,372 @@
+// w4a16.cu -- C ABI of the W4A16 library (declared in include/w4a16.h): argument
+// validation, kernel selection by M and launches.  All device work is in the kernels of
+// w4_quant.cuh, w4_decode.cuh and w4_prefill.cuh; nothing here touches tensor data.
+#include <climits>
+#include <cstring>
+#include <mutex>
+
+#include "w4a16.h"
+#include "w4_common.cuh"
+#include "w4_decode.cuh"
+#include "w4_prefill.cuh"
+#include "w4_quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kDecodeMaxM = 64;
+constexpr int kDecodeMaxCtasPerSm = 2;
+constexpr int kQuantMaxGroups = 1536;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+cudaStream_t as_stream(w4_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+w4_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+// Shape rules shared by quantisation and GEMM.
+w4_status check_layer_shape(int64_t N, int64_t K, int32_t group_size) {
+    if (N <= 0 || K <= 0 || group_size <= 0) return W4_ERR_INVALID_ARG;
+    if (N > INT_MAX / 2 || K > INT_MAX / 2) return W4_ERR_UNSUPPORTED;
+    if (K % group_size != 0) return W4_ERR_INVALID_ARG;
+    if (N % 16 != 0 || K % 64 != 0) return W4_ERR_UNSUPPORTED;
+    if (group_size != 32 && group_size % 64 != 0) return W4_ERR_UNSUPPORTED;
+    return W4_OK;
+}
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+int sm_count(int dev) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return v;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename Kernel>
+bool ensure_smem(Kernel k, int bytes, std::once_flag (&flags)[kMaxDevices], int dev) {
+    if (bytes <= 48 * 1024) return true;
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    bool ok = true;
+    std::call_once(flags[dev], [&] {
+        ok = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+             cudaSuccess;
+    });
+    // a failed first attempt is retried on the next call by the launch itself failing
+    return ok;
+}
+
+// ---------------------------------------------------------------- decode launch plan
+int decode_tiles_for(int64_t M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
+
+template <int NT, bool BF16, bool GIDX>
+struct DecodeKernel {
+    static constexpr int smem = w4d::SmemLayout<NT>::bytes;
+    static int ctas_per_sm[kMaxDevices];
+    static std::once_flag occ_flags[kMaxDevices];
+    static int occupancy(int dev) {
+        std::call_once(occ_flags[dev], [&] {
+            int b = 0;
+            cudaFuncSetAttribute(w4d::decode_kernel<NT, BF16, GIDX>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &b, w4d::decode_kernel<NT, BF16, GIDX>, w4d::kThreads, smem) != cudaSuccess)
+                b = 1;
+            ctas_per_sm[dev] = b < 1 ? 1 : (b > kDecodeMaxCtasPerSm ? kDecodeMaxCtasPerSm : b);
+        });
+        return ctas_per_sm[dev];
+    }
+};
+template <int NT, bool BF16, bool GIDX>
+int DecodeKernel<NT, BF16, GIDX>::ctas_per_sm[kMaxDevices];
+template <int NT, bool BF16, bool GIDX>
+std::once_flag DecodeKernel<NT, BF16, GIDX>::occ_flags[kMaxDevices];
+
+size_t decode_counter_bytes(int64_t N) {
+    const int64_t bands = (N / 16 + w4d::kWarps - 1) / w4d::kWarps;
+    return (size_t)((bands * 4 + 255) / 256 * 256);
+}
+
+size_t decode_workspace_bytes(int64_t M, int64_t N, int sms) {
+    const int Mp = 8 * decode_tiles_for(M);
+    const size_t partials = (size_t)sms * kDecodeMaxCtasPerSm * 2 * w4d::kBandRows * Mp * 4;
+    return decode_counter_bytes(N) + partials;
+}
+
+template <int NT, bool BF16, bool GIDX>
+w4_status launch_decode(w4d::DecodeParams p, unsigned char* ws, int dev, cudaStream_t stream) {
+    using DK = DecodeKernel<NT, BF16, GIDX>;
+    const int per_sm = DK::occupancy(dev);
+    const int bands = (p.tiles + w4d::kWarps - 1) / w4d::kWarps;
+    p.units = bands * p.KA;
+    int P = sm_count(dev) * per_sm;
+    if (P <= 0) return W4_ERR_CUDA;
+    if (P > p.units) P = p.units;
+    p.base = p.units / P;
+    p.rem = p.units % P;
+    p.counters = reinterpret_cast<unsigned*>(ws);
+    p.partials = reinterpret_cast<float*>(ws + decode_counter_bytes(p.N));
+    w4d::decode_kernel<NT, BF16, GIDX><<<P, w4d::kThreads, DK::smem, stream>>>(p);
+    return launch_status();
+}
+
+template <bool BF16, bool GIDX>
+w4_status dispatch_decode(w4d::DecodeParams p, unsigned char* ws, int dev, cudaStream_t s) {
+    switch (decode_tiles_for(p.M)) {
+        case 1: return launch_decode<1, BF16, GIDX>(p, ws, dev, s);
+        case 2: return launch_decode<2, BF16, GIDX>(p, ws, dev, s);
+        case 4: return launch_decode<4, BF16, GIDX>(p, ws, dev, s);
+        default: return launch_decode<8, BF16, GIDX>(p, ws, dev, s);
+    }
+}
+
+// ---------------------------------------------------------------- prefill launch plan
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+bool make_act_tensor_map(CUtensorMap* map, const void* X, bool bf16, int64_t M, int64_t K) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)w4p::BK, (cuuint32_t)w4p::BM};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+               const_cast<void*>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool BF16, bool GIDX>
+w4_status launch_prefill(const CUtensorMap& map, const w4p::PrefillParams& p, int dev,
+                         cudaStream_t stream) {
+    static std::once_flag flags[kMaxDevices];
+    auto k = w4p::prefill_kernel<BF16, GIDX>;
+    if (!ensure_smem(k, w4p::SmemLayout::bytes, flags, dev)) return W4_ERR_CUDA;
+    const dim3 grid((unsigned)((p.N + w4p::BN - 1) / w4p::BN), (unsigned)((p.M + w4p::BM - 1) / w4p::BM));
+    k<<<grid, w4p::kThreads, w4p::SmemLayout::bytes, stream>>>(map, p);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* w4_status_string(w4_status s) {
+    switch (s) {
+        case W4_OK: return "W4_OK";
+        case W4_ERR_INVALID_ARG: return "W4_ERR_INVALID_ARG";
+        case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED";
+        case W4_ERR_CUDA: return "W4_ERR_CUDA";
+        case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT";
+        case W4_ERR_DEVICE_ARG: return "W4_ERR_DEVICE_ARG";
+    }
+    return "W4_ERR_UNKNOWN";
+}
+
+w4_status w4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, const float* s,
+                           int32_t group_size, int32_t symmetric, const int32_t* g_idx,
+                           uint32_t* qweight, void* scales, void* zeros, w4_stream_t stream) {
+    if (!W || !qweight || !scales) return W4_ERR_INVALID_ARG;
+    if (w_dtype != W4_F16 && w_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
+    if (symmetric != 0 && symmetric != 1) return W4_ERR_INVALID_ARG;
+    if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return W4_ERR_INVALID_ARG;
+    if (!aligned(W, 2) || !aligned(qweight, 4) || !aligned(scales, 2) || !aligned(zeros, 2) ||
+        !aligned(s, 4) || !aligned(g_idx, 4))
+        return W4_ERR_INVALID_ARG;
+    w4_status st = check_layer_shape(N, K, group_size);
+    if (st != W4_OK) return st;
+    const int64_t G = K / group_size;
+    if (G > kQuantMaxGroups) return W4_ERR_UNSUPPORTED;
+
+    w4q::QuantParams p;
+    p.W = W;
+    p.s = s;
+    p.g_idx = g_idx;
+    p.qweight = qweight;
+    p.scales = reinterpret_cast<__half*>(scales);
+    p.zeros = reinterpret_cast<__half*>(zeros);
+    p.N = (int)N;
+    p.K = (int)K;
+    p.group_size = group_size;
+    p.G = (int)G;
+    p.symmetric = symmetric;
+    const int smem = (int)(2 * w4q::kRows * G * sizeof(int));
+    const int dev = current_device();
+    if (w_dtype == W4_BF16) {
+        static std::once_flag flags[kMaxDevices];
+        if (!ensure_smem(w4q::quantize_pack_kernel<true>, 2 * w4q::kRows * kQuantMaxGroups * 4, flags, dev))
+            return W4_ERR_CUDA;
+        w4q::quantize_pack_kernel<true><<<(unsigned)(N / 16), w4q::kThreads, smem, as_stream(stream)>>>(p);
+    } else {
+        static std::once_flag flags[kMaxDevices];
+        if (!ensure_smem(w4q::quantize_pack_kernel<false>, 2 * w4q::kRows * kQuantMaxGroups * 4, flags, dev))
+            return W4_ERR_CUDA;
+        w4q::quantize_pack_kernel<false><<<(unsigned)(N / 16), w4q::kThreads, smem, as_stream(stream)>>>(p);
+    }
+    return launch_status();
+}
+
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size) {
+    if (M < 0 || check_layer_shape(N, K, group_size) != W4_OK) return 0;
+    if (M == 0) return 0;
+    const int dev = current_device();
+    const int sms = dev >= 0 ? sm_count(dev) : 0;
+    if (sms <= 0) return 0;
+    if (M <= kDecodeMaxM) return decode_workspace_bytes(M, N, sms);
+    return (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
+}
+
+w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                     const uint32_t* qweight, const void* scales, const void* zeros,
+                     const int32_t* g_idx, int32_t group_size, const float* s_inv, void* Y,
+                     w4_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                     w4_stream_t stream) {
+    if (M < 0) return W4_ERR_INVALID_ARG;
+    if (act_dtype != W4_F16 && act_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
+    if (out_dtype != W4_F16 && out_dtype != W4_BF16 && out_dtype != W4_F32) return W4_ERR_INVALID_ARG;
+    w4_status st = check_layer_shape(N, K, group_size);
+    if (st != W4_OK) return st;
+    if (M == 0) return W4_OK;
+    if (M > INT_MAX / 2 || (size_t)M * (size_t)K > (size_t)INT_MAX * 8) return W4_ERR_UNSUPPORTED;
+    if (!X || !qweight || !scales || !Y) return W4_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(zeros, 16) ||
+        !aligned(g_idx, 16) || !aligned(s_inv, 16) || !aligned(Y, 16) || !aligned(workspace, 256))
+        return W4_ERR_INVALID_ARG;
+    const bool bf16 = act_dtype == W4_BF16;
+    const bool gidx = g_idx != nullptr;
+    if (bf16 && gidx) return W4_ERR_UNSUPPORTED;
+    const size_t need = w4a16_workspace_bytes(M, N, K, group_size);
+    if (need == 0) return W4_ERR_CUDA;
+    const bool prefill = M > kDecodeMaxM;
+    const bool needs_ws = !prefill || s_inv != nullptr;
+    if (needs_ws && (!workspace || workspace_bytes < need)) return W4_ERR_INVALID_ARG;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    cudaStream_t strm = as_stream(stream);
+
+    if (!prefill) {
+        w4d::DecodeParams p;
+        std::memset(&p, 0, sizeof(p));
+        p.X = X;
+        p.qw = qweight;
+        p.scales = reinterpret_cast<const __half*>(scales);
+        p.zeros = reinterpret_cast<const __half*>(zeros);
+        p.g_idx = g_idx;
+        p.s_inv = s_inv;
+        p.Y = Y;
+        p.M = (int)M;
+        p.N = (int)N;
+        p.K = (int)K;
+        p.group_size = group_size;
+        p.G = (int)(K / group_size);
+        p.out_dtype = (int)out_dtype;
+        p.KA = (int)(K / 64);
+        p.tiles = (int)(N / 16);
+        unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+        if (bf16) return dispatch_decode<true, false>(p, ws, dev, strm);
+        return gidx ? dispatch_decode<false, true>(p, ws, dev, strm)
+                    : dispatch_decode<false, false>(p, ws, dev, strm);
+    }
+
+    const void* Xeff = X;
+    if (s_inv) {
+        const size_t pairs = (size_t)M * (size_t)K / 2;
+        const unsigned blocks = (unsigned)((pairs + 255) / 256 < 65535 * 8 ? (pairs + 255) / 256 : 65535 * 8);
+        if (bf16) w4p::scale_acts_kernel<true><<<blocks, 256, 0, strm>>>(X, s_inv, workspace, (int)M, (int)K);
+        else w4p::scale_acts_kernel<false><<<blocks, 256, 0, strm>>>(X, s_inv, workspace, (int)M, (int)K);
+        if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+        Xeff = workspace;
+    }
+    CUtensorMap map;
+    if (!make_act_tensor_map(&map, Xeff, bf16, M, K)) return W4_ERR_CUDA;
+    w4p::PrefillParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.qw = qweight;
+    p.scales = reinterpret_cast<const __half*>(scales);
+    p.zeros = reinterpret_cast<const __half*>(zeros);
+    p.g_idx = g_idx;
+    p.Y = Y;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.group_size = group_size;
+    p.G = (int)(K / group_size);
+    p.out_dtype = (int)out_dtype;
+    p.KA = (int)(K / 64);
+    p.tiles = (int)(N / 16);
+    if (bf16) return launch_prefill<true, false>(map, p, dev, strm);
+    return gidx ? launch_prefill<false, true>(map, p, dev, strm)
+                : launch_prefill<false, false>(map, p, dev, strm);
+}
+
+w4_status w4_unpack_canonical(const uint32_t* qweight, int64_t N, int64_t K,
+                              uint32_t* qweight_canonical, w4_stream_t stream) {
+    if (!qweight || !qweight_canonical) return W4_ERR_INVALID_ARG;
+    if (!aligned(qweight, 4) || !aligned(qweight_canonical, 4)) return W4_ERR_INVALID_ARG;
+    w4_status st = check_layer_shape(N, K, 64);
+    if (st != W4_OK) return st;
+    const size_t total = (size_t)N * (size_t)(K / 8);
+    const unsigned blocks = (unsigned)((total + 255) / 256 < 65535 * 16 ? (total + 255) / 256 : 65535 * 16);
+    w4q::unpack_canonical_kernel<<<blocks, 256, 0, as_stream(stream)>>>(qweight, (int)N, (int)K,
+                                                                       qweight_canonical);
+    return launch_status();
+}
+
+w4_status w4_check_device_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return W4_ERR_CUDA;
+    unsigned word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_w4_error_word, sizeof(word)) != cudaSuccess) return W4_ERR_CUDA;
+    if (word != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_w4_error_word, &zero, sizeof(zero)) != cudaSuccess) return W4_ERR_CUDA;
+    }
+    if (word & W4_DEVERR_TIMEOUT) return W4_ERR_TIMEOUT;
+    if (word & W4_DEVERR_GIDX) return W4_ERR_DEVICE_ARG;
+    return W4_OK;
+}
+
+w4_status w4_set_wait_limit_ns(uint64_t ns) {
+    unsigned long long v = ns < 1000 ? 1000ull : (unsigned long long)ns;
+    return cudaMemcpyToSymbol(g_w4_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+// One thread waits on a barrier nothing will complete; the bounded wait expires.
+__global__ void expired_wait_kernel() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        (void)mbar_wait(&bar, 0);
+    }
+}
+}  // namespace
+
+extern "C" w4_status w4_selftest_expired_wait(w4_stream_t stream) {
+    expired_wait_kernel<<<1, 32, 0, as_stream(stream)>>>();
+    return launch_status();
+}

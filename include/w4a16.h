@@ -1,0 +1,171 @@
+/*
+ * w4a16.h -- C ABI of the B200 (sm_100a) W4A16 library: 4-bit weight-only quantised
+ * linear layers with 16-bit activations.
+ *
+ * The method (page title, section):
+ *  - AWQ equivalence transform: "Quantization Paradigms for Edge Inference: AWQ, GPTQ,
+ *    and FP8 Matrix Cores", sec. 3 "The Math Behind Activation-Aware Protection (AWQ)",
+ *    eq. 1: W' = W diag(s), X' = diag(s)^-1 X, so W'X' = WX.  Salient input channels
+ *    are scaled up in the weights and down in the activations instead of being kept in
+ *    fp16 (edgesiliconlab.com article on AWQ vs GPTQ, "What Is the Core Difference
+ *    Between AWQ and GPTQ Quantization?").
+ *  - Group-wise asymmetric round-to-nearest INT4 with per-group scales and zero points:
+ *    "The Ultimate Guide to Quantized LLMs: GPTQ", "Understanding Quantized Model
+ *    Compression"; edgesiliconlab.com article, "Quantization on Non-NVIDIA Silicon".
+ *  - Two 4-bit weights per byte, unpacked with shift/AND to 16-bit just before the
+ *    tensor cores, with staged, double-buffered weight tiles: edgesiliconlab.com
+ *    article, "Kernel Execution: Marlin vs. ExLlamaV2 INT4 GEMM Micro-Architecture",
+ *    items 1-3.  Decode reads every weight once and is bandwidth-bound, prefill is
+ *    compute-bound: same article, "The Mathematics of Memory Bandwidth Saturation".
+ *
+ * Conventions shared by every entry point
+ *  - All pointers named as "device" are CUDA device (or managed) pointers of the
+ *    current device; the caller owns every buffer and keeps it alive until the work
+ *    on `stream` has finished.  The library never allocates device memory.
+ *  - Calls are asynchronous and stream-ordered on `stream` (NULL = legacy default
+ *    stream).  Arguments are validated on the host before any launch; the returned
+ *    status is synchronous.  W4_ERR_CUDA means a launch failed (cudaGetLastError).
+ *  - Kernels never trap.  Every wait inside a kernel is bounded; on expiry the kernel
+ *    records a device-side error word and returns.  w4_check_device_error() reads it.
+ *  - No C++ exception crosses this ABI.  The library keeps no per-call host state, so
+ *    calls from several host threads on different streams are safe.
+ *  - Shapes: N % 16 == 0, K % 64 == 0, group_size == 32 or a multiple of 64, and
+ *    K % group_size == 0 (group_size == K is per-channel).  Pointers to packed weights,
+ *    activations, outputs and fp16 metadata must be 16-byte aligned.
+ *
+ * Packed weight format ("device layout")
+ *  The INT4 codes q[n][k] in [0,15] of W [N,K] are stored as N*K/8 uint32 words in
+ *  tiles of 16 rows x 64 columns.  Tile (t, a) -- rows 16t..16t+15, columns
+ *  64a..64a+63 -- occupies the 128 words starting at word 128*(t*(K/64) + a).  Word
+ *  4L+j of a tile (L = 0..31, j = 0..3) holds, with r0 = 16t + L/4, r1 = r0 + 8,
+ *  kb = 64a + 16j, c = 2*(L%4), nibble i in bits 4i..4i+3:
+ *     nibble 0: q[r0][kb+c]     nibble 4: q[r0][kb+c+1]
+ *     nibble 1: q[r1][kb+c]     nibble 5: q[r1][kb+c+1]
+ *     nibble 2: q[r0][kb+c+8]   nibble 6: q[r0][kb+c+9]
+ *     nibble 3: q[r1][kb+c+8]   nibble 7: q[r1][kb+c+9]
+ *  Lane L of a warp loads words 4L..4L+3 of a tile with one 16-byte load; each word is
+ *  then exactly the 16x16 weight operand slice that lane needs for one 16-deep step of
+ *  a warp-level MMA, and the eight codes come out as fp16/bf16 pairs with one
+ *  AND/OR per pair (the exponent-bias trick) plus one subtract.
+ *  The "canonical layout" (w4_unpack_canonical) is uint32 [N, K/8] with nibble j of
+ *  word i of row n equal to q[n][8i+j].
+ *
+ *  scales: fp16 [G, N] (G = K/group_size), scale of group g of output row n at
+ *          scales[g*N + n].  zeros: fp16 [G, N] holding the integer zero point z in
+ *          [0,15]; NULL means the symmetric format with implicit z = 8.
+ *  Dequantised weight: (q - z) * scale.
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* w4_stream_t;
+
+typedef enum {
+    W4_OK = 0,
+    W4_ERR_INVALID_ARG = 1, /* NULL / misaligned pointer, negative or inconsistent size */
+    W4_ERR_UNSUPPORTED = 2, /* legal but not tiled: see the shape rules above          */
+    W4_ERR_CUDA = 3,        /* a CUDA call or kernel launch failed                      */
+    W4_ERR_TIMEOUT = 4,     /* a kernel gave up a bounded wait (device error word)      */
+    W4_ERR_DEVICE_ARG = 5   /* a kernel found an out-of-range g_idx entry               */
+} w4_status;
+
+typedef enum { W4_F16 = 0, W4_BF16 = 1, W4_F32 = 2 } w4_dtype;
+
+/*
+ * w4_quantize_pack -- AWQ weight scaling + group-wise RTN INT4 + packing.
+ *
+ * Computes, for every output row n and group g (channels k with group(k) == g, where
+ * group(k) = g_idx[k] if g_idx != NULL else k / group_size):
+ *   W'[n,k] = float(W[n,k]) * s[k]                  (fp32, one rounding; s NULL = 1)
+ *   asymmetric: sc = fp16(max((max W' - min W')/15, 2^-14)),
+ *               z  = clamp(rint(-min W' / sc), 0, 15)           (stored as fp16 z)
+ *   symmetric:  sc = fp16(max(max|W'| / 7, 2^-14)), z = 8        (not stored)
+ *   q[n,k] = clamp(rint(W'[n,k] / sc) + z, 0, 15)   (IEEE fp32 division, rint =
+ *                                                    round half to even)
+ * and packs q into the device layout above.  Bit-exact: no fast-math anywhere.
+ *
+ *   W          device, [N,K] row-major, fp16 (w_dtype W4_F16) or bf16 (W4_BF16)
+ *   s          device fp32 [K] AWQ per-input-channel scale, or NULL
+ *   group_size 32 or a multiple of 64, K % group_size == 0
+ *   symmetric  0 = asymmetric (zeros required), 1 = symmetric (zeros must be NULL)
+ *   g_idx      device int32 [K] group of each input channel (act-order), or NULL;
+ *              entries outside [0, K/group_size) are skipped and reported as
+ *              W4_ERR_DEVICE_ARG by w4_check_device_error()
+ *   qweight    device uint32 [N*K/8] output, device layout
+ *   scales     device fp16 [G,N] output;  zeros device fp16 [G,N] output or NULL
+ * Uses 128*G bytes of shared memory per tile of 16 rows (G = K/group_size):
+ * K/group_size above 1536 returns W4_ERR_UNSUPPORTED.
+ */
+w4_status w4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K,
+                           const float* s, int32_t group_size, int32_t symmetric,
+                           const int32_t* g_idx, uint32_t* qweight, void* scales,
+                           void* zeros, w4_stream_t stream);
+
+/*
+ * w4a16_gemm -- fused dequantise-GEMM:  Y[M,N] = X'[M,K] * What[N,K]^T, with
+ *   X'[m,k]   = X[m,k] * s_inv[k]   (s_inv NULL: X' = X)   -- AWQ eq. 1, right factor
+ *   What[n,k] = (q[n,k] - z[group(k),n]) * scale[group(k),n]
+ * accumulated in fp32.  Without g_idx the (q - z) products are exact integers fed to
+ * the tensor cores and each group's fp32 partial sum is multiplied by its scale; with
+ * g_idx the scale is folded into an fp16 weight before the MMA (fp16 activations only).
+ * With s_inv, X' is rounded to the activation dtype before the MMA.
+ *
+ *   X          device [M,K] row-major, act_dtype W4_F16 or W4_BF16
+ *   qweight, scales, zeros, g_idx, group_size: as produced by w4_quantize_pack
+ *   s_inv      device fp32 [K] or NULL
+ *   Y          device [M,N] row-major output, out_dtype W4_F16, W4_BF16 or W4_F32
+ *   workspace  device scratch of at least w4a16_workspace_bytes(M,N,K,group_size)
+ *              bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE;
+ *              every call leaves it zero-filled again where that matters, so one
+ *              workspace may be reused by any number of calls on one stream.  Calls
+ *              that may overlap on the GPU need separate workspaces.  After a call
+ *              whose kernel reported W4_ERR_TIMEOUT, zero it again.
+ * M == 0 is a no-op.  M <= 64 runs the bandwidth-bound decode kernel (warp MMAs,
+ * split-K across the GPU), larger M the tcgen05 tensor-core kernel.
+ * bf16 activations with g_idx return W4_ERR_UNSUPPORTED.
+ */
+w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                     const uint32_t* qweight, const void* scales, const void* zeros,
+                     const int32_t* g_idx, int32_t group_size, const float* s_inv,
+                     void* Y, w4_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                     w4_stream_t stream);
+
+/* Bytes of workspace w4a16_gemm needs for these sizes on the current device
+ * (0 on invalid sizes). */
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size);
+
+/* Test aid: convert device-layout packed weights to the canonical layout
+ * (uint32 [N, K/8], nibble j of word i of row n = q[n][8i+j]).  Both device pointers. */
+w4_status w4_unpack_canonical(const uint32_t* qweight, int64_t N, int64_t K,
+                              uint32_t* qweight_canonical, w4_stream_t stream);
+
+/* Synchronises the current device, then reports and clears the device-side error word:
+ * W4_ERR_TIMEOUT if a kernel gave up a bounded wait, W4_ERR_DEVICE_ARG if a kernel met
+ * an out-of-range g_idx entry, W4_ERR_CUDA if the device reports a CUDA error, W4_OK. */
+w4_status w4_check_device_error(void);
+
+/* Bound, in nanoseconds, of every wait inside the library's kernels (default 2e9).
+ * Lowering it is a test aid; values below 1000 are raised to 1000. */
+w4_status w4_set_wait_limit_ns(uint64_t ns);
+
+/* Test aid for the watchdog: launches one block whose thread waits on a barrier that
+ * nothing completes; the bounded wait expires after the configured limit and sets the
+ * device error word (so w4_check_device_error() then returns W4_ERR_TIMEOUT). */
+w4_status w4_selftest_expired_wait(w4_stream_t stream);
+
+/* Static string naming a status. */
+const char* w4_status_string(w4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

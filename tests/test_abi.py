@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI: the sm_100a library builds, loads, exports every entry
+point declared in include/w4a16.h, and rejects bad arguments before touching a GPU.
+No compute call is made (this file runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_weight_only_w4_b200 as w4
+from bit_weight_only_w4_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return w4.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "w4a16.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4\w*)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("w4_quantize_pack", "w4a16_gemm", "w4a16_workspace_bytes", "w4_unpack_canonical",
+              "w4_check_device_error", "w4_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    # and nothing is hidden behind C++ mangling
+    out = os.popen(f"nm -D --defined-only {w4.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}$", out, re.M), name
+
+
+def test_status_strings(L):
+    assert w4.w4_status_string(0) == "W4_OK"
+    assert w4.w4_status_string(2) == "W4_ERR_UNSUPPORTED"
+    assert w4.w4_status_string(99) == "W4_ERR_UNKNOWN"
+
+
+def _gemm(L, M=1, N=128, K=128, g=128, X=16, qw=16, sc=16, Y=16, act=0, out=0, gidx=None):
+    v = ctypes.c_void_p
+    return L.w4a16_gemm(v(X), act, M, N, K, v(qw), v(sc), None, v(gidx) if gidx else None, g,
+                        None, v(Y), out, v(256), 1 << 30, None)
+
+
+def test_gemm_rejects_bad_shapes_before_launch(L):
+    assert _gemm(L, N=8) == w4.W4_ERR_UNSUPPORTED            # N % 16
+    assert _gemm(L, K=96, g=32) == w4.W4_ERR_UNSUPPORTED     # K % 64
+    assert _gemm(L, K=128, g=48) == w4.W4_ERR_INVALID_ARG    # K % g
+    assert _gemm(L, K=192, g=96) == w4.W4_ERR_UNSUPPORTED    # g not 32 or 64j
+    assert _gemm(L, N=0) == w4.W4_ERR_INVALID_ARG
+    assert _gemm(L, M=-1) == w4.W4_ERR_INVALID_ARG
+    assert _gemm(L, act=2) == w4.W4_ERR_INVALID_ARG          # fp32 activations
+    assert _gemm(L, out=7) == w4.W4_ERR_INVALID_ARG
+    assert _gemm(L, M=0) == w4.W4_OK                         # empty batch: no-op
+
+
+def test_gemm_rejects_null_and_misaligned_pointers(L):
+    assert _gemm(L, X=0) == w4.W4_ERR_INVALID_ARG
+    assert _gemm(L, Y=0) == w4.W4_ERR_INVALID_ARG
+    assert _gemm(L, X=24) == w4.W4_ERR_INVALID_ARG           # not 16-byte aligned
+    assert _gemm(L, qw=20) == w4.W4_ERR_INVALID_ARG
+    assert _gemm(L, act=1, gidx=16) == w4.W4_ERR_UNSUPPORTED  # bf16 + act-order
+
+
+def test_quantize_rejects_bad_arguments(L):
+    v = ctypes.c_void_p
+    q = L.w4_quantize_pack
+    # symmetric with zeros / asymmetric without zeros
+    assert q(v(16), 0, 16, 64, None, 32, 1, None, v(16), v(16), v(16), None) == w4.W4_ERR_INVALID_ARG
+    assert q(v(16), 0, 16, 64, None, 32, 0, None, v(16), v(16), None, None) == w4.W4_ERR_INVALID_ARG
+    assert q(None, 0, 16, 64, None, 32, 0, None, v(16), v(16), v(16), None) == w4.W4_ERR_INVALID_ARG
+    assert q(v(16), 2, 16, 64, None, 32, 0, None, v(16), v(16), v(16), None) == w4.W4_ERR_INVALID_ARG
+    assert q(v(16), 0, 15, 64, None, 32, 0, None, v(16), v(16), v(16), None) == w4.W4_ERR_UNSUPPORTED
+    # too many groups for the shared-memory tables
+    assert q(v(16), 0, 16, 64 * 1600, None, 32, 0, None, v(16), v(16), v(16), None) == \
+        w4.W4_ERR_UNSUPPORTED
+
+
+def test_workspace_bytes_invalid_sizes(L):
+    assert w4.w4a16_workspace_bytes(1, 8, 128, 128) == 0
+    assert w4.w4a16_workspace_bytes(0, 128, 128, 128) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    W = torch.zeros(16, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        w4.w4_quantize_pack(W, group_size=32)

@@ -1,0 +1,213 @@
+"""GPU parity of w4a16_gemm against the CPU oracle's fp32 product.
+
+Inputs to the GEMM are the oracle's own packed weights (device layout), so these tests do
+not depend on the GPU quantiser.  Tolerance (stated for the path): max-abs <= 2e-2 and
+relative L2 <= 1e-3 against the oracle's fp32 Y; bf16 outputs within one bf16 ulp of
+the rounded oracle value.  Shapes span several tiles and ragged tails along M, N and K,
+both kernels (M <= 64 and larger), every group size and both activation types.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import bit_weight_only_w4_b200 as w4
+from bit_weight_only_w4_b200 import workloads
+from tests.gpu_util import (act_order, check_y, dev, dev_bits, random_layer, skip_without_gpu,
+                            to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_gemm(X_bits, act, qd, scales, zeros, g, g_idx, s_inv, out):
+    import torch
+    tdt = {"fp16": torch.float16, "bf16": torch.bfloat16, "fp32": torch.float32}
+    Y = w4.w4a16_gemm(dev_bits(X_bits, tdt[act]), dev(qd.view(np.int32)),
+                      dev_bits(scales, torch.float16),
+                      None if zeros is None else dev_bits(zeros, torch.float16),
+                      g, dev(g_idx), dev(s_inv), out_dtype=tdt[out])
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    return to_f64(Y)
+
+
+def case(M, N, K, g, act="fp16", out="fp16", sym=False, gidx=False, use_s=True, seed=0,
+         tol_rel=None):
+    rng = np.random.default_rng(seed + M * 7919 + N * 31 + K + g)
+    X, W, s, s_inv = random_layer(rng, M, N, K, act)
+    g_idx = act_order(rng, K, g) if gidx else None
+    q, scales, zeros = oracle.quantize_weights(W, s, g, sym, g_idx)
+    qd = oracle.pack_device(q)
+    s_call = s_inv if use_s else None
+    Y = gpu_gemm(X, act, qd, scales, zeros, g, g_idx, s_call, out)
+    Y_ref = oracle.reference_y(X, s_call, q, scales, zeros, g, g_idx, x_is_bf16=(act == "bf16"))
+    kw = {} if tol_rel is None else {"tol_rel": tol_rel}
+    return check_y(Y, Y_ref, out, **kw)
+
+
+# ---------------------------------------------------------------- decode kernel (M <= 64)
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16, 17, 32, 33, 64])
+def test_decode_token_counts(M):
+    skip_without_gpu()
+    case(M, 256, 1024, 128)
+
+
+@pytest.mark.parametrize("N,K", [(16, 64), (48, 192), (144, 320), (400, 4096), (4096, 128)])
+def test_decode_ragged_shapes(N, K):
+    skip_without_gpu()
+    case(5, N, K, 64)
+
+
+@pytest.mark.parametrize("g", [32, 64, 128, 256, 1024])
+@pytest.mark.parametrize("sym", [False, True])
+def test_decode_group_sizes(g, sym):
+    skip_without_gpu()
+    case(4, 192, 1024, g, sym=sym)
+
+
+@pytest.mark.parametrize("out", ["fp16", "bf16", "fp32"])
+@pytest.mark.parametrize("act", ["fp16", "bf16"])
+def test_decode_dtypes(act, out):
+    skip_without_gpu()
+    # bf16 activations: X arrives already scaled (s^-1 absorbed upstream), like prefill
+    case(7, 320, 512, 128, act=act, out=out, use_s=(act == "fp16"))
+
+
+def test_decode_bf16_with_s_inv():
+    skip_without_gpu()
+    # X' is rounded to bf16 before the MMA: ~2^-9 relative error per activation
+    case(6, 256, 1024, 128, act="bf16", out="fp32", use_s=True, tol_rel=4e-3)
+
+
+@pytest.mark.parametrize("M", [1, 16, 33])
+@pytest.mark.parametrize("g", [32, 128, 1024])
+def test_decode_act_order(M, g):
+    skip_without_gpu()
+    case(M, 256, 1024, g, sym=True, gidx=True)
+
+
+def test_decode_act_order_asymmetric():
+    skip_without_gpu()
+    case(3, 128, 512, 64, sym=False, gidx=True)
+
+
+def test_decode_repeated_calls_are_deterministic():
+    """Split-K partials are combined in a fixed order and the fix-up counters are left at
+    zero, so back-to-back calls with one workspace give bit-identical results."""
+    skip_without_gpu()
+    import torch
+    rng = np.random.default_rng(17)
+    M, N, K, g = 3, 1024, 4096, 128
+    X, W, s, s_inv = random_layer(rng, M, N, K)
+    q, scales, zeros = oracle.quantize_weights(W, s, g)
+    args = (dev_bits(X, torch.float16), dev(oracle.pack_device(q).view(np.int32)),
+            dev_bits(scales, torch.float16), dev_bits(zeros, torch.float16), g)
+    ys = [w4.w4a16_gemm(*args, s_inv=dev(s_inv)).clone() for _ in range(4)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert torch.equal(y.view(torch.int16), ys[0].view(torch.int16))
+    Y_ref = oracle.reference_y(X, s_inv, q, scales, zeros, g)
+    check_y(to_f64(ys[0]), Y_ref, "fp16")
+
+
+def test_empty_batch_is_noop():
+    skip_without_gpu()
+    import torch
+    X = torch.empty(0, 128, dtype=torch.float16, device="cuda")
+    qw = torch.zeros(16 * 128 // 8, dtype=torch.int32, device="cuda")
+    sc = torch.ones(1, 16, dtype=torch.float16, device="cuda")
+    Y = w4.w4a16_gemm(X, qw, sc, sc, 128)
+    assert Y.shape == (0, 16)
+
+
+# ---------------------------------------------------------------- prefill kernel (M > 64)
+@pytest.mark.parametrize("M", [65, 128, 200, 384])
+def test_prefill_token_counts(M):
+    skip_without_gpu()
+    case(M, 256, 512, 128, act="bf16", out="fp32", use_s=False)
+
+
+@pytest.mark.parametrize("N,K", [(16, 64), (144, 320), (384, 2048)])
+def test_prefill_ragged_shapes(N, K):
+    skip_without_gpu()
+    case(130, N, K, 64, act="bf16", out="fp32", use_s=False)
+
+
+@pytest.mark.parametrize("g", [32, 64, 128, 512])
+@pytest.mark.parametrize("sym", [False, True])
+def test_prefill_group_sizes(g, sym):
+    skip_without_gpu()
+    case(160, 256, 1024, g, act="bf16", out="fp32", sym=sym, use_s=False)
+
+
+@pytest.mark.parametrize("act,out,use_s", [("fp16", "fp16", True), ("fp16", "fp32", False),
+                                           ("bf16", "bf16", False), ("bf16", "fp16", False)])
+def test_prefill_dtypes(act, out, use_s):
+    skip_without_gpu()
+    case(192, 256, 768, 128, act=act, out=out, use_s=use_s)
+
+
+@pytest.mark.parametrize("g", [32, 128, 1024])
+def test_prefill_act_order(g):
+    skip_without_gpu()
+    case(130, 256, 1024, g, sym=True, gidx=True, out="fp32")
+
+
+# ---------------------------------------------------------------- measured workloads
+def sampled_case(config_id, layer, M, g=None, rows=48, cols=192, seed=0):
+    """Full-size layer on the GPU, oracle on a seeded sample of outputs (row and column
+    subsets, always including the first and last of each)."""
+    import torch
+    wl = workloads.workload(config_id)
+    li = workloads.make_layer(wl, layer, M=M, group_size=g)
+    rng = np.random.default_rng(seed)
+    ms = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, min(rows, M))]))
+    ns = np.unique(np.concatenate([[0, li.N - 1], rng.integers(0, li.N, cols)]))
+    W_bits = li.W.view(np.uint16)
+    act = torch.bfloat16 if li.act_dtype == "bf16" else torch.float16
+    qw, sc, zr = w4.w4_quantize_pack(dev_bits(W_bits, torch.float16), dev(li.s), li.group_size,
+                                     li.symmetric, dev(li.g_idx))
+    out = "fp32" if li.act_dtype == "bf16" else "fp16"
+    Y = w4.w4a16_gemm(dev_bits(li.X, act), qw, sc, zr, li.group_size, dev(li.g_idx), dev(li.s_inv),
+                      out_dtype=torch.float32 if out == "fp32" else torch.float16)
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    Yg = to_f64(Y)[np.ix_(ms, ns)]
+    # the oracle quantises only the sampled output rows (rows are independent)
+    q, scales, zeros = oracle.quantize_weights(W_bits[ns], li.s, li.group_size, li.symmetric,
+                                               li.g_idx)
+    Y_ref = oracle.reference_y(li.X, li.s_inv, q, scales, zeros, li.group_size, li.g_idx,
+                               x_is_bf16=(li.act_dtype == "bf16"), rows=ms)
+    return check_y(Yg, Y_ref, out)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+def test_llama7b_decode_layers(layer, M):
+    skip_without_gpu()
+    sampled_case(2, layer, M)
+
+
+def test_single_layer_config():
+    skip_without_gpu()
+    sampled_case(1, 0, 1, rows=1, cols=4096)
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 64])
+@pytest.mark.parametrize("layer", [0, 2, 3])
+def test_llama70b_layers(layer, M):
+    skip_without_gpu()
+    sampled_case(3, layer, M)
+
+
+@pytest.mark.parametrize("M", [512, 4096])
+@pytest.mark.parametrize("layer", [0, 1])
+def test_llama8b_prefill_layers(layer, M):
+    skip_without_gpu()
+    sampled_case(4, layer, M, rows=24, cols=128)
+
+
+@pytest.mark.parametrize("M", [1, 16, 1024])
+@pytest.mark.parametrize("g", [32, 64, 128, 4096])
+def test_gptq_act_order_config(M, g):
+    skip_without_gpu()
+    sampled_case(5, 0, M, g=g, rows=24, cols=128)
