@@ -215,7 +215,9 @@ int oracle_quantize(const float* Wp, int64_t N, int64_t K, int32_t group_size, i
             if (symmetric) {
                 zf[g] = 8.0f;
             } else {
-                zf[g] = clampf(rintf(-mn[g] / sc[g]), 0.0f, 15.0f);
+                /* z is an integer in [0,15]: rint(-(+0)) = -0 must be stored as +0 */
+                int zi = (int)clampf(rintf(-mn[g] / sc[g]), 0.0f, 15.0f);
+                zf[g] = (float)zi;
                 if (zeros) zeros[g * N + n] = oracle_f32_to_f16(zf[g]);
             }
         }

@@ -215,6 +215,8 @@ def test_degenerate_groups_get_minimum_scale():
     q, scales, zeros = oracle.quantize(W, 32, False)
     assert scales[0, 0] == 0x0400 and scales[0, 1] == 0x0400
     assert np.all(q[0] == q[0, 0])
+    # the zero point is the integer 0, stored as +0 (never the fp16 pattern of -0)
+    assert zeros[0, 0] == 0x0000 and zeros[0, 1] == 0x0000
 
 
 def test_rejects_bad_arguments():
