@@ -261,7 +261,7 @@ def time_decode(M, steps, warmup, w4, torch, world, wl, projs, step_bytes, clock
             gj.replay()
             ms, _ = time_graph(torch, gj)
             us = ms * 1e3 / N_LAYERS
-            rows.append({"layer": f"{pr['li'].name} {pr['li'].K}x{pr['li'].N}",
+            rows.append({"layer": f"{wl.layers[j].name} {pr['li'].K}x{pr['li'].N}",
                          "us": round(us, 3), "gbs": round(pr["bytes"] / (us * 1e-6) / 1e9, 1)})
             del gj
         out["per_layer"] = rows

@@ -17,6 +17,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kDecodeMaxM = 64;
 constexpr int kDecodeMaxCtasPerSm = 2;
 constexpr int kQuantMaxGroups = 1536;
+constexpr int64_t kMaxBands = 8192;                       // N <= 1,048,576 (fix-up counters)
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -32,6 +33,7 @@ w4_status check_layer_shape(int64_t N, int64_t K, int32_t group_size) {
     if (N > INT_MAX / 2 || K > INT_MAX / 2) return W4_ERR_UNSUPPORTED;
     if (K % group_size != 0) return W4_ERR_INVALID_ARG;
     if (N % 16 != 0 || K % 64 != 0) return W4_ERR_UNSUPPORTED;
+    if (N > kMaxBands * 128) return W4_ERR_UNSUPPORTED;
     if (group_size != 32 && group_size % 64 != 0) return W4_ERR_UNSUPPORTED;
     return W4_OK;
 }
@@ -88,15 +90,15 @@ int DecodeKernel<NT, BF16, GIDX>::ctas_per_sm[kMaxDevices];
 template <int NT, bool BF16, bool GIDX>
 std::once_flag DecodeKernel<NT, BF16, GIDX>::occ_flags[kMaxDevices];
 
-size_t decode_counter_bytes(int64_t N) {
-    const int64_t bands = (N / 16 + w4d::kWarps - 1) / w4d::kWarps;
-    return (size_t)((bands * 4 + 255) / 256 * 256);
-}
+// Split-K fix-up counters live in a fixed region at the start of the workspace, one per
+// 128-row band, so that every call -- whatever its N -- finds its counters where earlier
+// calls left them at zero; the partial-sum slots follow the region.
+constexpr size_t kCounterBytes = (size_t)kMaxBands * 4;   // 32 KB
 
-size_t decode_workspace_bytes(int64_t M, int64_t N, int sms) {
+size_t decode_workspace_bytes(int64_t M, int sms) {
     const int Mp = 8 * decode_tiles_for(M);
     const size_t partials = (size_t)sms * kDecodeMaxCtasPerSm * 2 * w4d::kBandRows * Mp * 4;
-    return decode_counter_bytes(N) + partials;
+    return kCounterBytes + partials;
 }
 
 template <int NT, bool BF16, bool GIDX>
@@ -111,7 +113,7 @@ w4_status launch_decode(w4d::DecodeParams p, unsigned char* ws, int dev, cudaStr
     p.base = p.units / P;
     p.rem = p.units % P;
     p.counters = reinterpret_cast<unsigned*>(ws);
-    p.partials = reinterpret_cast<float*>(ws + decode_counter_bytes(p.N));
+    p.partials = reinterpret_cast<float*>(ws + kCounterBytes);
     w4d::decode_kernel<NT, BF16, GIDX><<<P, w4d::kThreads, DK::smem, stream>>>(p);
     return launch_status();
 }
@@ -234,7 +236,7 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size
     const int dev = current_device();
     const int sms = dev >= 0 ? sm_count(dev) : 0;
     if (sms <= 0) return 0;
-    if (M <= kDecodeMaxM) return decode_workspace_bytes(M, N, sms);
+    if (M <= kDecodeMaxM) return decode_workspace_bytes(M, sms);
     return (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
 }
 

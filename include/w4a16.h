@@ -29,8 +29,8 @@
  *    records a device-side error word and returns.  w4_check_device_error() reads it.
  *  - No C++ exception crosses this ABI.  The library keeps no per-call host state, so
  *    calls from several host threads on different streams are safe.
- *  - Shapes: N % 16 == 0, K % 64 == 0, group_size == 32 or a multiple of 64, and
- *    K % group_size == 0 (group_size == K is per-channel).  Pointers to packed weights,
+ *  - Shapes: N % 16 == 0, N <= 1048576, K % 64 == 0, group_size == 32 or a multiple
+ *    of 64, and K % group_size == 0 (group_size == K is per-channel).  Pointers to packed weights,
  *    activations, outputs and fp16 metadata must be 16-byte aligned.
  *
  * Packed weight format ("device layout")

@@ -41,6 +41,12 @@ def case(M, N, K, g, act="fp16", out="fp16", sym=False, gidx=False, use_s=True, 
     Y = gpu_gemm(X, act, qd, scales, zeros, g, g_idx, s_call, out)
     Y_ref = oracle.reference_y(X, s_call, q, scales, zeros, g, g_idx, x_is_bf16=(act == "bf16"))
     kw = {} if tol_rel is None else {"tol_rel": tol_rel}
+    if out == "bf16":
+        Xp = oracle.awq_scale_acts(X, s_call, act == "bf16").astype(np.float64)
+        What = oracle.dequant(q, scales, zeros, g, g_idx).astype(np.float64)
+        kw["absprod"] = np.abs(Xp) @ np.abs(What).T
+        kw["act_round"] = 0.0 if s_call is None else (2.0 ** -8 if act == "bf16" else 2.0 ** -11)
+        kw["K"] = K
     return check_y(Y, Y_ref, out, **kw)
 
 
@@ -107,6 +113,15 @@ def test_decode_repeated_calls_are_deterministic():
         assert torch.equal(y.view(torch.int16), ys[0].view(torch.int16))
     Y_ref = oracle.reference_y(X, s_inv, q, scales, zeros, g)
     check_y(to_f64(ys[0]), Y_ref, "fp16")
+
+
+def test_decode_workspace_reuse_across_shapes():
+    """One workspace shared by calls of different N and M: the split-K counters must be
+    found at zero by every call, whatever the previous call's shape."""
+    skip_without_gpu()
+    for (M, N, K) in [(2, 256, 512), (9, 12288, 1024), (1, 144, 4096), (33, 8192, 512),
+                      (3, 12288, 1024)]:
+        case(M, N, K, 128, seed=5)
 
 
 def test_empty_batch_is_noop():
