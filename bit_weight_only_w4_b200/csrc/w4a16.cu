@@ -237,7 +237,8 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size
     const int sms = dev >= 0 ? sm_count(dev) : 0;
     if (sms <= 0) return 0;
     if (M <= kDecodeMaxM) return decode_workspace_bytes(M, sms);
-    return (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
+    // prefill: scaled activations, behind the counter region (which must stay zero)
+    return kCounterBytes + (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
 }
 
 w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
@@ -296,10 +297,11 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
     if (s_inv) {
         const size_t pairs = (size_t)M * (size_t)K / 2;
         const unsigned blocks = (unsigned)((pairs + 255) / 256 < 65535 * 8 ? (pairs + 255) / 256 : 65535 * 8);
-        if (bf16) w4p::scale_acts_kernel<true><<<blocks, 256, 0, strm>>>(X, s_inv, workspace, (int)M, (int)K);
-        else w4p::scale_acts_kernel<false><<<blocks, 256, 0, strm>>>(X, s_inv, workspace, (int)M, (int)K);
+        void* xp = reinterpret_cast<unsigned char*>(workspace) + kCounterBytes;
+        if (bf16) w4p::scale_acts_kernel<true><<<blocks, 256, 0, strm>>>(X, s_inv, xp, (int)M, (int)K);
+        else w4p::scale_acts_kernel<false><<<blocks, 256, 0, strm>>>(X, s_inv, xp, (int)M, (int)K);
         if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
-        Xeff = workspace;
+        Xeff = xp;
     }
     CUtensorMap map;
     if (!make_act_tensor_map(&map, Xeff, bf16, M, K)) return W4_ERR_CUDA;

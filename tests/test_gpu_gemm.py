@@ -116,12 +116,15 @@ def test_decode_repeated_calls_are_deterministic():
 
 
 def test_decode_workspace_reuse_across_shapes():
-    """One workspace shared by calls of different N and M: the split-K counters must be
-    found at zero by every call, whatever the previous call's shape."""
+    """One workspace shared by decode and prefill calls of different shapes: the split-K
+    counters must be found at zero by every call, whatever the previous call used the
+    workspace for."""
     skip_without_gpu()
-    for (M, N, K) in [(2, 256, 512), (9, 12288, 1024), (1, 144, 4096), (33, 8192, 512),
-                      (3, 12288, 1024)]:
-        case(M, N, K, 128, seed=5)
+    for (M, N, K, act, use_s) in [(2, 256, 512, "fp16", True), (9, 12288, 1024, "fp16", True),
+                                  (200, 512, 2048, "fp16", True),   # prefill scratch use
+                                  (1, 144, 4096, "fp16", True), (33, 8192, 512, "fp16", True),
+                                  (130, 256, 4096, "fp16", True), (3, 12288, 1024, "fp16", True)]:
+        case(M, N, K, 128, act=act, use_s=use_s, seed=5)
 
 
 def test_empty_batch_is_noop():
