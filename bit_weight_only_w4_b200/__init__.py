@@ -52,6 +52,8 @@ def lib():
         L.w4_quantize_pack.restype = st
         L.w4a16_gemm.argtypes = [vp, st, i64, i64, i64, vp, vp, vp, vp, i32, vp, vp, st, vp, sz, vp]
         L.w4a16_gemm.restype = st
+        L.w4a16_gemm_noalloc.argtypes = [vp, st, i64, i64, i64, vp, vp, vp, vp, i32, vp, vp, st, vp]
+        L.w4a16_gemm_noalloc.restype = st
         L.w4a16_workspace_bytes.argtypes = [i64, i64, i64, i32]
         L.w4a16_workspace_bytes.restype = sz
         L.w4_unpack_canonical.argtypes = [vp, i64, i64, vp, vp]
@@ -203,6 +205,27 @@ def w4a16_gemm(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None
                               _dtype_code(Y.dtype), _ptr(workspace), ws_bytes,
                               _stream_handle(stream, dev))
     _check(st, "w4a16_gemm")
+    return Y
+
+
+def w4a16_gemm_noalloc(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None,
+                       out_dtype=None, Y=None, stream=None):
+    """w4a16_gemm without a workspace, for callers that cannot allocate device memory at
+    the point of the call: the library's fixed per-device scratch is used instead.  Only
+    Y is allocated here, and only when not passed in."""
+    torch = _torch()
+    M, K = X.shape
+    N = scales.shape[1]
+    dev = _need_cuda(X, qweight, scales, zeros, g_idx, s_inv, Y)
+    out_dtype = out_dtype or X.dtype
+    if Y is None:
+        Y = torch.empty(M, N, dtype=out_dtype, device=dev)
+    with _DeviceGuard(dev):
+        st = lib().w4a16_gemm_noalloc(_ptr(X), _dtype_code(X.dtype), M, N, K, _ptr(qweight),
+                                      _ptr(scales), _ptr(zeros), _ptr(g_idx), int(group_size),
+                                      _ptr(s_inv), _ptr(Y), _dtype_code(Y.dtype),
+                                      _stream_handle(stream, dev))
+    _check(st, "w4a16_gemm_noalloc")
     return Y
 
 

@@ -374,3 +374,88 @@ extern "C" w4_status w4_selftest_expired_wait(w4_stream_t stream) {
     expired_wait_kernel<<<1, 32, 0, as_stream(stream)>>>();
     return launch_status();
 }
+
+// ---------------------------------------------------------------------------------------
+// w4a16_gemm_noalloc: the small-batch GEMM for callers that cannot hand the library a
+// workspace.  Its scratch (split-K counters and partial sums) is one fixed array in
+// device memory that exists on every GPU that loads this library, from module load to
+// process exit.  Host code never dereferences the array's name: it is only a host-side
+// handle, so the device address is fetched once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;   // 8 MiB
+__device__ __align__(256) unsigned char g_w4_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocScratch {
+    std::once_flag once;
+    void* ptr = nullptr;
+    cudaError_t err = cudaSuccess;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+// Set-up on the first call per device (that device current): look up the array's device
+// address and zero its counter region, the part that every call expects to find at zero.
+void* noalloc_scratch(int dev) {
+    NoAllocScratch& s = g_noalloc[dev];
+    std::call_once(s.once, [&] {
+        void* p = nullptr;
+        s.err = cudaGetSymbolAddress(&p, g_w4_noalloc_scratch);
+        if (s.err == cudaSuccess) s.err = cudaMemset(p, 0, kCounterBytes);
+        if (s.err == cudaSuccess) s.err = cudaDeviceSynchronize();
+        if (s.err == cudaSuccess) s.ptr = p;
+    });
+    return s.ptr;
+}
+
+}  // namespace
+
+extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64_t M, int64_t N,
+                                        int64_t K, const uint32_t* qweight, const void* scales,
+                                        const void* zeros, const int32_t* g_idx, int32_t group_size,
+                                        const float* s_inv, void* Y, w4_dtype out_dtype,
+                                        w4_stream_t stream) {
+    if (M < 0) return W4_ERR_INVALID_ARG;
+    if (act_dtype != W4_F16 && act_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
+    if (out_dtype != W4_F16 && out_dtype != W4_BF16 && out_dtype != W4_F32) return W4_ERR_INVALID_ARG;
+    w4_status st = check_layer_shape(N, K, group_size);
+    if (st != W4_OK) return st;
+    if (M == 0) return W4_OK;
+    if (M > kDecodeMaxM) return W4_ERR_UNSUPPORTED;
+    if (!X || !qweight || !scales || !Y) return W4_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(zeros, 16) ||
+        !aligned(g_idx, 16) || !aligned(s_inv, 16) || !aligned(Y, 16))
+        return W4_ERR_INVALID_ARG;
+    const bool bf16 = act_dtype == W4_BF16;
+    const bool gidx = g_idx != nullptr;
+    if (bf16 && gidx) return W4_ERR_UNSUPPORTED;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    const int sms = sm_count(dev);
+    if (sms <= 0) return W4_ERR_CUDA;
+    if (decode_workspace_bytes(M, sms) > kNoAllocScratchBytes) return W4_ERR_UNSUPPORTED;
+    unsigned char* ws = reinterpret_cast<unsigned char*>(noalloc_scratch(dev));
+    if (!ws) return W4_ERR_CUDA;
+
+    w4d::DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.X = X;
+    p.qw = qweight;
+    p.scales = reinterpret_cast<const __half*>(scales);
+    p.zeros = reinterpret_cast<const __half*>(zeros);
+    p.g_idx = g_idx;
+    p.s_inv = s_inv;
+    p.Y = Y;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.group_size = group_size;
+    p.G = (int)(K / group_size);
+    p.out_dtype = (int)out_dtype;
+    p.KA = (int)(K / 64);
+    p.tiles = (int)(N / 16);
+    cudaStream_t strm = as_stream(stream);
+    if (bf16) return dispatch_decode<true, false>(p, ws, dev, strm);
+    return gidx ? dispatch_decode<false, true>(p, ws, dev, strm)
+                : dispatch_decode<false, false>(p, ws, dev, strm);
+}

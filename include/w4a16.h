@@ -138,6 +138,29 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
                      void* Y, w4_dtype out_dtype, void* workspace, size_t workspace_bytes,
                      w4_stream_t stream);
 
+/*
+ * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 16 (M <= 64 where the scratch fits)
+ * without a caller-supplied workspace.  The pages have no counterpart to this call; it
+ * exists for callers that cannot allocate device memory where they run the GEMM, such as
+ * plug-ins of inference runtimes that forbid allocation after their set-up phase, or C
+ * callers without a caching allocator, for whom cudaMalloc/cudaFree per call would
+ * synchronise the whole device.
+ *
+ * Arguments, layouts and results are those of w4a16_gemm minus the workspace.  The
+ * scratch is one fixed 8 MiB array in device memory that every GPU loading this library
+ * holds until the process exits.  Calls whose scratch would exceed it (M above 16 on a
+ * 148-SM B200; any M > 64) return W4_ERR_UNSUPPORTED; use w4a16_gemm for them.  The
+ * first call on a device sets up that device (looks up the array's address, zeroes its
+ * counters and synchronises the device); make that first call before any stream
+ * capture.  Every call on a device shares the one array: calls that may overlap on the
+ * GPU (different streams without ordering) race and give wrong results.  The call
+ * allocates nothing and frees nothing.
+ */
+w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                             const uint32_t* qweight, const void* scales, const void* zeros,
+                             const int32_t* g_idx, int32_t group_size, const float* s_inv,
+                             void* Y, w4_dtype out_dtype, w4_stream_t stream);
+
 /* Bytes of workspace w4a16_gemm needs for these sizes on the current device
  * (0 on invalid sizes). */
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size);
