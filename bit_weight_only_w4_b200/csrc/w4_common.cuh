@@ -120,6 +120,16 @@ W4_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c
         : "memory");
 }
 
+// 3-D tiled tensor copy global -> shared (box given by the tensor map).
+W4_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int32_t c0, int32_t c1, int32_t c2,
+                        uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
 W4_DEV void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -197,7 +207,7 @@ W4_DEV ZeroConsts zero_consts_bf16(float z0, float z1) {
 template <bool BF16>
 W4_DEV void unpack_word(uint32_t w, const ZeroConsts& zc, uint32_t (&a)[4]) {
     if constexpr (!BF16) {
-        const __half2 sixteenth = __float2half2_rn(0.0625f);
+        const __half2 sixteenth = u32_as_h2(0x2C002C00u);   // (1/16, 1/16) in fp16
         const uint32_t w8 = w >> 8;
         a[0] = h2_as_u32(__hsub2(u32_as_h2(and_or(w, 0x000F000Fu, 0x64006400u)), u32_as_h2(zc.lo0)));
         a[1] = h2_as_u32(__hfma2(u32_as_h2(and_or(w, 0x00F000F0u, 0x64006400u)), sixteenth,

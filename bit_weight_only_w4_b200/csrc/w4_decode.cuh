@@ -9,18 +9,21 @@
 // tensor-core MMA (item 3).
 //
 // Work decomposition (B200-specific):
-//   unit      = 128 output rows (8 tiles of 16) x 64 input channels; the units of the
-//               layer are ordered row-band-major and split into equal contiguous
-//               ranges, one per CTA (stream-K), so every SM streams the same number of
+//   atom      = 16 output rows x 64 input channels (512 B of codes); the atoms of one
+//               128-row band are stored column block by column block, so up to 4
+//               consecutive column blocks of a band (up to 16 KB) are one contiguous copy;
+//   stream-K  = all (band, column block) atoms of the layer are split into equal
+//               contiguous ranges, one per CTA, so every SM streams the same number of
 //               bytes whatever N and K are;
-//   CTA       = 1 producer warp (one elected lane drives TMA bulk copies into an
-//               8-stage shared-memory ring) + 8 consumer warps (warp w owns rows
-//               16w..16w+15 of the band);
-//   consumer  = for each 16-deep step, one 32-bit word per lane is unpacked into the
-//               A operand of mma.m16n8k16 (weights as the 16-row side, up to 64 tokens
-//               as 8-column tiles), multiplied by exact integer weights (q - z) with
-//               fp32 accumulation, and each group's partial sum is multiplied by its
-//               scale in fp32;
+//   stage     = up to 4 column blocks of one band, 5 copies: the codes (one contiguous
+//               bulk copy), the activations (one 3-D TMA box of 4 column blocks x 8*NT
+//               token rows, 128B swizzle, rows >= M zero-filled), the s_inv slice, and the
+//               group rows of scales and of zero points met by the stage (2-D TMA boxes);
+//   CTA       = 1 producer warp + 8 consumer warps; consumer warp w owns rows
+//               16w..16w+15 of the band; per 16-deep step one 32-bit word per lane is
+//               unpacked into the A operand of mma.m16n8k16 (weights as the 16-row side,
+//               up to 64 tokens as 8-column tiles), multiplied as exact integers (q - z)
+//               with fp32 accumulation; each group's partial sum is scaled in fp32;
 //   fix-up    = a band split between CTAs is completed by the last CTA to finish it,
 //               which adds the fp32 partials of all contributors in CTA order
 //               (deterministic) and stores Y; its counter is reset to zero.
@@ -31,33 +34,17 @@ namespace w4d {
 
 constexpr int kWarps = 8;                 // consumer warps = row tiles per band
 constexpr int kBandRows = 16 * kWarps;    // 128
-constexpr int kStages = 8;
-constexpr int kXRow = 144;                // bytes per token row of a staged activation chunk
+constexpr int kAtomsPerStage = 4;         // column blocks per stage (256 input channels)
 constexpr int kThreads = 32 * (kWarps + 1);
 
-// shared-memory layout of one ring stage
 template <int NT>
-struct StageLayout {
-    static constexpr int w = 0;                         // 8 tiles x 512 B packed weights
-    static constexpr int x = 4096;                      // up to 8*NT rows x 144 B
-    static constexpr int si = x + 8 * NT * kXRow;       // 64 fp32 s_inv
-    static constexpr int sc = si + 256;                 // up to 2 groups x 128 fp16 scales
-    static constexpr int zr = sc + 512;                 // up to 2 groups x 128 fp16 zeros
-    static constexpr int gi = zr + 512;                 // 64 int32 g_idx
-    static constexpr int bytes = ((gi + 256) + 127) / 128 * 128;
-};
-
-template <int NT>
-struct SmemLayout {
-    static constexpr int ring = 0;
-    static constexpr int xc = ring + kStages * StageLayout<NT>::bytes;   // 2 converted chunks
-    static constexpr int bars = xc + 2 * 8 * NT * kXRow;
-    static constexpr int flags = bars + 2 * kStages * 8;
-    static constexpr int bytes = flags + 16;
+struct Cfg {
+    static constexpr int stages = NT == 1 ? 4 : 3;
+    static constexpr int mpad = 8 * NT;               // token rows per activation box slot
+    static constexpr int xbox = mpad * 128;           // bytes per activation box slot
 };
 
 struct DecodeParams {
-    const void* X;            // [M,K] fp16/bf16
     const uint32_t* qw;       // device layout
     const __half* scales;     // [G,N]
     const __half* zeros;      // [G,N] or null
@@ -69,8 +56,11 @@ struct DecodeParams {
     int M, N, K, group_size, G, out_dtype;
     int KA;                   // K / 64
     int tiles;                // N / 16
-    int units;                // bands * KA
-    int base, rem;            // units per CTA: base (+1 for the first rem CTAs)
+    int units;                // bands * KA atoms
+    int base, rem;            // atoms per CTA: base (+1 for the first rem CTAs)
+    int ngs;                  // group rows staged per stage (scale / zero-point box height)
+    // byte offsets inside one stage
+    int off_x, off_si, off_sc, off_zr, off_gi, stage_bytes;
 };
 
 W4_DEV int unit_begin(const DecodeParams& p, int c) { return c * p.base + min(c, p.rem); }
@@ -78,6 +68,7 @@ W4_DEV int cta_of_unit(const DecodeParams& p, int u) {
     const int split = p.rem * (p.base + 1);
     return u < split ? u / (p.base + 1) : p.rem + (u - split) / p.base;
 }
+W4_DEV int band_tiles(const DecodeParams& p, int band) { return min(kWarps, p.tiles - band * kWarps); }
 
 W4_DEV void store_out(const DecodeParams& p, int m, int n, float v) {
     const size_t idx = (size_t)m * p.N + n;
@@ -87,13 +78,22 @@ W4_DEV void store_out(const DecodeParams& p, int m, int n, float v) {
 }
 
 W4_DEV uint32_t lds32(const unsigned char* p) { return *reinterpret_cast<const uint32_t*>(p); }
+W4_DEV uint32_t lds32_at(uint32_t saddr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(saddr));
+    return v;
+}
+
+// byte offset of the 4-byte pair (token row, k-pair kp < 32) inside a 128B-swizzled box
+W4_DEV int xsw(int tok, int kp) { return tok * 128 + (((kp >> 2) ^ (tok & 7)) << 4) + ((kp & 3) << 2); }
 
 // Complete or hand off the accumulators of one band.
 template <int NT>
 W4_DEV void flush_band(const DecodeParams& p, int band, int u0, int u1, int cta, int w,
-                       int lane, int ctid, bool tile_ok, bool aborted,
-                       float (&acc)[NT][4], volatile int* s_flag) {
+                       int lane, int ctid, bool aborted, float (&acc)[NT][4],
+                       volatile int* s_flag) {
     const int Mp = 8 * NT;
+    const bool tile_ok = w < band_tiles(p, band);
     const int rl0 = 16 * w + (lane >> 2);            // row within the band
     const int n0 = band * kBandRows + rl0;
     const int q2 = 2 * (lane & 3);
@@ -122,7 +122,7 @@ W4_DEV void flush_band(const DecodeParams& p, int band, int u0, int u1, int cta,
             for (int e = 0; e < 4; ++e) {
                 const int m = 8 * nt + q2 + (e & 1);
                 const int rl = rl0 + ((e >> 1) << 3);
-                slot[rl * Mp + m] = acc[nt][e];
+                if (m < p.M) slot[rl * Mp + m] = acc[nt][e];
             }
     }
     __threadfence();
@@ -162,23 +162,35 @@ W4_DEV void flush_band(const DecodeParams& p, int band, int u0, int u1, int cta,
     named_bar_sync(2, 32 * kWarps);
 }
 
+W4_DEV void fold(float s0, float s1, float (&c)[4], float (&acc)[4]) {
+    acc[0] = fmaf(s0, c[0], acc[0]);
+    acc[1] = fmaf(s0, c[1], acc[1]);
+    acc[2] = fmaf(s1, c[2], acc[2]);
+    acc[3] = fmaf(s1, c[3], acc[3]);
+    c[0] = c[1] = c[2] = c[3] = 0.0f;
+}
+
 template <int NT, bool BF16, bool GIDX>
-__global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2) decode_kernel(const DecodeParams p) {
-    using SL = StageLayout<NT>;
-    using ML = SmemLayout<NT>;
-    extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ML::bars);
-    uint64_t* empty = full + kStages;
-    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + ML::flags);
+__global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_sc,
+                  const __grid_constant__ CUtensorMap tmap_zr, const DecodeParams p) {
+    using C = Cfg<NT>;
+    constexpr int S = C::stages;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * p.stage_bytes);
+    uint64_t* empty = full + S;
+    volatile int* s_abort = reinterpret_cast<volatile int*>(empty + S);
     volatile int* s_last = s_abort + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
     const int u0 = unit_begin(p, cta), u1 = unit_begin(p, cta + 1);
-    const int ngroups = (p.group_size == 32) ? 2 : 1;   // groups met by one 64-deep unit
+    const int g = p.group_size;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kWarps);
         }
@@ -186,60 +198,72 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2) decode_kernel(const
         *s_last = 0;
         fence_mbar_init();
     }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_x);
+        if (!GIDX) {
+            prefetch_tensormap(&tmap_sc);
+            if (p.zeros) prefetch_tensormap(&tmap_zr);
+        }
+    }
     __syncthreads();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         const uint64_t policy = policy_evict_first();
-        int issued = 0;
-        for (int u = u0; u < u1; ++u, ++issued) {
-            const int i = u - u0, s = i % kStages, ph = (i / kStages) & 1;
-            if (i >= kStages) {
-                bool ok = !*s_abort && mbar_wait(&empty[s], ph ^ 1);
+        int i = 0;
+        for (int u = u0; u < u1; ++i) {
+            const int band = u / p.KA, a0 = u - band * p.KA;
+            const int na = min(kAtomsPerStage, min(p.KA - a0, u1 - u));
+            const int s = i % S, ph = (i / S) & 1;
+            if (i >= S) {
+                const bool ok = !*s_abort && mbar_wait(&empty[s], ph ^ 1);
                 if (!ok) { *s_abort = 1; break; }
             }
-            unsigned char* st = smem + s * SL::bytes;
-            const int band = u / p.KA, a = u - band * p.KA;
-            const int tiles = min(kWarps, p.tiles - band * kWarps);
-            const int rows = 16 * tiles;
-            uint32_t bytes = tiles * 512 + p.M * 128;
-            if (p.s_inv) bytes += 256;
-            if (GIDX) bytes += 256;
-            else bytes += ngroups * rows * 2 * (p.zeros ? 2 : 1);
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
-            __syncwarp();
-            for (int c = lane; c < tiles; c += 32)
-                bulk_g2s_hint(st + SL::w + c * 512,
-                              p.qw + ((size_t)(band * kWarps + c) * p.KA + a) * 128, 512,
-                              &full[s], policy);
-            for (int c = lane; c < p.M; c += 32)
-                bulk_g2s(st + SL::x + c * kXRow,
-                         reinterpret_cast<const unsigned char*>(p.X) +
-                             ((size_t)c * p.K + (size_t)a * 64) * 2,
-                         128, &full[s]);
-            if (lane == 0 && p.s_inv) bulk_g2s(st + SL::si, p.s_inv + a * 64, 256, &full[s]);
-            if (GIDX) {
-                if (lane == 1) bulk_g2s(st + SL::gi, p.g_idx + a * 64, 256, &full[s]);
-            } else if (lane >= 2 && lane < 2 + ngroups) {
-                const int gg = lane - 2;
-                const int grp = (a * 64) / p.group_size + gg;
-                const size_t off = (size_t)grp * p.N + (size_t)band * kBandRows;
-                bulk_g2s(st + SL::sc + gg * 256, p.scales + off, rows * 2, &full[s]);
-                if (p.zeros) bulk_g2s(st + SL::zr + gg * 256, p.zeros + off, rows * 2, &full[s]);
+            unsigned char* st = smem + s * p.stage_bytes;
+            const int tb = band_tiles(p, band);
+            // one copy per operand: codes (contiguous run of the band), activations (one
+            // 3-D box: 4 column blocks x 8*NT token rows, rows >= M and blocks beyond K
+            // zero-filled), s_inv slice, scale rows and zero-point rows (2-D boxes)
+            const int g_first = (64 * a0) / g;
+            uint32_t bytes = na * tb * 512 + kAtomsPerStage * C::xbox;
+            if (p.s_inv) bytes += na * 256;
+            if (GIDX) bytes += na * 256;
+            else bytes += p.ngs * 256 * (p.zeros ? 2 : 1);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full[s], bytes);
+                bulk_g2s_hint(st, p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)a0 * tb),
+                              na * tb * 512, &full[s], policy);
+                tma_load_3d(st + p.off_x, &tmap_x, 0, 0, a0, &full[s]);
+                if (p.s_inv) bulk_g2s(st + p.off_si, p.s_inv + 64 * a0, na * 256, &full[s]);
+                if (GIDX) {
+                    bulk_g2s(st + p.off_gi, p.g_idx + 64 * a0, na * 256, &full[s]);
+                } else {
+                    tma_load_2d(st + p.off_sc, &tmap_sc, band * kBandRows, g_first, &full[s]);
+                    if (p.zeros) tma_load_2d(st + p.off_zr, &tmap_zr, band * kBandRows, g_first, &full[s]);
+                }
             }
             __syncwarp();
+            u += na;
         }
-        // On abort, wait (bounded) for copies already issued before leaving.
-        if (*s_abort && lane == 0) {
-            for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-                (void)mbar_wait(&full[i % kStages], (i / kStages) & 1);
-        }
+        // On abort, wait (bounded) for the copies already issued before leaving.
+        if (*s_abort && lane == 0)
+            for (int k = (i > S ? i - S : 0); k < i; ++k) (void)mbar_wait(&full[k % S], (k / S) & 1);
     } else {
         // ------------------------------------------------------------ consumers
         const int w = warp - 1;
         const int ctid = threadIdx.x - 32;
         const int q = lane & 3, g8 = lane >> 2;
         const int rl0 = 16 * w + g8, rl1 = rl0 + 8;
+        // activation fragment offsets inside a 128B-swizzled box: row g8 (+8 per token
+        // tile), k pairs 8j+q (b0) and 8j+4+q (b1) of the 16-deep step j
+        const int xrow = g8 * 128;
+        int xlo[4], xhi[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            xlo[j] = (((2 * j) ^ g8) << 4) + 4 * q;
+            xhi[j] = (((2 * j + 1) ^ g8) << 4) + 4 * q;
+        }
+        const bool g32 = (g == 32);
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -248,13 +272,13 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2) decode_kernel(const
         int cur_band = (u0 < u1) ? u0 / p.KA : -1;
         bool aborted = false;
 
-        for (int u = u0; u < u1; ++u) {
-            const int i = u - u0, s = i % kStages, ph = (i / kStages) & 1;
-            const int band = u / p.KA;
-            const bool tile_ok = band * kWarps + w < p.tiles;
+        int i = 0;
+        for (int u = u0; u < u1; ++i) {
+            const int band = u / p.KA, a0 = u - band * p.KA;
+            const int na = min(kAtomsPerStage, min(p.KA - a0, u1 - u));
+            const int s = i % S, ph = (i / S) & 1;
             if (band != cur_band) {
-                flush_band<NT>(p, cur_band, u0, u1, cta, w, lane, ctid,
-                               cur_band * kWarps + w < p.tiles, aborted, acc, s_last);
+                flush_band<NT>(p, cur_band, u0, u1, cta, w, lane, ctid, aborted, acc, s_last);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -265,133 +289,158 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2) decode_kernel(const
                 aborted = *s_abort || !mbar_wait(&full[s], ph);
                 if (aborted) *s_abort = 1;
             }
-            const unsigned char* st = smem + s * SL::bytes;
-            const unsigned char* xb = st + SL::x;
+            unsigned char* st = smem + s * p.stage_bytes;
+            unsigned char* xb = st + p.off_x;
             if (p.s_inv) {
-                // X' = X * s_inv, rounded to the activation type, once per chunk for all warps
-                unsigned char* xc = smem + ML::xc + (i & 1) * (8 * NT * kXRow);
+                // X' = X * s_inv rounded to the activation type, in place, once per stage
                 if (!aborted) {
-                    for (int e = ctid; e < p.M * 32; e += 32 * kWarps) {
-                        const int tok = e >> 5, kp = e & 31;
-                        const float2 v = unpack2<BF16>(lds32(xb + tok * kXRow + kp * 4));
-                        const float2 si = *reinterpret_cast<const float2*>(st + SL::si + kp * 8);
-                        *reinterpret_cast<uint32_t*>(xc + tok * kXRow + kp * 4) =
-                            pack2<BF16>(__fmul_rn(v.x, si.x), __fmul_rn(v.y, si.y));
+                    const float* si = reinterpret_cast<const float*>(st + p.off_si);
+                    const int per_box = p.M * 32;
+#pragma unroll
+                    for (int a = 0; a < kAtomsPerStage; ++a) {
+                        if (a < na) {
+                            for (int r = ctid; r < per_box; r += 32 * kWarps) {
+                                const int tok = r >> 5, kp = r & 31;
+                                uint32_t* px = reinterpret_cast<uint32_t*>(xb + a * C::xbox + xsw(tok, kp));
+                                const float2 v = unpack2<BF16>(*px);
+                                const float2 sv = *reinterpret_cast<const float2*>(si + 64 * a + 2 * kp);
+                                *px = pack2<BF16>(__fmul_rn(v.x, sv.x), __fmul_rn(v.y, sv.y));
+                            }
+                        }
                     }
                 }
                 named_bar_sync(1, 32 * kWarps);
-                xb = xc;
             }
-            if (!aborted && tile_ok) {
-                const uint4 wq = *reinterpret_cast<const uint4*>(st + SL::w + w * 512 + lane * 16);
-                const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+            const int tb = band_tiles(p, band);
+            if (!aborted && w < tb) {
                 if constexpr (!GIDX) {
-                    // scale and zero-point constants of the (at most two) groups of this unit
-                    const bool two = (ngroups == 2);
-                    const __half* sca = reinterpret_cast<const __half*>(st + SL::sc);
-                    const __half* zra = reinterpret_cast<const __half*>(st + SL::zr);
-                    const float sa0 = __half2float(sca[rl0]), sa1 = __half2float(sca[rl1]);
-                    const float sb0 = two ? __half2float(sca[128 + rl0]) : sa0;
-                    const float sb1 = two ? __half2float(sca[128 + rl1]) : sa1;
-                    float za0 = 8.0f, za1 = 8.0f, zb0 = 8.0f, zb1 = 8.0f;
-                    if (p.zeros) {
-                        za0 = __half2float(zra[rl0]);
-                        za1 = __half2float(zra[rl1]);
-                        zb0 = two ? __half2float(zra[128 + rl0]) : za0;
-                        zb1 = two ? __half2float(zra[128 + rl1]) : za1;
-                    }
-                    const ZeroConsts zca = BF16 ? zero_consts_bf16(za0, za1) : zero_consts_f16(za0, za1);
-                    const ZeroConsts zcb = BF16 ? zero_consts_bf16(zb0, zb1) : zero_consts_f16(zb0, zb1);
-                    float c[NT][4];
+                    // group rows staged for this stage start at group g_first; later groups
+                    // begin at multiples of g (no division inside the loop)
+                    const int g_first = (64 * a0) / g;
+                    int next_b = (g_first + 1) * g;
+                    const __half* scp = reinterpret_cast<const __half*>(st + p.off_sc);
+                    const __half* zrp = reinterpret_cast<const __half*>(st + p.off_zr);
+                    float s0, s1;
+                    ZeroConsts zc;
+                    auto load_group = [&]() {
+                        s0 = __half2float(scp[rl0]);
+                        s1 = __half2float(scp[rl1]);
+                        const float z0 = p.zeros ? __half2float(zrp[rl0]) : 8.0f;
+                        const float z1 = p.zeros ? __half2float(zrp[rl1]) : 8.0f;
+                        zc = BF16 ? zero_consts_bf16(z0, z1) : zero_consts_f16(z0, z1);
+                    };
+                    load_group();
+                    // two accumulator chains (even / odd 16-deep steps) for MMA overlap
+                    float c0[NT][4], c1[NT][4];
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) c[nt][e] = 0.0f;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t af[4];
-                        unpack_word<BF16>(wv[j], j < 2 ? zca : zcb, af);
+                        for (int e = 0; e < 4; ++e) c0[nt][e] = c1[nt][e] = 0.0f;
+                    auto next_group = [&]() {
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            const int tok = 8 * nt + g8;
-                            uint32_t b0 = 0, b1 = 0;
-                            if (tok < p.M) {
-                                const unsigned char* xr = xb + tok * kXRow + (16 * j + 2 * q) * 2;
-                                b0 = lds32(xr);
-                                b1 = lds32(xr + 16);
-                            }
-                            mma_16816<BF16>(c[nt], af, b0, b1);
+                            fold(s0, s1, c0[nt], acc[nt]);
+                            fold(s0, s1, c1[nt], acc[nt]);
                         }
-                        // end of a group: fold the group's partial into the accumulators
-                        if (j == 3 || (j == 1 && two)) {
-                            const float s0 = j < 2 ? sa0 : sb0;
-                            const float s1 = j < 2 ? sa1 : sb1;
+                        next_b += g;
+                        scp += 128;
+                        zrp += 128;
+                        load_group();
+                    };
+                    // per-stage fragment base addresses: every load below is one of these
+                    // registers plus a compile-time offset
+                    uint32_t xl[4], xh[4];
+                    const uint32_t xs = smem_u32(xb) + xrow;
 #pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                acc[nt][0] = fmaf(s0, c[nt][0], acc[nt][0]);
-                                acc[nt][1] = fmaf(s0, c[nt][1], acc[nt][1]);
-                                acc[nt][2] = fmaf(s1, c[nt][2], acc[nt][2]);
-                                acc[nt][3] = fmaf(s1, c[nt][3], acc[nt][3]);
-                                c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.0f;
+                    for (int j = 0; j < 4; ++j) {
+                        xl[j] = xs + xlo[j];
+                        xh[j] = xs + xhi[j];
+                    }
+                    const unsigned char* wbase = st + w * 512 + lane * 16;
+#pragma unroll
+                    for (int a = 0; a < kAtomsPerStage; ++a) {
+                        if (a < na) {
+                            const int ka = 64 * (a0 + a);
+                            if (ka >= next_b) next_group();
+                            const uint4 wq = *reinterpret_cast<const uint4*>(wbase + a * tb * 512);
+                            const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                if (j == 2 && g32 && ka + 32 >= next_b) next_group();
+                                uint32_t af[4];
+                                unpack_word<BF16>(wv[j], zc, af);
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    // token rows >= M were zero-filled by the tensor copy
+                                    const uint32_t b0 = lds32_at(xl[j] + a * C::xbox + nt * 1024);
+                                    const uint32_t b1 = lds32_at(xh[j] + a * C::xbox + nt * 1024);
+                                    // with few token tiles a second chain breaks the MMA
+                                    // dependency; with more tiles they already interleave
+                                    mma_16816<BF16>((NT <= 2 && (j & 1)) ? c1[nt] : c0[nt], af, b0, b1);
+                                }
                             }
                         }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        fold(s0, s1, c0[nt], acc[nt]);
+                        fold(s0, s1, c1[nt], acc[nt]);
                     }
                 } else {
                     // act-order: every channel has its own group; fold the scale into an
                     // fp16 weight (q - z) * scale before the MMA
-                    const int32_t* gis = reinterpret_cast<const int32_t*>(st + SL::gi);
+                    const int32_t* gis = reinterpret_cast<const int32_t*>(st + p.off_gi);
                     const int n_r0 = band * kBandRows + rl0, n_r1 = n_r0 + 8;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int kk = 16 * j + 2 * q;
-                        int gk[4] = {gis[kk], gis[kk + 1], gis[kk + 8], gis[kk + 9]};
+                    for (int a = 0; a < kAtomsPerStage; ++a) {
+                        if (a < na) {
+                            const uint4 wq = *reinterpret_cast<const uint4*>(
+                                st + (a * tb + w) * 512 + lane * 16);
+                            const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+                            const unsigned char* xa = xb + a * C::xbox;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if (gk[e] < 0 || gk[e] >= p.G) {
-                                atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
-                                gk[e] = 0;
+                            for (int j = 0; j < 4; ++j) {
+                                const int kk = 64 * a + 16 * j + 2 * q;
+                                int gk[4] = {gis[kk], gis[kk + 1], gis[kk + 8], gis[kk + 9]};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    if (gk[e] < 0 || gk[e] >= p.G) {
+                                        atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
+                                        gk[e] = 0;
+                                    }
+                                uint32_t af[4];
+#pragma unroll
+                                for (int r = 0; r < 4; ++r) {
+                                    const int row = (r & 1) ? n_r1 : n_r0;
+                                    const int kl = (r & 2) ? 2 : 0;
+                                    const float qlo = (float)((wv[j] >> (4 * r)) & 0xF);
+                                    const float qhi = (float)((wv[j] >> (4 * (r + 4))) & 0xF);
+                                    const __half z_lo = p.zeros ? __ldg(p.zeros + (size_t)gk[kl] * p.N + row)
+                                                                : __float2half_rn(8.0f);
+                                    const __half z_hi = p.zeros ? __ldg(p.zeros + (size_t)gk[kl + 1] * p.N + row)
+                                                                : __float2half_rn(8.0f);
+                                    const __half2 ss = __halves2half2(__ldg(p.scales + (size_t)gk[kl] * p.N + row),
+                                                                      __ldg(p.scales + (size_t)gk[kl + 1] * p.N + row));
+                                    af[r] = h2_as_u32(__hmul2(
+                                        __hsub2(__floats2half2_rn(qlo, qhi), __halves2half2(z_lo, z_hi)), ss));
+                                }
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    const uint32_t b0 = lds32(xa + xrow + nt * 1024 + xlo[j]);
+                                    const uint32_t b1 = lds32(xa + xrow + nt * 1024 + xhi[j]);
+                                    mma_16816<false>(acc[nt], af, b0, b1);
+                                }
                             }
-                        auto sc_of = [&](int g, int n) {
-                            return __ldg(p.scales + (size_t)g * p.N + n);
-                        };
-                        auto z_of = [&](int g, int n) {
-                            return p.zeros ? __ldg(p.zeros + (size_t)g * p.N + n) : __float2half_rn(8.0f);
-                        };
-                        const uint32_t wj = wv[j];
-                        // codes in the order of the A registers: (r0: c,c+1) (r1: c,c+1)
-                        // (r0: c+8,c+9) (r1: c+8,c+9) = nibbles (0,4) (1,5) (2,6) (3,7)
-                        uint32_t af[4];
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int row = (r & 1) ? n_r1 : n_r0;
-                            const int klo = (r & 2) ? 2 : 0;   // index into gk
-                            const float qlo = (float)((wj >> (4 * r)) & 0xF);
-                            const float qhi = (float)((wj >> (4 * (r + 4))) & 0xF);
-                            const __half2 qq = __floats2half2_rn(qlo, qhi);
-                            const __half2 zz = __halves2half2(z_of(gk[klo], row), z_of(gk[klo + 1], row));
-                            const __half2 ss = __halves2half2(sc_of(gk[klo], row), sc_of(gk[klo + 1], row));
-                            af[r] = h2_as_u32(__hmul2(__hsub2(qq, zz), ss));
-                        }
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            const int tok = 8 * nt + g8;
-                            uint32_t b0 = 0, b1 = 0;
-                            if (tok < p.M) {
-                                const unsigned char* xr = xb + tok * kXRow + (16 * j + 2 * q) * 2;
-                                b0 = lds32(xr);
-                                b1 = lds32(xr + 16);
-                            }
-                            mma_16816<false>(acc[nt], af, b0, b1);
                         }
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
+            u += na;
         }
         if (cur_band >= 0)
-            flush_band<NT>(p, cur_band, u0, u1, cta, w, lane, ctid,
-                           cur_band * kWarps + w < p.tiles, aborted, acc, s_last);
+            flush_band<NT>(p, cur_band, u0, u1, cta, w, lane, ctid, aborted, acc, s_last);
     }
 }
 

@@ -36,13 +36,15 @@ constexpr int kTmemCols = 256; // two fp32 partial buffers of BM columns
 constexpr int kABytes = BN * BK * 2;   // 16 KB
 constexpr int kBBytes = BM * BK * 2;   // 16 KB
 constexpr int kPBytes = BN * BK / 2;   // 4 KB packed codes
-constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+constexpr int kZBytes = 2 * BN * 2;    // zero-point rows of up to two groups
+constexpr int kStageBytes = kABytes + kBBytes + kPBytes + kZBytes;
 
 struct SmemLayout {
     static constexpr int a = 0;                              // kStages x 16 KB (1024-aligned)
     static constexpr int b = a + kStages * kABytes;          // kStages x 16 KB
     static constexpr int pk = b + kStages * kBBytes;         // kStages x 4 KB
-    static constexpr int bars = pk + kStages * kPBytes;      // barriers
+    static constexpr int zr = pk + kStages * kPBytes;        // kStages x 512 B
+    static constexpr int bars = zr + kStages * kZBytes;      // barriers
     static constexpr int nbars = 3 * kStages + 4 + 1;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int flags = tmem_slot + 8;
@@ -206,17 +208,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            // this CTA's 128 rows are band blockIdx.x; its codes for column block kt are
+            // one contiguous run of tiles x 512 bytes
+            const int band = blockIdx.x;
             const int tiles = min(BN / 16, p.tiles - n0 / 16);
-            const uint32_t bytes = kBBytes + tiles * 512;
+            const int zgroups = (!GIDX && p.zeros) ? (g == 32 ? 2 : 1) : 0;
+            const uint32_t bytes = kBBytes + tiles * 512 + zgroups * tiles * 32;
             int issued = 0;
             for (int kt = 0; kt < KT; ++kt, ++issued) {
                 const int s = kt % kStages, ph = (kt / kStages) & 1;
                 if (kt >= kStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 tma_load_2d(smem + L::b + s * kBBytes, &tmap_x, kt * BK, m0, &full[s]);
-                for (int t = 0; t < tiles; ++t)
-                    bulk_g2s(smem + L::pk + s * kPBytes + t * 512,
-                             p.qw + ((size_t)(n0 / 16 + t) * p.KA + kt) * 128, 512, &full[s]);
+                bulk_g2s(smem + L::pk + s * kPBytes,
+                         p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)kt * tiles), tiles * 512,
+                         &full[s]);
+                for (int zg = 0; zg < zgroups; ++zg)
+                    bulk_g2s(smem + L::zr + s * kZBytes + zg * BN * 2,
+                             p.zeros + (size_t)((kt * BK) / g + zg) * p.N + n0, tiles * 32, &full[s]);
             }
             if (*abort_flag)
                 for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
@@ -278,6 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_or_abort(&full[s], ph, abort_flag)) break;
             unsigned char* a_tile = smem + L::a + s * kABytes;
             const unsigned char* pk = smem + L::pk + s * kPBytes;
+            const __half* zs = reinterpret_cast<const __half*>(smem + L::zr + s * kZBytes);
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
                 const int t = 2 * dq + tt;
@@ -292,11 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int kabs = kt * BK + kk;
                     uint32_t af[4];
                     if constexpr (!GIDX) {
-                        const int grp = kabs / g;
+                        // zero points of this stage's group(s), staged by the producer
+                        const int zg = (g == 32) ? (j >> 1) : 0;
                         float z0 = 8.0f, z1 = 8.0f;
                         if (p.zeros) {
-                            z0 = __half2float(__ldg(p.zeros + (size_t)grp * p.N + nr0));
-                            z1 = __half2float(__ldg(p.zeros + (size_t)grp * p.N + nr1));
+                            z0 = __half2float(zs[zg * BN + r0]);
+                            z1 = __half2float(zs[zg * BN + r1]);
                         }
                         const ZeroConsts zc = BF16 ? zero_consts_bf16(z0, z1) : zero_consts_f16(z0, z1);
                         unpack_word<BF16>(wv[j], zc, af);

@@ -121,10 +121,14 @@ __global__ void __launch_bounds__(kThreads) quantize_pack_kernel(QuantParams p) 
     }
     __syncthreads();
 
-    // pass 3: quantise and pack, one device-layout word per thread iteration
+    // pass 3: quantise and pack, one device-layout word per thread iteration.  Row tile
+    // t = blockIdx.x is tile tt of band b; its atom for column block a is atom
+    // 8*(K/64)*b + a*Tb + tt (Tb = tiles in the band).
     const int KA = p.K / 64;
     const int words = KA * 128;
-    uint32_t* out = p.qweight + (size_t)blockIdx.x * words;
+    const int T = p.N / 16, b = blockIdx.x >> 3, tt = blockIdx.x & 7;
+    const int Tb = min(8, T - 8 * b);
+    uint32_t* out = p.qweight + (size_t)128 * ((size_t)8 * KA * b + tt);
     for (int wi = tid; wi < words; wi += kThreads) {
         const int a = wi >> 7, inw = wi & 127;
         const int L = inw >> 2, j = inw & 3;
@@ -147,11 +151,14 @@ __global__ void __launch_bounds__(kThreads) quantize_pack_kernel(QuantParams p) 
             }
             word |= qv << (4 * i);
         }
-        out[wi] = word;
+        out[(size_t)128 * a * Tb + inw] = word;
     }
 }
 
-// Device layout -> canonical layout (uint32 [N, K/8], nibble j of word i = q[n][8i+j]).
+// Device layout -> canonical layout (uint32 [N, K/8], nibble j of word i = q[n][8i+j]):
+// code (n, k) sits in atom 8*(K/64)*b + a*Tb + tt of band b = n/128 (tile tt = (n/16)%8,
+// column block a = k/64), word 4L + j with L = 4*(n%8) + (k%8)/2, j = (k%64)/16, nibble
+// ((n%16)>=8) + 2*((k%16)>=8) + 4*(k%2).
 __global__ void unpack_canonical_kernel(const uint32_t* __restrict__ qd, int N, int K,
                                         uint32_t* __restrict__ qc) {
     const int KW = K / 8, KA = K / 64;
@@ -160,6 +167,7 @@ __global__ void unpack_canonical_kernel(const uint32_t* __restrict__ qd, int N, 
          idx += (size_t)gridDim.x * blockDim.x) {
         const int n = (int)(idx / KW), i = (int)(idx % KW);
         const int t = n >> 4, rr = n & 15, half = rr >> 3, rg = rr & 7;
+        const int b = t >> 3, tt = t & 7, Tb = min(8, N / 16 - 8 * b);
         uint32_t out = 0;
         for (int jn = 0; jn < 8; ++jn) {
             const int k = 8 * i + jn;
@@ -167,7 +175,7 @@ __global__ void unpack_canonical_kernel(const uint32_t* __restrict__ qd, int N, 
             const int hi8 = cc >> 3, odd = cc & 1, cpair = (cc & 7) >> 1;
             const int L = 4 * rg + cpair;
             const int nib = half + 2 * hi8 + 4 * odd;
-            const uint32_t w = qd[(size_t)128 * ((size_t)t * KA + a) + 4 * L + j];
+            const uint32_t w = qd[(size_t)128 * ((size_t)8 * KA * b + (size_t)a * Tb + tt) + 4 * L + j];
             out |= ((w >> (4 * nib)) & 0xFu) << (4 * jn);
         }
         qc[idx] = out;

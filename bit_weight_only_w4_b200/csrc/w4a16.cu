@@ -1,6 +1,7 @@
 // w4a16.cu -- C ABI of the W4A16 library (declared in include/w4a16.h): argument
 // validation, kernel selection by M and launches.  All device work is in the kernels of
 // w4_quant.cuh, w4_decode.cuh and w4_prefill.cuh; nothing here touches tensor data.
+#include <algorithm>
 #include <climits>
 #include <cstring>
 #include <mutex>
@@ -67,29 +68,6 @@ bool ensure_smem(Kernel k, int bytes, std::once_flag (&flags)[kMaxDevices], int 
 // ---------------------------------------------------------------- decode launch plan
 int decode_tiles_for(int64_t M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 
-template <int NT, bool BF16, bool GIDX>
-struct DecodeKernel {
-    static constexpr int smem = w4d::SmemLayout<NT>::bytes;
-    static int ctas_per_sm[kMaxDevices];
-    static std::once_flag occ_flags[kMaxDevices];
-    static int occupancy(int dev) {
-        std::call_once(occ_flags[dev], [&] {
-            int b = 0;
-            cudaFuncSetAttribute(w4d::decode_kernel<NT, BF16, GIDX>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &b, w4d::decode_kernel<NT, BF16, GIDX>, w4d::kThreads, smem) != cudaSuccess)
-                b = 1;
-            ctas_per_sm[dev] = b < 1 ? 1 : (b > kDecodeMaxCtasPerSm ? kDecodeMaxCtasPerSm : b);
-        });
-        return ctas_per_sm[dev];
-    }
-};
-template <int NT, bool BF16, bool GIDX>
-int DecodeKernel<NT, BF16, GIDX>::ctas_per_sm[kMaxDevices];
-template <int NT, bool BF16, bool GIDX>
-std::once_flag DecodeKernel<NT, BF16, GIDX>::occ_flags[kMaxDevices];
-
 // Split-K fix-up counters live in a fixed region at the start of the workspace, one per
 // 128-row band, so that every call -- whatever its N -- finds its counters where earlier
 // calls left them at zero; the partial-sum slots follow the region.
@@ -101,34 +79,17 @@ size_t decode_workspace_bytes(int64_t M, int sms) {
     return kCounterBytes + partials;
 }
 
-template <int NT, bool BF16, bool GIDX>
-w4_status launch_decode(w4d::DecodeParams p, unsigned char* ws, int dev, cudaStream_t stream) {
-    using DK = DecodeKernel<NT, BF16, GIDX>;
-    const int per_sm = DK::occupancy(dev);
-    const int bands = (p.tiles + w4d::kWarps - 1) / w4d::kWarps;
-    p.units = bands * p.KA;
-    int P = sm_count(dev) * per_sm;
-    if (P <= 0) return W4_ERR_CUDA;
-    if (P > p.units) P = p.units;
-    p.base = p.units / P;
-    p.rem = p.units % P;
-    p.counters = reinterpret_cast<unsigned*>(ws);
-    p.partials = reinterpret_cast<float*>(ws + kCounterBytes);
-    w4d::decode_kernel<NT, BF16, GIDX><<<P, w4d::kThreads, DK::smem, stream>>>(p);
-    return launch_status();
+int smem_per_sm(int dev) {
+    static int cache[kMaxDevices];
+    static std::once_flag flags[kMaxDevices];
+    std::call_once(flags[dev], [&] {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        cache[dev] = v;
+    });
+    return cache[dev];
 }
 
-template <bool BF16, bool GIDX>
-w4_status dispatch_decode(w4d::DecodeParams p, unsigned char* ws, int dev, cudaStream_t s) {
-    switch (decode_tiles_for(p.M)) {
-        case 1: return launch_decode<1, BF16, GIDX>(p, ws, dev, s);
-        case 2: return launch_decode<2, BF16, GIDX>(p, ws, dev, s);
-        case 4: return launch_decode<4, BF16, GIDX>(p, ws, dev, s);
-        default: return launch_decode<8, BF16, GIDX>(p, ws, dev, s);
-    }
-}
-
-// ---------------------------------------------------------------- prefill launch plan
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -147,12 +108,15 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-bool make_act_tensor_map(CUtensorMap* map, const void* X, bool bf16, int64_t M, int64_t K) {
+// 2-D map over activations [M,K] (K innermost) with boxes of 64 channels x box_rows rows,
+// 128-byte swizzle (the layout the tcgen05 descriptors expect).
+bool make_act_tensor_map(CUtensorMap* map, const void* X, bool bf16, int64_t M, int64_t K,
+                         int box_rows) {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)w4p::BK, (cuuint32_t)w4p::BM};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                const_cast<void*>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -160,6 +124,95 @@ bool make_act_tensor_map(CUtensorMap* map, const void* X, bool bf16, int64_t M, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view of activations [M,K] as (64 channels, M rows, K/64 column blocks): one box of
+// 4 column blocks x box_rows rows lands as [block][row][64], each row a 128-byte swizzled
+// line; rows >= M and blocks beyond K/64 are zero-filled.
+bool make_act_blocks_map(CUtensorMap* map, const void* X, bool bf16, int64_t M, int64_t K,
+                         int box_rows, int blocks) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, (cuuint32_t)blocks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+               const_cast<void*>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over fp16 group metadata [G,N] (N innermost): boxes of 128 columns x rows groups.
+bool make_meta_map(CUtensorMap* map, const void* base, int64_t G, int64_t N, int rows) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)G};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    const cuuint32_t box[2] = {128u, (cuuint32_t)rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NT, bool BF16, bool GIDX>
+w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
+                        cudaStream_t stream) {
+    using C = w4d::Cfg<NT>;
+    static std::once_flag flags[kMaxDevices];
+    constexpr int kMaxSmem = 227 * 1024;
+    bool attr_ok = true;
+    std::call_once(flags[dev], [&] {
+        attr_ok = cudaFuncSetAttribute(w4d::decode_kernel<NT, BF16, GIDX>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxSmem) == cudaSuccess;
+    });
+    if (!attr_ok) return W4_ERR_CUDA;
+    // stage layout: codes | activation boxes | s_inv | scale rows | zero rows | g_idx
+    const int g = p.group_size;
+    p.ngs = GIDX ? 0 : (g == 32 ? 8 : std::min(p.G, (256 + 2 * g - 65) / g));
+    p.off_x = w4d::kAtomsPerStage * w4d::kWarps * 512;
+    p.off_si = p.off_x + w4d::kAtomsPerStage * C::xbox;
+    p.off_sc = p.off_si + (p.s_inv ? 1024 : 0);
+    p.off_zr = p.off_sc + p.ngs * 256;
+    p.off_gi = p.off_zr + (p.zeros ? p.ngs * 256 : 0);
+    p.stage_bytes = (p.off_gi + (GIDX ? 1024 : 0) + 1023) / 1024 * 1024;
+    const int smem = C::stages * p.stage_bytes + 2 * C::stages * 8 + 16 + 1024;
+    if (smem > kMaxSmem) return W4_ERR_UNSUPPORTED;
+    int per_sm = NT >= 8 ? 1 : std::min(kDecodeMaxCtasPerSm, smem_per_sm(dev) / (smem + 1024));
+    if (per_sm < 1) per_sm = 1;
+    const int bands = (p.tiles + w4d::kWarps - 1) / w4d::kWarps;
+    p.units = bands * p.KA;
+    int P = sm_count(dev) * per_sm;
+    if (P <= 0) return W4_ERR_CUDA;
+    if (P > p.units) P = p.units;
+    p.base = p.units / P;
+    p.rem = p.units % P;
+    p.counters = reinterpret_cast<unsigned*>(ws);
+    p.partials = reinterpret_cast<float*>(ws + kCounterBytes);
+    CUtensorMap map_x, map_sc, map_zr;
+    if (!make_act_blocks_map(&map_x, X, BF16, p.M, p.K, C::mpad, w4d::kAtomsPerStage)) return W4_ERR_CUDA;
+    map_sc = map_x;
+    map_zr = map_x;
+    if (!GIDX) {
+        if (!make_meta_map(&map_sc, p.scales, p.G, p.N, p.ngs)) return W4_ERR_CUDA;
+        if (p.zeros && !make_meta_map(&map_zr, p.zeros, p.G, p.N, p.ngs)) return W4_ERR_CUDA;
+    }
+    w4d::decode_kernel<NT, BF16, GIDX><<<P, w4d::kThreads, smem, stream>>>(map_x, map_sc, map_zr, p);
+    return launch_status();
+}
+
+template <bool BF16, bool GIDX>
+w4_status dispatch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
+                          cudaStream_t s) {
+    switch (decode_tiles_for(p.M)) {
+        case 1: return launch_decode<1, BF16, GIDX>(p, X, ws, dev, s);
+        case 2: return launch_decode<2, BF16, GIDX>(p, X, ws, dev, s);
+        case 4: return launch_decode<4, BF16, GIDX>(p, X, ws, dev, s);
+        default: return launch_decode<8, BF16, GIDX>(p, X, ws, dev, s);
+    }
+}
+
+// ---------------------------------------------------------------- prefill launch plan
 template <bool BF16, bool GIDX>
 w4_status launch_prefill(const CUtensorMap& map, const w4p::PrefillParams& p, int dev,
                          cudaStream_t stream) {
@@ -272,8 +325,7 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
     if (!prefill) {
         w4d::DecodeParams p;
         std::memset(&p, 0, sizeof(p));
-        p.X = X;
-        p.qw = qweight;
+            p.qw = qweight;
         p.scales = reinterpret_cast<const __half*>(scales);
         p.zeros = reinterpret_cast<const __half*>(zeros);
         p.g_idx = g_idx;
@@ -288,9 +340,9 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
         p.KA = (int)(K / 64);
         p.tiles = (int)(N / 16);
         unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
-        if (bf16) return dispatch_decode<true, false>(p, ws, dev, strm);
-        return gidx ? dispatch_decode<false, true>(p, ws, dev, strm)
-                    : dispatch_decode<false, false>(p, ws, dev, strm);
+        if (bf16) return dispatch_decode<true, false>(p, X, ws, dev, strm);
+        return gidx ? dispatch_decode<false, true>(p, X, ws, dev, strm)
+                    : dispatch_decode<false, false>(p, X, ws, dev, strm);
     }
 
     const void* Xeff = X;
@@ -304,7 +356,7 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
         Xeff = xp;
     }
     CUtensorMap map;
-    if (!make_act_tensor_map(&map, Xeff, bf16, M, K)) return W4_ERR_CUDA;
+    if (!make_act_tensor_map(&map, Xeff, bf16, M, K, w4p::BM)) return W4_ERR_CUDA;
     w4p::PrefillParams p;
     std::memset(&p, 0, sizeof(p));
     p.qw = qweight;
@@ -439,7 +491,6 @@ extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64
 
     w4d::DecodeParams p;
     std::memset(&p, 0, sizeof(p));
-    p.X = X;
     p.qw = qweight;
     p.scales = reinterpret_cast<const __half*>(scales);
     p.zeros = reinterpret_cast<const __half*>(zeros);
@@ -455,7 +506,7 @@ extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64
     p.KA = (int)(K / 64);
     p.tiles = (int)(N / 16);
     cudaStream_t strm = as_stream(stream);
-    if (bf16) return dispatch_decode<true, false>(p, ws, dev, strm);
-    return gidx ? dispatch_decode<false, true>(p, ws, dev, strm)
-                : dispatch_decode<false, false>(p, ws, dev, strm);
+    if (bf16) return dispatch_decode<true, false>(p, X, ws, dev, strm);
+    return gidx ? dispatch_decode<false, true>(p, X, ws, dev, strm)
+                : dispatch_decode<false, false>(p, X, ws, dev, strm);
 }

@@ -35,15 +35,18 @@
  *
  * Packed weight format ("device layout")
  *  The INT4 codes q[n][k] in [0,15] of W [N,K] are stored as N*K/8 uint32 words in
- *  tiles of 16 rows x 64 columns.  Tile (t, a) -- rows 16t..16t+15, columns
- *  64a..64a+63 -- occupies the 128 words starting at word 128*(t*(K/64) + a).  Word
- *  4L+j of a tile (L = 0..31, j = 0..3) holds, with r0 = 16t + L/4, r1 = r0 + 8,
+ *  atoms of 16 rows x 64 columns (128 words).  Eight consecutive row tiles form a band of
+ *  128 rows (the last band holds Tb = min(8, N/16 - 8b) tiles).  Band b starts at atom
+ *  8*(K/64)*b; inside it the atom of row tile tt (rows 16(8b+tt)..+15) and column block a
+ *  (columns 64a..64a+63) is atom a*Tb + tt, i.e. a band is stored column block by column
+ *  block, so consecutive column blocks of a band are one contiguous run.  Word 4L+j of an
+ *  atom (L = 0..31, j = 0..3) holds, with t = 8b+tt, r0 = 16t + L/4, r1 = r0 + 8,
  *  kb = 64a + 16j, c = 2*(L%4), nibble i in bits 4i..4i+3:
  *     nibble 0: q[r0][kb+c]     nibble 4: q[r0][kb+c+1]
  *     nibble 1: q[r1][kb+c]     nibble 5: q[r1][kb+c+1]
  *     nibble 2: q[r0][kb+c+8]   nibble 6: q[r0][kb+c+9]
  *     nibble 3: q[r1][kb+c+8]   nibble 7: q[r1][kb+c+9]
- *  Lane L of a warp loads words 4L..4L+3 of a tile with one 16-byte load; each word is
+ *  Lane L of a warp loads words 4L..4L+3 of an atom with one 16-byte load; each word is
  *  then exactly the 16x16 weight operand slice that lane needs for one 16-deep step of
  *  a warp-level MMA, and the eight codes come out as fp16/bf16 pairs with one
  *  AND/OR per pair (the exponent-bias trick) plus one subtract.

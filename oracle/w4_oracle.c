@@ -256,21 +256,25 @@ void oracle_unpack_canonical(const uint32_t* qc, int64_t N, int64_t K, uint8_t* 
 
 /* ------------------------------------------------------------------ */
 /* Device packing (the library's own layout; N % 16 == 0, K % 64 == 0).  */
-/* The weight matrix is cut into tiles of 16 rows x 64 columns; tile     */
-/* (t, a) covers rows 16t..16t+15 and columns 64a..64a+63 and occupies   */
-/* 128 consecutive words starting at word 128*(t*(K/64) + a).  Inside a  */
-/* tile, word 4*L + j (L = 0..31, j = 0..3) holds, for r0 = 16t + L/4,   */
-/* r1 = r0 + 8, kb = 64a + 16j, c = 2*(L%4), the eight codes              */
+/* The weight matrix is cut into atoms of 16 rows x 64 columns.  Eight   */
+/* consecutive row tiles form a band of 128 rows (the last band holds    */
+/* Tb = min(8, N/16 - 8b) tiles).  Band b starts at atom 8*(K/64)*b and  */
+/* inside it atom (tile tt of the band, column block a) is atom           */
+/* a*Tb + tt; atom i occupies words 128*i .. 128*i+127.  Inside an atom,  */
+/* word 4*L + j (L = 0..31, j = 0..3) holds, for r0 = 16t + L/4 (t the    */
+/* tile's row index), r1 = r0 + 8, kb = 64a + 16j, c = 2*(L%4), the codes */
 /*   nibble 0: q[r0][kb+c]    nibble 4: q[r0][kb+c+1]                     */
 /*   nibble 1: q[r1][kb+c]    nibble 5: q[r1][kb+c+1]                     */
 /*   nibble 2: q[r0][kb+c+8]  nibble 6: q[r0][kb+c+9]                     */
 /*   nibble 3: q[r1][kb+c+8]  nibble 7: q[r1][kb+c+9]                     */
 /* with nibble i in bits 4i..4i+3.                                        */
 /* ------------------------------------------------------------------ */
-static void device_slot(int64_t K, int64_t word, int nib, int64_t* n, int64_t* k) {
-    int64_t KA = K / 64;
-    int64_t tile = word / 128, inw = word % 128;
-    int64_t t = tile / KA, a = tile % KA;
+static void device_slot(int64_t N, int64_t K, int64_t word, int nib, int64_t* n, int64_t* k) {
+    int64_t KA = K / 64, T = N / 16;
+    int64_t atom = word / 128, inw = word % 128;
+    int64_t b = atom / (8 * KA), in_band = atom % (8 * KA);
+    int64_t Tb = (T - 8 * b) < 8 ? (T - 8 * b) : 8;
+    int64_t a = in_band / Tb, t = 8 * b + in_band % Tb;
     int64_t L = inw / 4, j = inw % 4;
     int64_t r0 = 16 * t + L / 4, c = 2 * (L % 4), kb = 64 * a + 16 * j;
     static const int row_hi[8] = {0, 1, 0, 1, 0, 1, 0, 1};
@@ -286,7 +290,7 @@ int oracle_pack_device(const uint8_t* q, int64_t N, int64_t K, uint32_t* qd) {
         uint32_t v = 0;
         for (int i = 0; i < 8; ++i) {
             int64_t n, k;
-            device_slot(K, w, i, &n, &k);
+            device_slot(N, K, w, i, &n, &k);
             v |= (uint32_t)(q[n * K + k] & 0xF) << (4 * i);
         }
         qd[w] = v;
@@ -300,7 +304,7 @@ int oracle_unpack_device(const uint32_t* qd, int64_t N, int64_t K, uint8_t* q) {
     for (int64_t w = 0; w < words; ++w)
         for (int i = 0; i < 8; ++i) {
             int64_t n, k;
-            device_slot(K, w, i, &n, &k);
+            device_slot(N, K, w, i, &n, &k);
             q[n * K + k] = (uint8_t)((qd[w] >> (4 * i)) & 0xF);
         }
     return 0;

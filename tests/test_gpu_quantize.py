@@ -73,9 +73,10 @@ def test_quantize_config_layers(config_id, layer, g):
     run_and_compare(li.W.view(np.uint16), li.s, li.group_size, li.symmetric, li.g_idx)
 
 
-def test_quantize_70b_gate_up_sampled_tiles():
+def test_quantize_70b_gate_up_sampled_bands():
     """The largest layer (57344 x 8192): GPU over the whole matrix, oracle on sampled
-    16-row tiles (first, last and seeded random ones)."""
+    128-row bands (first, last and seeded random ones); a band's packed words are one
+    contiguous run of the device layout."""
     skip_without_gpu()
     import torch
     wl = workloads.workload(3)
@@ -84,12 +85,12 @@ def test_quantize_70b_gate_up_sampled_tiles():
     qw, sc, zr = w4.w4_quantize_pack(dev_bits(li.W.view(np.uint16), torch.float16), dev(li.s), g)
     torch.cuda.synchronize()
     rng = np.random.default_rng(3)
-    tiles = sorted(set([0, N // 16 - 1] + rng.integers(0, N // 16, 6).tolist()))
-    words = K // 64 * 128
+    bands = sorted(set([0, N // 128 - 1] + rng.integers(0, N // 128, 4).tolist()))
+    words = K // 64 * 128 * 8
     qw_h, sc_h, zr_h = host_u32(qw), host_bits(sc), host_bits(zr)
-    for t in tiles:
-        rows = slice(16 * t, 16 * t + 16)
+    for b in bands:
+        rows = slice(128 * b, 128 * b + 128)
         q, s_ref, z_ref = oracle.quantize_weights(li.W.view(np.uint16)[rows], li.s, g)
-        assert np.array_equal(qw_h[t * words:(t + 1) * words], oracle.pack_device(q))
+        assert np.array_equal(qw_h[b * words:(b + 1) * words], oracle.pack_device(q))
         assert np.array_equal(sc_h[:, rows], s_ref)
         assert np.array_equal(zr_h[:, rows], z_ref)

@@ -31,6 +31,8 @@ def _pattern(name, N, K):
         q = np.broadcast_to(r % 16, (N, K))
     elif name == "tile":
         q = 4 * (r // 16) + k // 64
+    elif name == "band":
+        q = (r // 16 + 3 * (k // 64)) % 16
     else:
         raise KeyError(name)
     return np.ascontiguousarray(q, dtype=np.uint8)
@@ -58,7 +60,7 @@ def test_pack_golden_words(case):
         assert qd[int(idx)] == word, hex(int(qd[int(idx)]))
 
 
-@pytest.mark.parametrize("N,K", [(16, 64), (48, 192), (32, 4096)])
+@pytest.mark.parametrize("N,K", [(16, 64), (48, 192), (32, 4096), (160, 128), (272, 320)])
 def test_pack_round_trips(N, K):
     rng = np.random.default_rng(N + K)
     q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
