@@ -78,6 +78,13 @@ W4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Let the next kernel on the stream (launched with programmatic stream serialization)
+// start its prologue while this grid finishes.
+W4_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Wait until the preceding grid has completed and its memory operations are visible.
+W4_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- named barriers
 W4_DEV void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -198,6 +205,33 @@ W4_DEV ZeroConsts zero_consts_bf16(float z0, float z1) {
     zc.lo1 = b2_as_u32(__float2bfloat162_rn(128.0f + z1));
     zc.hi0 = zc.lo0;
     zc.hi1 = zc.lo1;
+    return zc;
+}
+
+// The same constants straight from the fp16 zero points (integers 0..15) of rows r0 / r1,
+// with fp16 arithmetic and byte permutes only (no type conversions):
+//   s = (1024 + z0, 1024 + z1)   exact in fp16, and its low mantissa nibbles are z0, z1;
+//   fp16: lo0 = (1024 + z0) x2, hi1 = (960 - (1024 + z1)) x2 = -(64 + z1) x2;
+//   bf16: lo0 = 0x4300 | z0 (x2), lo1 = 0x4300 | z1 (x2)   (128 + z in bf16).
+// The symmetric format's implicit zero point is z = 8 (fp16 bits 0x4800).
+template <bool BF16>
+W4_DEV ZeroConsts zero_consts_h(uint32_t z0_bits, uint32_t z1_bits) {
+    const uint32_t zz = __byte_perm(z0_bits, z1_bits, 0x5410);              // (z0, z1)
+    const uint32_t s = h2_as_u32(__hadd2(u32_as_h2(zz), u32_as_h2(0x64006400u)));
+    ZeroConsts zc;
+    if constexpr (!BF16) {
+        const uint32_t t = h2_as_u32(__hsub2(u32_as_h2(0x63806380u), u32_as_h2(s)));
+        zc.lo0 = __byte_perm(s, 0, 0x1010);
+        zc.lo1 = __byte_perm(s, 0, 0x3232);
+        zc.hi0 = __byte_perm(t, 0, 0x1010);
+        zc.hi1 = __byte_perm(t, 0, 0x3232);
+    } else {
+        const uint32_t z0 = s & 0xFu, z1 = (s >> 16) & 0xFu;
+        zc.lo0 = 0x43004300u | z0 | (z0 << 16);
+        zc.lo1 = 0x43004300u | z1 | (z1 << 16);
+        zc.hi0 = zc.lo0;
+        zc.hi1 = zc.lo1;
+    }
     return zc;
 }
 

@@ -141,6 +141,10 @@ W4_DEV void flush_band(const DecodeParams& p, int band, int u0, int u1, int cta,
     if (*s_flag) {
         __threadfence();
         if (tile_ok) {
+            // Only the first contributor can hold this band in its second slot (its range
+            // began in an earlier band); every later one began inside this band.
+            const int first_slot = (unit_begin(p, c_first) < band * p.KA) ? 1 : 0;
+            const size_t slot_elems = (size_t)kBandRows * Mp;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -148,11 +152,19 @@ W4_DEV void flush_band(const DecodeParams& p, int band, int u0, int u1, int cta,
                     const int m = 8 * nt + q2 + (e & 1);
                     const int rl = rl0 + ((e >> 1) << 3);
                     if (m >= p.M) continue;
+                    const float* base = p.partials + rl * Mp + m;
                     float v = 0.0f;
-                    for (int c = c_first; c <= c_last; ++c) {
-                        const int wc = (unit_begin(p, c) / p.KA == band) ? 0 : 1;
-                        v += __ldcg(p.partials + ((size_t)c * 2 + wc) * (size_t)(kBandRows * Mp) +
-                                    rl * Mp + m);
+                    // contributors in CTA order, loads issued a batch at a time
+                    for (int cb = c_first; cb <= c_last; cb += 8) {
+                        float part[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int c = cb + t;
+                            const int wc = (c == c_first) ? first_slot : 0;
+                            part[t] = (c <= c_last) ? __ldcg(base + ((size_t)c * 2 + wc) * slot_elems) : 0.0f;
+                        }
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) v += part[t];
                     }
                     store_out(p, m, band * kBandRows + rl, v);
                 }
@@ -168,6 +180,80 @@ W4_DEV void fold(float s0, float s1, float (&c)[4], float (&acc)[4]) {
     acc[2] = fmaf(s1, c[2], acc[2]);
     acc[3] = fmaf(s1, c[3], acc[3]);
     c[0] = c[1] = c[2] = c[3] = 0.0f;
+}
+
+// One stage of the decode consumer (contiguous groups): the warp's 16-row tile times
+// up to kAtomsPerStage column blocks staged at `st`; partial sums of each group are
+// folded into acc with the group's fp32 scale.  nb = first column of the next group.
+template <int NT, bool BF16>
+W4_DEV void consume_stage(const unsigned char* st, int off_x, int off_sc, int off_zr, bool has_zeros,
+                          int na, int a0, int tb, int nb, int g, bool g32, int w, int lane,
+                          int rl0, int rl1, uint32_t xrow, const int (&xlo)[4], const int (&xhi)[4],
+                          const ZeroConsts& zc_sym, float (&acc)[NT][4]) {
+    using C = Cfg<NT>;
+    const __half* scp = reinterpret_cast<const __half*>(st + off_sc);
+    const unsigned short* zrp = reinterpret_cast<const unsigned short*>(st + off_zr);
+    float s0 = __half2float(scp[rl0]), s1 = __half2float(scp[rl1]);
+    ZeroConsts zc = has_zeros ? zero_consts_h<BF16>(zrp[rl0], zrp[rl1]) : zc_sym;
+    // two accumulator chains (even / odd 16-deep steps) for MMA overlap
+    float c0[NT][4], c1[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c0[nt][e] = c1[nt][e] = 0.0f;
+    // per-stage fragment base addresses: every load below is one of these registers plus
+    // a compile-time offset
+    uint32_t xl[4], xh[4];
+    const uint32_t xs = smem_u32(st + off_x) + xrow;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        xl[j] = xs + xlo[j];
+        xh[j] = xs + xhi[j];
+    }
+    const unsigned char* wbase = st + w * 512 + lane * 16;
+    const int wstride = tb * 512;
+    int ka = 64 * a0;
+#pragma unroll
+    for (int a = 0; a < kAtomsPerStage; ++a) {
+        if (a < na) {
+            const uint4 wq = *reinterpret_cast<const uint4*>(wbase + a * wstride);
+            const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if ((j == 0 || (j == 2 && g32)) && ka + 16 * j >= nb) {
+                    // group boundary: fold the finished group's partials, load the next
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        fold(s0, s1, c0[nt], acc[nt]);
+                        fold(s0, s1, c1[nt], acc[nt]);
+                    }
+                    nb += g;
+                    scp += 128;
+                    zrp += 128;
+                    s0 = __half2float(scp[rl0]);
+                    s1 = __half2float(scp[rl1]);
+                    if (has_zeros) zc = zero_consts_h<BF16>(zrp[rl0], zrp[rl1]);
+                }
+                uint32_t af[4];
+                unpack_word<BF16>(wv[j], zc, af);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    // token rows >= M were zero-filled by the tensor copy
+                    const uint32_t b0 = lds32_at(xl[j] + a * C::xbox + nt * 1024);
+                    const uint32_t b1 = lds32_at(xh[j] + a * C::xbox + nt * 1024);
+                    // with few token tiles a second chain breaks the MMA dependency; with
+                    // more tiles they already interleave
+                    mma_16816<BF16>((NT <= 2 && (j & 1)) ? c1[nt] : c0[nt], af, b0, b1);
+                }
+            }
+            ka += 64;
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        fold(s0, s1, c0[nt], acc[nt]);
+        fold(s0, s1, c1[nt], acc[nt]);
+    }
 }
 
 template <int NT, bool BF16, bool GIDX>
@@ -206,6 +292,10 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
         }
     }
     __syncthreads();
+    // The next kernel may be scheduled as soon as every CTA of this grid is running.
+    // Everything this kernel reads before pdl_wait() (codes, scales, zero points, g_idx)
+    // is never written by the kernels of this library.
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -223,7 +313,9 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
             const int tb = band_tiles(p, band);
             // one copy per operand: codes (contiguous run of the band), activations (one
             // 3-D box: 4 column blocks x 8*NT token rows, rows >= M and blocks beyond K
-            // zero-filled), s_inv slice, scale rows and zero-point rows (2-D boxes)
+            // zero-filled), s_inv slice, scale rows and zero-point rows (2-D boxes).  The
+            // read-only weight operands of the first stages go out before pdl_wait(), the
+            // activations (possibly produced by the preceding kernel) after it.
             const int g_first = (64 * a0) / g;
             uint32_t bytes = na * tb * 512 + kAtomsPerStage * C::xbox;
             if (p.s_inv) bytes += na * 256;
@@ -233,14 +325,15 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
                 mbar_arrive_expect_tx(&full[s], bytes);
                 bulk_g2s_hint(st, p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)a0 * tb),
                               na * tb * 512, &full[s], policy);
-                tma_load_3d(st + p.off_x, &tmap_x, 0, 0, a0, &full[s]);
-                if (p.s_inv) bulk_g2s(st + p.off_si, p.s_inv + 64 * a0, na * 256, &full[s]);
                 if (GIDX) {
                     bulk_g2s(st + p.off_gi, p.g_idx + 64 * a0, na * 256, &full[s]);
                 } else {
                     tma_load_2d(st + p.off_sc, &tmap_sc, band * kBandRows, g_first, &full[s]);
                     if (p.zeros) tma_load_2d(st + p.off_zr, &tmap_zr, band * kBandRows, g_first, &full[s]);
                 }
+                if (i == 0) pdl_wait();
+                tma_load_3d(st + p.off_x, &tmap_x, 0, 0, a0, &full[s]);
+                if (p.s_inv) bulk_g2s(st + p.off_si, p.s_inv + 64 * a0, na * 256, &full[s]);
             }
             __syncwarp();
             u += na;
@@ -250,13 +343,14 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
             for (int k = (i > S ? i - S : 0); k < i; ++k) (void)mbar_wait(&full[k % S], (k / S) & 1);
     } else {
         // ------------------------------------------------------------ consumers
+        pdl_wait();   // before any store to Y or the workspace
         const int w = warp - 1;
         const int ctid = threadIdx.x - 32;
         const int q = lane & 3, g8 = lane >> 2;
         const int rl0 = 16 * w + g8, rl1 = rl0 + 8;
         // activation fragment offsets inside a 128B-swizzled box: row g8 (+8 per token
         // tile), k pairs 8j+q (b0) and 8j+4+q (b1) of the 16-deep step j
-        const int xrow = g8 * 128;
+        const uint32_t xrow = g8 * 128;
         int xlo[4], xhi[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -264,17 +358,23 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
             xhi[j] = (((2 * j + 1) ^ g8) << 4) + 4 * q;
         }
         const bool g32 = (g == 32);
+        // symmetric format: the implicit zero point 8 never changes
+        const ZeroConsts zc_sym = zero_consts_h<BF16>(0x4800u, 0x4800u);
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-        int cur_band = (u0 < u1) ? u0 / p.KA : -1;
+        // stage coordinates advance incrementally (one division per CTA)
+        int band = (u0 < u1) ? u0 / p.KA : 0;
+        int a0 = u0 - band * p.KA;
+        int cur_band = (u0 < u1) ? band : -1;
+        int gcur = (64 * a0) / g;          // group of the next column to process
+        int next_b = (gcur + 1) * g;       // first column of the following group
         bool aborted = false;
 
         int i = 0;
         for (int u = u0; u < u1; ++i) {
-            const int band = u / p.KA, a0 = u - band * p.KA;
             const int na = min(kAtomsPerStage, min(p.KA - a0, u1 - u));
             const int s = i % S, ph = (i / S) & 1;
             if (band != cur_band) {
@@ -312,80 +412,19 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
                 named_bar_sync(1, 32 * kWarps);
             }
             const int tb = band_tiles(p, band);
+            if (!GIDX) {
+                // the group containing this stage's first column (the staged scale and
+                // zero-point rows start there)
+                while (64 * a0 >= next_b) {
+                    next_b += g;
+                    ++gcur;
+                }
+            }
             if (!aborted && w < tb) {
                 if constexpr (!GIDX) {
-                    // group rows staged for this stage start at group g_first; later groups
-                    // begin at multiples of g (no division inside the loop)
-                    const int g_first = (64 * a0) / g;
-                    int next_b = (g_first + 1) * g;
-                    const __half* scp = reinterpret_cast<const __half*>(st + p.off_sc);
-                    const __half* zrp = reinterpret_cast<const __half*>(st + p.off_zr);
-                    float s0, s1;
-                    ZeroConsts zc;
-                    auto load_group = [&]() {
-                        s0 = __half2float(scp[rl0]);
-                        s1 = __half2float(scp[rl1]);
-                        const float z0 = p.zeros ? __half2float(zrp[rl0]) : 8.0f;
-                        const float z1 = p.zeros ? __half2float(zrp[rl1]) : 8.0f;
-                        zc = BF16 ? zero_consts_bf16(z0, z1) : zero_consts_f16(z0, z1);
-                    };
-                    load_group();
-                    // two accumulator chains (even / odd 16-deep steps) for MMA overlap
-                    float c0[NT][4], c1[NT][4];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) c0[nt][e] = c1[nt][e] = 0.0f;
-                    auto next_group = [&]() {
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            fold(s0, s1, c0[nt], acc[nt]);
-                            fold(s0, s1, c1[nt], acc[nt]);
-                        }
-                        next_b += g;
-                        scp += 128;
-                        zrp += 128;
-                        load_group();
-                    };
-                    // per-stage fragment base addresses: every load below is one of these
-                    // registers plus a compile-time offset
-                    uint32_t xl[4], xh[4];
-                    const uint32_t xs = smem_u32(xb) + xrow;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        xl[j] = xs + xlo[j];
-                        xh[j] = xs + xhi[j];
-                    }
-                    const unsigned char* wbase = st + w * 512 + lane * 16;
-#pragma unroll
-                    for (int a = 0; a < kAtomsPerStage; ++a) {
-                        if (a < na) {
-                            const int ka = 64 * (a0 + a);
-                            if (ka >= next_b) next_group();
-                            const uint4 wq = *reinterpret_cast<const uint4*>(wbase + a * tb * 512);
-                            const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                if (j == 2 && g32 && ka + 32 >= next_b) next_group();
-                                uint32_t af[4];
-                                unpack_word<BF16>(wv[j], zc, af);
-#pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    // token rows >= M were zero-filled by the tensor copy
-                                    const uint32_t b0 = lds32_at(xl[j] + a * C::xbox + nt * 1024);
-                                    const uint32_t b1 = lds32_at(xh[j] + a * C::xbox + nt * 1024);
-                                    // with few token tiles a second chain breaks the MMA
-                                    // dependency; with more tiles they already interleave
-                                    mma_16816<BF16>((NT <= 2 && (j & 1)) ? c1[nt] : c0[nt], af, b0, b1);
-                                }
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        fold(s0, s1, c0[nt], acc[nt]);
-                        fold(s0, s1, c1[nt], acc[nt]);
-                    }
+                    consume_stage<NT, BF16>(st, p.off_x, p.off_sc, p.off_zr, p.zeros != nullptr, na, a0,
+                                            tb, next_b, g, g32, w, lane, rl0, rl1, xrow, xlo, xhi,
+                                            zc_sym, acc);
                 } else {
                     // act-order: every channel has its own group; fold the scale into an
                     // fp16 weight (q - z) * scale before the MMA
@@ -438,6 +477,13 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
             u += na;
+            a0 += na;
+            if (a0 == p.KA) {
+                a0 = 0;
+                ++band;
+                gcur = 0;
+                next_b = g;
+            }
         }
         if (cur_band >= 0)
             flush_band<NT>(p, cur_band, u0, u1, cta, w, lane, ctid, aborted, acc, s_last);

@@ -204,6 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // The next kernel may be scheduled while this grid runs; codes and zero points, read
+    // before pdl_wait(), are never written by the kernels of this library.
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -219,13 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = kt % kStages, ph = (kt / kStages) & 1;
                 if (kt >= kStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
                 mbar_arrive_expect_tx(&full[s], bytes);
-                tma_load_2d(smem + L::b + s * kBBytes, &tmap_x, kt * BK, m0, &full[s]);
                 bulk_g2s(smem + L::pk + s * kPBytes,
                          p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)kt * tiles), tiles * 512,
                          &full[s]);
                 for (int zg = 0; zg < zgroups; ++zg)
                     bulk_g2s(smem + L::zr + s * kZBytes + zg * BN * 2,
                              p.zeros + (size_t)((kt * BK) / g + zg) * p.N + n0, tiles * 32, &full[s]);
+                if (kt == 0) pdl_wait();   // activations may come from the preceding kernel
+                tma_load_2d(smem + L::b + s * kBBytes, &tmap_x, kt * BK, m0, &full[s]);
             }
             if (*abort_flag)
                 for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
@@ -347,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue warps
+        pdl_wait();   // before any store to Y
         const int quad = warp & 3;                 // tensor-memory lanes 32*quad..
         const int row = 32 * quad + lane;          // output row within the tile
         const int n = n0 + row;

@@ -197,7 +197,21 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
         if (!make_meta_map(&map_sc, p.scales, p.G, p.N, p.ngs)) return W4_ERR_CUDA;
         if (p.zeros && !make_meta_map(&map_zr, p.zeros, p.G, p.N, p.ngs)) return W4_ERR_CUDA;
     }
-    w4d::decode_kernel<NT, BF16, GIDX><<<P, w4d::kThreads, smem, stream>>>(map_x, map_sc, map_zr, p);
+    // programmatic dependent launch: this kernel's prologue and weight loads may overlap
+    // the tail of the preceding kernel on the stream
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P);
+    cfg.blockDim = dim3(w4d::kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, w4d::decode_kernel<NT, BF16, GIDX>, map_x, map_sc, map_zr, p) !=
+        cudaSuccess)
+        return W4_ERR_CUDA;
     return launch_status();
 }
 
@@ -220,7 +234,17 @@ w4_status launch_prefill(const CUtensorMap& map, const w4p::PrefillParams& p, in
     auto k = w4p::prefill_kernel<BF16, GIDX>;
     if (!ensure_smem(k, w4p::SmemLayout::bytes, flags, dev)) return W4_ERR_CUDA;
     const dim3 grid((unsigned)((p.N + w4p::BN - 1) / w4p::BN), (unsigned)((p.M + w4p::BM - 1) / w4p::BM));
-    k<<<grid, w4p::kThreads, w4p::SmemLayout::bytes, stream>>>(map, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(w4p::kThreads);
+    cfg.dynamicSmemBytes = (size_t)w4p::SmemLayout::bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k, map, p) != cudaSuccess) return W4_ERR_CUDA;
     return launch_status();
 }
 

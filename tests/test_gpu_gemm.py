@@ -229,3 +229,53 @@ def test_llama8b_prefill_layers(layer, M):
 def test_gptq_act_order_config(M, g):
     skip_without_gpu()
     sampled_case(5, 0, M, g=g, rows=24, cols=128)
+
+
+@pytest.mark.parametrize("M", [3, 192])
+def test_chained_layers_in_a_graph(M):
+    """Each GEMM reads the previous GEMM's output; launched back to back from a CUDA
+    graph, so a kernel that overlaps its predecessor (programmatic dependent launch)
+    must still see the finished activations and leave the shared workspace intact."""
+    skip_without_gpu()
+    import torch
+    K = N = 1024
+    g = 128
+    depth = 6
+    rng = np.random.default_rng(M + 11)
+    X0 = (rng.standard_normal((M, K)).astype(np.float32)).astype(np.float16).view(np.uint16)
+    layers = []
+    for _ in range(depth):
+        W = (rng.standard_normal((N, K)).astype(np.float32) * 0.03).astype(np.float16).view(np.uint16)
+        q, sc, zr = oracle.quantize_weights(W, None, g)
+        layers.append((q, sc, zr, dev(oracle.pack_device(q).view(np.int32)),
+                       dev_bits(sc, torch.float16), dev_bits(zr, torch.float16)))
+    # oracle chain: each output rounded to fp16, as the GPU path stores it
+    x = X0
+    for q, sc, zr, *_ in layers:
+        x = oracle.f32_to_f16(oracle.reference_y(x, None, q, sc, zr, g))
+    ref = x.view(np.float16).astype(np.float64)
+    bufs = [dev_bits(X0, torch.float16)] + [torch.empty(M, N, dtype=torch.float16, device="cuda")
+                                            for _ in range(depth)]
+    ws = torch.zeros(w4.w4a16_workspace_bytes(M, N, K, g) + (1 << 20), dtype=torch.uint8,
+                     device="cuda")
+
+    def chain():
+        for i, (_, _, _, qw, scd, zrd) in enumerate(layers):
+            w4.w4a16_gemm(bufs[i], qw, scd, zrd, g, Y=bufs[i + 1], workspace=ws)
+
+    chain()                       # eager once (kernel attributes, first-call set-up)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            chain()
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        for b in bufs[1:]:
+            b.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        w4.w4_check_device_error()
+        check_y(to_f64(bufs[-1]), ref, "fp16", tol_rel=5e-3)
