@@ -21,6 +21,13 @@ W4_DEV uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned address of a dynamic shared-memory array, by pointer
+// arithmetic on the array itself so that the compiler still knows the result points to
+// shared memory (loads through it stay shared-memory loads, not generic ones).
+W4_DEV unsigned char* align_smem_1024(unsigned char* raw) {
+    return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 W4_DEV uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -60,20 +67,37 @@ W4_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that may suspend the thread for up to `ns` nanoseconds while the phase is
+// incomplete; the thread resumes when the phase completes.  A waiting warp then takes no
+// issue slots from the warps doing work.
+W4_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Bounded: after the configured
-// limit the device error word records a timeout and false is returned.
+// limit the device error word records a timeout and false is returned.  Each try suspends
+// the warp (up to 20 us) instead of spinning, so waiting warps leave the issue slots to
+// the working ones; the clock and the limit (a global load) are only read once a wait has
+// lasted a while.
 W4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < 8; ++i)
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     const uint64_t t0 = globaltimer_ns();
     const uint64_t limit = *(volatile unsigned long long*)&g_w4_wait_limit_ns;
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0u) {
-            if (globaltimer_ns() - t0 > limit) {
-                atomicOr(&g_w4_error_word, W4_DEVERR_TIMEOUT);
-                return false;
-            }
-            __nanosleep(32);
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (globaltimer_ns() - t0 > limit) {
+            atomicOr(&g_w4_error_word, W4_DEVERR_TIMEOUT);
+            return false;
         }
     }
 }

@@ -10,39 +10,66 @@
 //
 // Work decomposition (B200-specific):
 //   atom      = 16 output rows x 64 input channels (512 B of codes); the atoms of one
-//               128-row band are stored column block by column block, so up to 4
-//               consecutive column blocks of a band (up to 16 KB) are one contiguous copy;
-//   stream-K  = all (band, column block) atoms of the layer are split into equal
-//               contiguous ranges, one per CTA, so every SM streams the same number of
-//               bytes whatever N and K are;
-//   stage     = up to 4 column blocks of one band, 5 copies: the codes (one contiguous
-//               bulk copy), the activations (one 3-D TMA box of 4 column blocks x 8*NT
-//               token rows, 128B swizzle, rows >= M zero-filled), the s_inv slice, and the
-//               group rows of scales and of zero points met by the stage (2-D TMA boxes);
-//   CTA       = 1 producer warp + 8 consumer warps; consumer warp w owns rows
-//               16w..16w+15 of the band; per 16-deep step one 32-bit word per lane is
-//               unpacked into the A operand of mma.m16n8k16 (weights as the 16-row side,
-//               up to 64 tokens as 8-column tiles), multiplied as exact integers (q - z)
-//               with fp32 accumulation; each group's partial sum is scaled in fp32;
-//   fix-up    = a band split between CTAs is completed by the last CTA to finish it,
-//               which adds the fp32 partials of all contributors in CTA order
-//               (deterministic) and stores Y; its counter is reset to zero.
+//               128-row band are stored column block by column block, so consecutive
+//               column blocks of a band are one contiguous copy;
+//   unit      = 2 column blocks (128 input channels) of one band; all units of the layer
+//               are split into equal contiguous ranges, one per CTA (stream-K), so every
+//               SM streams the same number of bytes whatever N and K are;
+//   stage     = up to 2 units of one band: the codes (one bulk copy), the activations (one
+//               3-D TMA box of 4 column blocks x 8*NT token rows, 128B swizzle, rows >= M
+//               zero-filled), the s_inv slice and the group rows of scales and zero points;
+//   CTA       = 1 producer warp (its lanes issue the copies of a stage in parallel), XW
+//               activation warps and 16 MMA warps in two groups that take alternate
+//               stages; one CTA per SM, its ring filling the SM's shared memory, so every
+//               SM holds exactly one CTA of a GEMM even when the next GEMM's CTAs start
+//               early under programmatic dependent launch;
+//   activation= per stage, the activation warps write X' = X * s_inv (when given) to a
+//   warps       buffer of their own, the activation sums S and the fold constants of every
+//               staged (group, row);
+//   zero point= the MMA multiplies the biased codes o + m*q (o + m*q is what the AND/OR
+//               unpack yields; no subtraction per weight) and the per-group fold removes
+//               the bias and the zero point with the activation sums S = sum_k X'[m,k] of
+//               the group: sum_k (q-z) X' = (c - (o + m*z) S) / m, in fp32;
+//   fix-up    = a band split between CTAs is completed by the CTA holding its last unit;
+//               the others process their share first and publish fp32 partials as
+//               {value, flag} words, so the finishing CTA only reads them (deterministic
+//               order, no atomics).
 #pragma once
 #include "w4_common.cuh"
 
 namespace w4d {
 
-constexpr int kWarps = 8;                 // consumer warps = row tiles per band
-constexpr int kBandRows = 16 * kWarps;    // 128
-constexpr int kAtomsPerStage = 4;         // column blocks per stage (256 input channels)
-constexpr int kThreads = 32 * (kWarps + 1);
+constexpr int kBandRows = 128;
+constexpr int kTilesPerBand = 8;
+constexpr int kMmaWarps = 8;
+
+// Group handling of the MMA warps.
+enum : int {
+    kModeHalf = 0,   // group size a multiple of 128, K a multiple of 128: one fold per half stage
+    kModeAtom = 1,   // group size a multiple of 64: folds at 64-channel boundaries
+    kModeG32 = 2,    // group size 32: folds every 32 channels
+    kModeGidx = 3,   // act-order g_idx: the scale is folded into each fp16 weight
+};
 
 template <int NT>
 struct Cfg {
-    static constexpr int stages = NT == 1 ? 4 : 3;
-    static constexpr int mpad = 8 * NT;               // token rows per activation box slot
-    static constexpr int xbox = mpad * 128;           // bytes per activation box slot
+    static constexpr int tpw = NT <= 2 ? 2 : 1;          // row tiles per MMA warp
+    static constexpr int aps = NT <= 2 ? 8 : 4;          // atoms (64-channel blocks) per stage
+    static constexpr int xw = NT == 1 ? 1 : NT <= 4 ? 2 : 4;   // activation warps
+    static constexpr int mma_warps = NT <= 4 ? 16 : 8;   // two stage groups (one when 8)
+    static constexpr int groups = mma_warps / 8;         // stage-parity groups
+    static constexpr int warps = 1 + xw + mma_warps;
+    static constexpr int threads = 32 * warps;
+    static constexpr int mpad = 8 * NT;                  // token rows per activation box slot
+    // activation sums of one stage: per token, over 32, 64 and 128 consecutive channels
+    static constexpr int sx32 = 0, sx64 = 2 * aps, sx128 = 3 * aps;
+    static constexpr int sx_floats = 4 * aps * mpad;
+    // partial-sum sets per row tile at a flush: stage groups x K halves
+    static constexpr int nset = groups * (tpw == 2 ? 2 : 1);
+    // MMA-warp exchange buffer: [nset-1][8 tiles][NT][4][32 lanes] fp32
+    static constexpr int xchg_bytes = (nset - 1) * 8 * NT * 4 * 32 * 4;
 };
+constexpr int kMaxStages = 8;
 
 struct DecodeParams {
     const uint32_t* qw;       // device layout
@@ -51,16 +78,17 @@ struct DecodeParams {
     const int32_t* g_idx;     // [K] or null
     const float* s_inv;       // [K] or null
     void* Y;                  // [M,N]
-    float* partials;          // [P][2][128][8*NT] fp32 (workspace)
-    unsigned* counters;       // [bands] (workspace, zero between calls)
+    unsigned long long* slots;   // split-K partials: [P][8 tiles][NT][4][32] {fp32 bits, flag}
     int M, N, K, group_size, G, out_dtype;
-    int KA;                   // K / 64
+    int KA;                   // K / 64 atoms per band
+    int KU;                   // units (2 atoms) per band
     int tiles;                // N / 16
-    int units;                // bands * KA atoms
-    int base, rem;            // atoms per CTA: base (+1 for the first rem CTAs)
+    int units;                // bands * KU
+    int base, rem;            // units per CTA: base (+1 for the first rem CTAs)
     int ngs;                  // group rows staged per stage (scale / zero-point box height)
+    int stages;               // ring depth (<= kMaxStages)
     // byte offsets inside one stage
-    int off_x, off_si, off_sc, off_zr, off_gi, stage_bytes;
+    int off_x, off_xs, off_sx, off_si, off_sc, off_zr, off_gi, stage_bytes;
 };
 
 W4_DEV int unit_begin(const DecodeParams& p, int c) { return c * p.base + min(c, p.rem); }
@@ -68,7 +96,37 @@ W4_DEV int cta_of_unit(const DecodeParams& p, int u) {
     const int split = p.rem * (p.base + 1);
     return u < split ? u / (p.base + 1) : p.rem + (u - split) / p.base;
 }
-W4_DEV int band_tiles(const DecodeParams& p, int band) { return min(kWarps, p.tiles - band * kWarps); }
+W4_DEV int band_tiles(const DecodeParams& p, int band) {
+    return min(kTilesPerBand, p.tiles - band * kTilesPerBand);
+}
+
+// The parts of a CTA's unit range [u0,u1), one per band it touches, in processing order:
+// when the range ends inside a band, that (contributor) part comes first, so its partial
+// sums are published early; every other part either is a whole band or holds the band's
+// last unit and completes it.
+struct PartIter {
+    int b0, b1;
+    bool contrib_first;
+    W4_DEV PartIter(const DecodeParams& p, int u0, int u1) {
+        b0 = u0 / p.KU;
+        b1 = (u1 - 1) / p.KU;
+        contrib_first = u1 < (b1 + 1) * p.KU;
+    }
+    W4_DEV int count() const { return b1 - b0 + 1; }
+    W4_DEV int band(int pi) const {
+        if (contrib_first) return pi == 0 ? b1 : b0 + pi - 1;
+        return b0 + pi;
+    }
+};
+
+// Atom range [a0, a0+na) of stage st of the part [ps,pe) of `band`, UPS units per stage.
+template <int UPS>
+W4_DEV void stage_atoms(const DecodeParams& p, int band, int ps, int pe, int st, int& a0, int& na) {
+    const int u = ps + UPS * st;
+    const int nu = min(UPS, pe - u);
+    a0 = 2 * (u - band * p.KU);
+    na = min(2 * nu, p.KA - a0);
+}
 
 W4_DEV void store_out(const DecodeParams& p, int m, int n, float v) {
     const size_t idx = (size_t)m * p.N + n;
@@ -77,198 +135,588 @@ W4_DEV void store_out(const DecodeParams& p, int m, int n, float v) {
     else reinterpret_cast<__half*>(p.Y)[idx] = __float2half_rn(v);
 }
 
-W4_DEV uint32_t lds32(const unsigned char* p) { return *reinterpret_cast<const uint32_t*>(p); }
-W4_DEV uint32_t lds32_at(uint32_t saddr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(saddr));
-    return v;
+// Shared-memory loads through pointers derived from the dynamic shared array (the
+// compiler keeps them after the mbarrier waits, whose asm clobbers memory, and is free to
+// schedule them otherwise).
+W4_DEV uint32_t ld_u32(const unsigned char* p) { return *reinterpret_cast<const uint32_t*>(p); }
+W4_DEV uint32_t ld_u16(const unsigned char* p) { return *reinterpret_cast<const unsigned short*>(p); }
+W4_DEV uint4 ld_u128(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
+W4_DEV float2 ld_f2(const unsigned char* p) { return *reinterpret_cast<const float2*>(p); }
+
+// Split-K partial words: {fp32 bits (low), flag 1 (high)}, one 64-bit access each.
+W4_DEV void slot_put(unsigned long long* a, float v) {
+    const unsigned long long w = (1ull << 32) | (unsigned long long)__float_as_uint(v);
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(a), "l"(w) : "memory");
+}
+W4_DEV unsigned long long slot_get(const unsigned long long* a) {
+    unsigned long long w;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(a) : "memory");
+    return w;
+}
+W4_DEV void slot_clear(unsigned long long* a) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(a), "l"(0ull) : "memory");
 }
 
-// byte offset of the 4-byte pair (token row, k-pair kp < 32) inside a 128B-swizzled box
-W4_DEV int xsw(int tok, int kp) { return tok * 128 + (((kp >> 2) ^ (tok & 7)) << 4) + ((kp & 3) << 2); }
+// Wait (bounded) until a published partial word carries its flag; returns its value.
+W4_DEV bool slot_wait(const unsigned long long* a, float& v) {
+    unsigned long long w = slot_get(a);
+    if ((w >> 32) == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        const uint64_t limit = *(volatile unsigned long long*)&g_w4_wait_limit_ns;
+        for (uint32_t it = 1;; ++it) {
+            w = slot_get(a);
+            if ((w >> 32) != 0) break;
+            if ((it & 15u) == 0u) {
+                if (globaltimer_ns() - t0 > limit) {
+                    atomicOr(&g_w4_error_word, W4_DEVERR_TIMEOUT);
+                    return false;
+                }
+                __nanosleep(64);
+            }
+        }
+    }
+    v = __uint_as_float((uint32_t)w);
+    return true;
+}
 
-// Complete or hand off the accumulators of one band.
+// ---------------------------------------------------------------- MMA-warp building blocks
+// Biased unpack of one device-layout word (see the layout in w4a16.h): four A-operand
+// registers of a 16x16 MMA slice, a[0] = row r0 cols c,c+1; a[1] = row r1 cols c,c+1;
+// a[2] = row r0 cols c+8,c+9; a[3] = row r1 cols c+8,c+9, each element o + m*q exactly:
+//   fp16: rows r0 (nibbles 0,2,4,6): 1024 + q;  rows r1 (nibbles 1,3,5,7): 1024 + 16 q;
+//   bf16: every element 128 + q.
+template <bool BF16>
+W4_DEV void unpack_biased(uint32_t w, uint32_t (&a)[4]) {
+    if constexpr (!BF16) {
+        const uint32_t w8 = w >> 8;
+        a[0] = and_or(w, 0x000F000Fu, 0x64006400u);
+        a[1] = and_or(w, 0x00F000F0u, 0x64006400u);
+        a[2] = and_or(w8, 0x000F000Fu, 0x64006400u);
+        a[3] = and_or(w8, 0x00F000F0u, 0x64006400u);
+    } else {
+        a[0] = and_or(w, 0x000F000Fu, 0x43004300u);
+        a[1] = and_or(w >> 4, 0x000F000Fu, 0x43004300u);
+        a[2] = and_or(w >> 8, 0x000F000Fu, 0x43004300u);
+        a[3] = and_or(w >> 12, 0x000F000Fu, 0x43004300u);
+    }
+}
+
+// Fold constants of one row for one group: sum_k (q - z) X' = (c + bz * S) * mul ... times
+// the scale, i.e. acc += sc' * (c + bz * S) with sc' = scale / m and bz = -(o + m z).
+struct RowFold {
+    float scp, bz;
+};
+
+template <bool BF16, bool HI>
+W4_DEV RowFold row_fold(uint32_t sc_bits, uint32_t z_bits) {
+    const float sc = __half2float(__ushort_as_half((unsigned short)sc_bits));
+    const float z = __half2float(__ushort_as_half((unsigned short)z_bits));
+    RowFold f;
+    if constexpr (BF16) {
+        f.scp = sc;
+        f.bz = -(128.0f + z);
+    } else if constexpr (HI) {
+        f.scp = sc * 0.0625f;
+        f.bz = -fmaf(16.0f, z, 1024.0f);
+    } else {
+        f.scp = sc;
+        f.bz = -(1024.0f + z);
+    }
+    return f;
+}
+
+// Per-lane constants of an MMA warp.
+struct Lane {
+    int lane, g8, q;
+    int xlo[4], xhi[4];      // activation fragment byte offsets of the 16-deep steps
+};
+
+// xrows: token rows stored per column block of X'; with fewer than 8 rows, lanes of token
+// rows >= M read row M-1 instead (their products land in accumulator columns that are
+// never stored).
+W4_DEV Lane make_lane(int lane, int xrows) {
+    Lane L;
+    L.lane = lane;
+    L.g8 = lane >> 2;
+    L.q = lane & 3;
+    const int row = min(L.g8, xrows - 1);
+    // row `row` of a 128B-swizzled line, k pairs 8j+q (b0) and 8j+4+q (b1) of step j
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        L.xlo[j] = row * 128 + ((((2 * j) ^ row) & 7) << 4) + 4 * L.q;
+        L.xhi[j] = row * 128 + ((((2 * j + 1) ^ row) & 7) << 4) + 4 * L.q;
+    }
+    return L;
+}
+
+
+// What an MMA warp needs about the stage being consumed.
+struct StageView {
+    const unsigned char* codes;   // the stage's packed tiles: [atom][tile][512 B]
+    const unsigned char* x;       // activations X': [column block][token row][128 B swizzled]
+    const unsigned char* sx;      // activation sums: [segment][token] fp32
+    const unsigned char* sc;      // scale rows: [group row][128] fp16
+    const unsigned char* zr;      // zero-point rows, or null (symmetric)
+    int xstride;                  // bytes per column block of X' (token rows x 128)
+    int tb, a0, gfirst;
+    int r0;                       // (64 * a0) mod group size: offset of the stage in its group
+};
+
+// D(16x8, fp32) = A(16x16) * B(16x8), no accumulator input.
+template <bool BF16>
+W4_DEV void mma_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    if constexpr (BF16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+            "{%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+            "{%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+    }
+}
+
+// One 16-deep step of TPW row tiles against NT token tiles; FIRST starts the partial sums.
+template <int NT, int TPW, bool BF16, bool FIRST>
+W4_DEV void mma_step(const uint32_t (&wj)[TPW], const unsigned char* xa, int xl, int xh,
+                     float (&c)[TPW][NT][4]) {
+    uint32_t b0[NT], b1[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        b0[nt] = ld_u32(xa + nt * 1024 + xl);
+        b1[nt] = ld_u32(xa + nt * 1024 + xh);
+    }
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+        uint32_t af[4];
+        unpack_biased<BF16>(wj[tt], af);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            if constexpr (FIRST) mma_16816_z<BF16>(c[tt][nt], af, b0[nt], b1[nt]);
+            else mma_16816<BF16>(c[tt][nt], af, b0[nt], b1[nt]);
+        }
+    }
+}
+
 template <int NT>
-W4_DEV void flush_band(const DecodeParams& p, int band, int u0, int u1, int cta, int w,
-                       int lane, int ctid, bool aborted, float (&acc)[NT][4],
-                       volatile int* s_flag) {
-    const int Mp = 8 * NT;
-    const bool tile_ok = w < band_tiles(p, band);
-    const int rl0 = 16 * w + (lane >> 2);            // row within the band
-    const int n0 = band * kBandRows + rl0;
-    const int q2 = 2 * (lane & 3);
-    const bool whole = (u0 <= band * p.KA) && (u1 >= (band + 1) * p.KA);
-    if (whole) {
-        if (tile_ok && !aborted) {
+W4_DEV void load_sums(const unsigned char* sx, int seg, const Lane& L, float2 (&S)[NT]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) S[nt] = ld_f2(sx + (seg * 8 * NT + 8 * nt + 2 * L.q) * 4);
+}
+
+// Fold the partial sums c of one group (staged group row `grow`) into acc:
+// acc += sc' * (c + bz * S) per element, with the row's {sc', bz} from its staged fp16
+// scale and zero point and S, per token tile, the activation sums of tokens 8nt+2q and
+// 8nt+2q+1 over the folded channels.
+template <int NT, int TPW, bool BF16>
+W4_DEV void fold(const StageView& v, const Lane& L, int t0, int grow, const float2 (&S)[NT],
+                 const float (&c)[TPW][NT][4], float (&acc)[TPW][NT][4]) {
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+        const int o0 = (grow * kBandRows + 16 * (t0 + tt) + L.g8) * 2, o1 = o0 + 16;
+        const uint32_t sc0 = ld_u16(v.sc + o0), sc1 = ld_u16(v.sc + o1);
+        const uint32_t z0 = v.zr ? ld_u16(v.zr + o0) : 0x4800u;   // symmetric: z = 8
+        const uint32_t z1 = v.zr ? ld_u16(v.zr + o1) : 0x4800u;
+        const RowFold f0 = row_fold<BF16, false>(sc0, z0);
+        const RowFold f1 = row_fold<BF16, true>(sc1, z1);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            acc[tt][nt][0] = fmaf(f0.scp, fmaf(f0.bz, S[nt].x, c[tt][nt][0]), acc[tt][nt][0]);
+            acc[tt][nt][1] = fmaf(f0.scp, fmaf(f0.bz, S[nt].y, c[tt][nt][1]), acc[tt][nt][1]);
+            acc[tt][nt][2] = fmaf(f1.scp, fmaf(f1.bz, S[nt].x, c[tt][nt][2]), acc[tt][nt][2]);
+            acc[tt][nt][3] = fmaf(f1.scp, fmaf(f1.bz, S[nt].y, c[tt][nt][3]), acc[tt][nt][3]);
+        }
+    }
+}
+
+template <int TPW>
+W4_DEV uint32_t word_j(const uint4& w, int j) { return j == 0 ? w.x : j == 1 ? w.y : j == 2 ? w.z : w.w; }
+
+template <int NT, int TPW>
+W4_DEV void zero_acc(float (&c)[TPW][NT][4]) {
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[tt][nt][e] = 0.0f;
+}
+
+// Consume atoms [ab, ae) of the stage for row tiles t0..t0+TPW-1 (contiguous groups).
+template <int NT, int TPW, bool BF16, int MODE>
+W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, int g,
+                    float (&acc)[TPW][NT][4]) {
+    const unsigned char* wl = v.codes + t0 * 512 + L.lane * 16;
+    if constexpr (MODE == kModeHalf) {
+        // atoms come in pairs, each pair inside one group; with one token tile the odd
+        // 16-deep steps accumulate into a second register set so consecutive MMAs of a
+        // tile do not wait on each other
+        constexpr int CH = NT == 1 ? 2 : 1;
+        // staged group row of the first pair and the pair's offset inside its group
+        int kin = v.r0 + 64 * ab;
+        int grow = kin / g;
+        kin -= grow * g;
+#pragma unroll 1
+        for (int a = ab; a < ae; a += 2) {
+            uint4 w[2][TPW];
+#pragma unroll
+            for (int aa = 0; aa < 2; ++aa)
+#pragma unroll
+                for (int tt = 0; tt < TPW; ++tt) w[aa][tt] = ld_u128(wl + ((a + aa) * v.tb + tt) * 512);
+            float c[TPW][NT][4], c2[TPW][NT][4];
+#pragma unroll
+            for (int aa = 0; aa < 2; ++aa) {
+                const unsigned char* xa = v.x + (a + aa) * v.xstride;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t wj[TPW];
+#pragma unroll
+                    for (int tt = 0; tt < TPW; ++tt) wj[tt] = word_j<TPW>(w[aa][tt], j);
+                    const int st = 4 * aa + j;
+                    if (CH == 2 && (st & 1)) {
+                        if (st == 1) mma_step<NT, TPW, BF16, true>(wj, xa, L.xlo[j], L.xhi[j], c2);
+                        else mma_step<NT, TPW, BF16, false>(wj, xa, L.xlo[j], L.xhi[j], c2);
+                    } else {
+                        if (st == 0) mma_step<NT, TPW, BF16, true>(wj, xa, L.xlo[j], L.xhi[j], c);
+                        else mma_step<NT, TPW, BF16, false>(wj, xa, L.xlo[j], L.xhi[j], c);
+                    }
+                }
+            }
+            if constexpr (CH == 2) {
+#pragma unroll
+                for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) c[tt][nt][e] += c2[tt][nt][e];
+            }
+            float2 S[NT];
+            load_sums<NT>(v.sx, Cfg<NT>::sx128 + (a >> 1), L, S);
+            fold<NT, TPW, BF16>(v, L, t0, grow, S, c, acc);
+            kin += 128;
+            if (kin >= g) {
+                kin -= g;
+                ++grow;
+            }
+        }
+    } else {
+        // atom by atom; the activation sums accumulate until the fold
+        float c[TPW][NT][4];
+        zero_acc<NT, TPW>(c);
+        float2 S[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) S[nt] = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+        for (int a = ab; a < ae; ++a) {
+            uint4 w[TPW];
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt) w[tt] = ld_u128(wl + (a * v.tb + tt) * 512);
+            const unsigned char* xa = v.x + a * v.xstride;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t wj[TPW];
+#pragma unroll
+                for (int tt = 0; tt < TPW; ++tt) wj[tt] = word_j<TPW>(w[tt], j);
+                mma_step<NT, TPW, BF16, false>(wj, xa, L.xlo[j], L.xhi[j], c);
+                if constexpr (MODE == kModeG32) {
+                    if (j & 1) {
+                        float2 S32[NT];
+                        load_sums<NT>(v.sx, Cfg<NT>::sx32 + 2 * a + (j >> 1), L, S32);
+                        fold<NT, TPW, BF16>(v, L, t0, 2 * a + (j >> 1), S32, c, acc);
+                        zero_acc<NT, TPW>(c);
+                    }
+                }
+            }
+            if constexpr (MODE == kModeAtom) {
+                float2 S64[NT];
+                load_sums<NT>(v.sx, Cfg<NT>::sx64 + a, L, S64);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    S[nt].x += S64[nt].x;
+                    S[nt].y += S64[nt].y;
+                }
+                if ((64 * (v.a0 + a + 1)) % g == 0 || a == ae - 1) {
+                    fold<NT, TPW, BF16>(v, L, t0, (64 * (v.a0 + a)) / g - v.gfirst, S, c, acc);
+                    zero_acc<NT, TPW>(c);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) S[nt] = make_float2(0.0f, 0.0f);
+                }
+            }
+        }
+    }
+}
+
+// Act-order: every input channel k has its own group g_idx[k]; each weight is dequantised
+// to fp16 (q - z[g_idx[k], n]) * scale[g_idx[k], n] before the MMA (fp16 activations only).
+template <int NT, int TPW>
+W4_DEV void consume_gidx(const StageView& v, const DecodeParams& p, const Lane& L, int band, int t0,
+                         int ab, int ae, const unsigned char* gis, float (&acc)[TPW][NT][4]) {
+    const unsigned char* wl = v.codes + t0 * 512 + L.lane * 16;
+#pragma unroll 1
+    for (int a = ab; a < ae; ++a) {
+        const unsigned char* xa = v.x + a * v.xstride;
+#pragma unroll 1
+        for (int j = 0; j < 4; ++j) {
+            const int kk = 64 * a + 16 * j + 2 * L.q;
+            int gk[4] = {(int)ld_u32(gis + 4 * kk), (int)ld_u32(gis + 4 * (kk + 1)),
+                         (int)ld_u32(gis + 4 * (kk + 8)), (int)ld_u32(gis + 4 * (kk + 9))};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (gk[e] < 0 || gk[e] >= p.G) {
+                    atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
+                    gk[e] = 0;
+                }
+            uint32_t b0[NT], b1[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                b0[nt] = ld_u32(xa + nt * 1024 + L.xlo[j]);
+                b1[nt] = ld_u32(xa + nt * 1024 + L.xhi[j]);
+            }
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt) {
+                if (t0 + tt >= v.tb) continue;   // rows beyond N: no metadata to gather
+                const uint32_t wv = word_j<TPW>(ld_u128(wl + (a * v.tb + tt) * 512), j);
+                const int nr0 = band * kBandRows + 16 * (t0 + tt) + L.g8, nr1 = nr0 + 8;
+                uint32_t af[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    // register r holds nibbles r and r+4: rows r0/r1 (r odd), columns
+                    // c,c+1 (r < 2) or c+8,c+9 (r >= 2)
+                    const int row = (r & 1) ? nr1 : nr0;
+                    const int kl = (r & 2) ? 2 : 0;
+                    const float qlo = (float)((wv >> (4 * r)) & 0xF);
+                    const float qhi = (float)((wv >> (4 * (r + 4))) & 0xF);
+                    const __half z_lo = p.zeros ? __ldg(p.zeros + (size_t)gk[kl] * p.N + row) : __float2half_rn(8.0f);
+                    const __half z_hi = p.zeros ? __ldg(p.zeros + (size_t)gk[kl + 1] * p.N + row) : __float2half_rn(8.0f);
+                    const __half2 ss = __halves2half2(__ldg(p.scales + (size_t)gk[kl] * p.N + row),
+                                                      __ldg(p.scales + (size_t)gk[kl + 1] * p.N + row));
+                    af[r] = h2_as_u32(__hmul2(__hsub2(__floats2half2_rn(qlo, qhi), __halves2half2(z_lo, z_hi)), ss));
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_16816<false>(acc[tt][nt], af, b0[nt], b1[nt]);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- activation warps
+// Per stage: X' = X * s_inv rounded to the activation type (into the X' buffer, when s_inv
+// is given; otherwise the MMA warps read the tensor box itself), the sums of X' over 32,
+// 64 and 128 consecutive channels per token, and the fold constants {sc', bz} of every
+// staged (group row, band row).  The stage's channels form 8-channel chunks (column block
+// c/8, 16-byte chunk c%8); each warp pass covers 32 consecutive chunks of one token.
+template <int NT, bool BF16, bool GIDX>
+W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw, int lane) {
+    using C = Cfg<NT>;
+    constexpr int CPT = 8 * C::aps;    // chunks per token
+    const int xrows = NT == 1 ? p.M : C::mpad;
+    const unsigned char* xb = st + p.off_x;
+    unsigned char* xs = st + p.off_xs;
+    float* sx = reinterpret_cast<float*>(st + p.off_sx);
+    const float* si = reinterpret_cast<const float*>(st + p.off_si);
+    for (int base = 32 * xw; base < p.M * CPT; base += 32 * C::xw) {
+        const int m = base / CPT;
+        const int c = base % CPT + lane;
+        const int blk = c >> 3, ch = c & 7;
+        float s = 0.0f;
+        if (c < 8 * na) {
+            // the tensor box holds M rows per column block, 128B-swizzled by line index
+            const int line = blk * p.M + m;
+            const uint4 v = ld_u128(xb + line * 128 + ((ch ^ (line & 7)) << 4));
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            if (p.s_inv) {
+                const float4 s0 = *reinterpret_cast<const float4*>(si + 8 * c);
+                const float4 s1 = *reinterpret_cast<const float4*>(si + 8 * c + 4);
+                const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = unpack2<BF16>(w[i]);
+                    w[i] = pack2<BF16>(__fmul_rn(f.x, sv[2 * i]), __fmul_rn(f.y, sv[2 * i + 1]));
+                }
+            }
+            // X' rows: xrows per column block, swizzled by token row
+            *reinterpret_cast<uint4*>(xs + (blk * xrows + m) * 128 + ((ch ^ (m & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+            if constexpr (!GIDX) {
+                float2 f[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) f[i] = unpack2<BF16>(w[i]);
+                s = ((f[0].x + f[0].y) + (f[1].x + f[1].y)) + ((f[2].x + f[2].y) + (f[3].x + f[3].y));
+            }
+        }
+        if constexpr (!GIDX) {
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            if ((lane & 3) == 0) sx[(C::sx32 + (c >> 2)) * C::mpad + m] = s;
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            if ((lane & 7) == 0) sx[(C::sx64 + (c >> 3)) * C::mpad + m] = s;
+            s += __shfl_xor_sync(0xffffffffu, s, 8);
+            if ((lane & 15) == 0) sx[(C::sx128 + (c >> 4)) * C::mpad + m] = s;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- end of a part
+// Combine, then store, publish or complete the band's sums.  Slot entry of (tile t, token
+// tile nt, element e, lane) is ((t * NT + nt) * 4 + e) * 32 + lane.
+template <int NT, int TPW>
+W4_DEV void flush_part(const DecodeParams& p, unsigned char* xchg, int band, int ps, int pe, int cta,
+                       int set, int t0, const Lane& L, bool aborted, float (&acc)[TPW][NT][4]) {
+    using C = Cfg<NT>;
+    if constexpr (C::nset > 1) {
+        // the partial sums of a row tile (stage groups x K halves) meet in shared memory;
+        // set 0 adds the others in a fixed order
+        float* xc = reinterpret_cast<float*>(xchg);
+        constexpr int kSet = 8 * NT * 4 * 32;
+        if (set > 0) {
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        xc[(set - 1) * kSet + (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane] = acc[tt][nt][e];
+        }
+        named_bar_sync(1, 32 * C::mma_warps);
+        if (set == 0) {
+#pragma unroll
+            for (int k = 1; k < C::nset; ++k)
+#pragma unroll
+                for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            acc[tt][nt][e] += xc[(k - 1) * kSet + (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane];
+        }
+        named_bar_sync(2, 32 * C::mma_warps);
+        if (set > 0) return;
+    }
+    if (aborted) return;
+    const int tb = band_tiles(p, band);
+    const int bu0 = band * p.KU, bu1 = bu0 + p.KU;
+    constexpr int kSlot = kTilesPerBand * NT * 4 * 32;
+    if (pe < bu1) {
+        // contributor: publish this CTA's share of the band
+        unsigned long long* base = p.slots + (size_t)cta * kSlot;
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt) {
+            if (t0 + tt >= tb) continue;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int m = 8 * nt + q2 + (e & 1);
-                    const int n = n0 + ((e >> 1) << 3);
-                    if (m < p.M) store_out(p, m, n, acc[nt][e]);
-                }
+                for (int e = 0; e < 4; ++e)
+                    if (8 * nt + 2 * L.q + (e & 1) < p.M)
+                        slot_put(base + (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane, acc[tt][nt][e]);
         }
         return;
     }
-    // partial band: write this CTA's fp32 partial sums to its slot
-    const int first_band = unit_begin(p, cta) / p.KA;
-    const int which = (band == first_band) ? 0 : 1;
-    float* slot = p.partials + ((size_t)cta * 2 + which) * (size_t)(kBandRows * Mp);
-    if (tile_ok && !aborted) {
+    if (ps > bu0) {
+        // the band's last unit: add the contributors' shares (CTA order) before this one's
+        float tot[TPW][NT][4];
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) tot[tt][nt][e] = 0.0f;
+        const int c_first = cta_of_unit(p, bu0);
+        bool ok = true;
+        for (int c = c_first; c < cta && ok; ++c) {
+            unsigned long long* base = p.slots + (size_t)c * kSlot;
+            unsigned long long w[TPW][NT][4];
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const bool valid = t0 + tt < tb && 8 * nt + 2 * L.q + (e & 1) < p.M;
+                        w[tt][nt][e] = valid ? slot_get(base + (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane)
+                                             : (1ull << 32);
+                    }
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const bool valid = t0 + tt < tb && 8 * nt + 2 * L.q + (e & 1) < p.M;
+                        if (!valid || !ok) continue;
+                        unsigned long long* a = base + (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane;
+                        float v = __uint_as_float((uint32_t)w[tt][nt][e]);
+                        if ((w[tt][nt][e] >> 32) == 0 && !slot_wait(a, v)) {
+                            ok = false;
+                            continue;
+                        }
+                        tot[tt][nt][e] += v;
+                        slot_clear(a);
+                    }
+        }
+        if (!ok) return;
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[tt][nt][e] = tot[tt][nt][e] + acc[tt][nt][e];
+    }
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+        if (t0 + tt >= tb) continue;
+        const int n0 = band * kBandRows + 16 * (t0 + tt) + L.g8;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int m = 8 * nt + q2 + (e & 1);
-                const int rl = rl0 + ((e >> 1) << 3);
-                if (m < p.M) slot[rl * Mp + m] = acc[nt][e];
+                const int m = 8 * nt + 2 * L.q + (e & 1);
+                if (m < p.M) store_out(p, m, n0 + ((e >> 1) << 3), acc[tt][nt][e]);
             }
     }
-    __threadfence();
-    named_bar_sync(2, 32 * kWarps);
-    const int c_first = cta_of_unit(p, band * p.KA);
-    const int c_last = cta_of_unit(p, (band + 1) * p.KA - 1);
-    if (ctid == 0) {
-        int last = 0;
-        if (!aborted) {
-            const unsigned prev = atomicAdd(p.counters + band, 1u);
-            last = (prev == (unsigned)(c_last - c_first));
-        }
-        *s_flag = last;
-    }
-    named_bar_sync(2, 32 * kWarps);
-    if (*s_flag) {
-        __threadfence();
-        if (tile_ok) {
-            // Only the first contributor can hold this band in its second slot (its range
-            // began in an earlier band); every later one began inside this band.
-            const int first_slot = (unit_begin(p, c_first) < band * p.KA) ? 1 : 0;
-            const size_t slot_elems = (size_t)kBandRows * Mp;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int m = 8 * nt + q2 + (e & 1);
-                    const int rl = rl0 + ((e >> 1) << 3);
-                    if (m >= p.M) continue;
-                    const float* base = p.partials + rl * Mp + m;
-                    float v = 0.0f;
-                    // contributors in CTA order, loads issued a batch at a time
-                    for (int cb = c_first; cb <= c_last; cb += 8) {
-                        float part[8];
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) {
-                            const int c = cb + t;
-                            const int wc = (c == c_first) ? first_slot : 0;
-                            part[t] = (c <= c_last) ? __ldcg(base + ((size_t)c * 2 + wc) * slot_elems) : 0.0f;
-                        }
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) v += part[t];
-                    }
-                    store_out(p, m, band * kBandRows + rl, v);
-                }
-        }
-        if (ctid == 0) p.counters[band] = 0u;
-    }
-    named_bar_sync(2, 32 * kWarps);
 }
 
-W4_DEV void fold(float s0, float s1, float (&c)[4], float (&acc)[4]) {
-    acc[0] = fmaf(s0, c[0], acc[0]);
-    acc[1] = fmaf(s0, c[1], acc[1]);
-    acc[2] = fmaf(s1, c[2], acc[2]);
-    acc[3] = fmaf(s1, c[3], acc[3]);
-    c[0] = c[1] = c[2] = c[3] = 0.0f;
+// ---------------------------------------------------------------- the kernel
+template <int UPS>
+W4_DEV int total_stages(const DecodeParams& p, const PartIter& it, int u0, int u1) {
+    int n = 0;
+    for (int pi = 0; pi < it.count(); ++pi) {
+        const int band = it.band(pi);
+        const int ps = max(u0, band * p.KU), pe = min(u1, (band + 1) * p.KU);
+        n += (pe - ps + UPS - 1) / UPS;
+    }
+    return n;
 }
 
-// One stage of the decode consumer (contiguous groups): the warp's 16-row tile times
-// up to kAtomsPerStage column blocks staged at `st`; partial sums of each group are
-// folded into acc with the group's fp32 scale.  nb = first column of the next group.
-template <int NT, bool BF16>
-W4_DEV void consume_stage(const unsigned char* st, int off_x, int off_sc, int off_zr, bool has_zeros,
-                          int na, int a0, int tb, int nb, int g, bool g32, int w, int lane,
-                          int rl0, int rl1, uint32_t xrow, const int (&xlo)[4], const int (&xhi)[4],
-                          const ZeroConsts& zc_sym, float (&acc)[NT][4]) {
-    using C = Cfg<NT>;
-    const __half* scp = reinterpret_cast<const __half*>(st + off_sc);
-    const unsigned short* zrp = reinterpret_cast<const unsigned short*>(st + off_zr);
-    float s0 = __half2float(scp[rl0]), s1 = __half2float(scp[rl1]);
-    ZeroConsts zc = has_zeros ? zero_consts_h<BF16>(zrp[rl0], zrp[rl1]) : zc_sym;
-    // two accumulator chains (even / odd 16-deep steps) for MMA overlap
-    float c0[NT][4], c1[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) c0[nt][e] = c1[nt][e] = 0.0f;
-    // per-stage fragment base addresses: every load below is one of these registers plus
-    // a compile-time offset
-    uint32_t xl[4], xh[4];
-    const uint32_t xs = smem_u32(st + off_x) + xrow;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        xl[j] = xs + xlo[j];
-        xh[j] = xs + xhi[j];
-    }
-    const unsigned char* wbase = st + w * 512 + lane * 16;
-    const int wstride = tb * 512;
-    int ka = 64 * a0;
-#pragma unroll
-    for (int a = 0; a < kAtomsPerStage; ++a) {
-        if (a < na) {
-            const uint4 wq = *reinterpret_cast<const uint4*>(wbase + a * wstride);
-            const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if ((j == 0 || (j == 2 && g32)) && ka + 16 * j >= nb) {
-                    // group boundary: fold the finished group's partials, load the next
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        fold(s0, s1, c0[nt], acc[nt]);
-                        fold(s0, s1, c1[nt], acc[nt]);
-                    }
-                    nb += g;
-                    scp += 128;
-                    zrp += 128;
-                    s0 = __half2float(scp[rl0]);
-                    s1 = __half2float(scp[rl1]);
-                    if (has_zeros) zc = zero_consts_h<BF16>(zrp[rl0], zrp[rl1]);
-                }
-                uint32_t af[4];
-                unpack_word<BF16>(wv[j], zc, af);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    // token rows >= M were zero-filled by the tensor copy
-                    const uint32_t b0 = lds32_at(xl[j] + a * C::xbox + nt * 1024);
-                    const uint32_t b1 = lds32_at(xh[j] + a * C::xbox + nt * 1024);
-                    // with few token tiles a second chain breaks the MMA dependency; with
-                    // more tiles they already interleave
-                    mma_16816<BF16>((NT <= 2 && (j & 1)) ? c1[nt] : c0[nt], af, b0, b1);
-                }
-            }
-            ka += 64;
+// Ring position: slot and phase parity of consecutive stages.
+struct Ring {
+    int s = 0, ph = 0;
+    W4_DEV void next(int S) {
+        if (++s == S) {
+            s = 0;
+            ph ^= 1;
         }
     }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        fold(s0, s1, c0[nt], acc[nt]);
-        fold(s0, s1, c1[nt], acc[nt]);
-    }
-}
+};
 
-template <int NT, bool BF16, bool GIDX>
-__global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
+template <int NT, bool BF16, int MODE>
+__global__ void __launch_bounds__(Cfg<NT>::threads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_sc,
                   const __grid_constant__ CUtensorMap tmap_zr, const DecodeParams p) {
     using C = Cfg<NT>;
-    constexpr int S = C::stages;
+    constexpr bool GIDX = MODE == kModeGidx;
+    constexpr int UPS = C::aps / 2;   // units per stage
+    const int S = p.stages;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * p.stage_bytes);
-    uint64_t* empty = full + S;
-    volatile int* s_abort = reinterpret_cast<volatile int*>(empty + S);
-    volatile int* s_last = s_abort + 1;
+    unsigned char* smem = align_smem_1024(smem_raw);
+    unsigned char* xchg = smem + S * p.stage_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(xchg + C::xchg_bytes);
+    uint64_t* xready = full + kMaxStages;
+    uint64_t* empty = xready + kMaxStages;
+    volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
@@ -278,11 +726,17 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kWarps);
+            mbar_init(&xready[s], 32 * C::xw);
+            mbar_init(&empty[s], kMmaWarps);
         }
         *s_abort = 0;
-        *s_last = 0;
         fence_mbar_init();
+    }
+    // activation sums and X' rows of tokens >= M are never written: start from zero
+    {
+        const int words = (p.off_si - p.off_xs) / 4;   // X' and sums of one stage
+        for (int i = threadIdx.x; i < S * words; i += C::threads)
+            reinterpret_cast<uint32_t*>(smem + (i / words) * p.stage_bytes + p.off_xs)[i % words] = 0u;
     }
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmap_x);
@@ -296,197 +750,159 @@ __global__ void __launch_bounds__(kThreads, NT >= 8 ? 1 : 2)
     // Everything this kernel reads before pdl_wait() (codes, scales, zero points, g_idx)
     // is never written by the kernels of this library.
     pdl_launch_dependents();
+    if (u0 >= u1) return;
+    const PartIter it(p, u0, u1);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        // lane 0 arms the stage's barrier and issues one copy per operand: the codes
+        // (a contiguous run of the band), the scale and zero-point rows (2-D boxes) or the
+        // g_idx slice, the activations (3-D box: 4 column blocks x 8*NT token rows, rows
+        // >= M and blocks beyond K zero-filled) and the s_inv slice.  The read-only weight
+        // operands of the first stages go out before pdl_wait(), the activations (possibly
+        // produced by the preceding kernel) after it.
         const uint64_t policy = policy_evict_first();
+        const int total = total_stages<UPS>(p, it, u0, u1);
+        const int pro = min(S, total);
+        Ring r;
         int i = 0;
-        for (int u = u0; u < u1; ++i) {
-            const int band = u / p.KA, a0 = u - band * p.KA;
-            const int na = min(kAtomsPerStage, min(p.KA - a0, u1 - u));
-            const int s = i % S, ph = (i / S) & 1;
-            if (i >= S) {
-                const bool ok = !*s_abort && mbar_wait(&empty[s], ph ^ 1);
-                if (!ok) { *s_abort = 1; break; }
-            }
-            unsigned char* st = smem + s * p.stage_bytes;
+        bool abort = false;
+        for (int pi = 0; pi < it.count() && !abort; ++pi) {
+            const int band = it.band(pi);
+            const int ps = max(u0, band * p.KU), pe = min(u1, (band + 1) * p.KU);
             const int tb = band_tiles(p, band);
-            // one copy per operand: codes (contiguous run of the band), activations (one
-            // 3-D box: 4 column blocks x 8*NT token rows, rows >= M and blocks beyond K
-            // zero-filled), s_inv slice, scale rows and zero-point rows (2-D boxes).  The
-            // read-only weight operands of the first stages go out before pdl_wait(), the
-            // activations (possibly produced by the preceding kernel) after it.
-            const int g_first = (64 * a0) / g;
-            uint32_t bytes = na * tb * 512 + kAtomsPerStage * C::xbox;
-            if (p.s_inv) bytes += na * 256;
-            if (GIDX) bytes += na * 256;
-            else bytes += p.ngs * 256 * (p.zeros ? 2 : 1);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&full[s], bytes);
-                bulk_g2s_hint(st, p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)a0 * tb),
-                              na * tb * 512, &full[s], policy);
-                if (GIDX) {
-                    bulk_g2s(st + p.off_gi, p.g_idx + 64 * a0, na * 256, &full[s]);
-                } else {
-                    tma_load_2d(st + p.off_sc, &tmap_sc, band * kBandRows, g_first, &full[s]);
-                    if (p.zeros) tma_load_2d(st + p.off_zr, &tmap_zr, band * kBandRows, g_first, &full[s]);
+            for (int stg = 0; UPS * stg < pe - ps; ++stg, ++i, r.next(S)) {
+                int a0, na;
+                stage_atoms<UPS>(p, band, ps, pe, stg, a0, na);
+                if (i >= S) {
+                    int ok = 1;
+                    if (lane == 0) ok = (!*s_abort && mbar_wait(&empty[r.s], r.ph ^ 1)) ? 1 : 0;
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) {
+                        if (lane == 0) *s_abort = 1;
+                        abort = true;
+                        break;
+                    }
                 }
-                if (i == 0) pdl_wait();
-                tma_load_3d(st + p.off_x, &tmap_x, 0, 0, a0, &full[s]);
-                if (p.s_inv) bulk_g2s(st + p.off_si, p.s_inv + 64 * a0, na * 256, &full[s]);
+                unsigned char* st = smem + r.s * p.stage_bytes;
+                const int g_first = GIDX ? 0 : (64 * a0) / g;
+                if (lane == 0) {
+                    uint32_t bytes = na * tb * 512 + C::aps * p.M * 128;
+                    if (p.s_inv) bytes += na * 256;
+                    if (GIDX) bytes += na * 256;
+                    else bytes += p.ngs * 256 * (p.zeros ? 2 : 1);
+                    mbar_arrive_expect_tx(&full[r.s], bytes);
+                    bulk_g2s_hint(st, p.qw + 128 * ((size_t)kTilesPerBand * p.KA * band + (size_t)a0 * tb),
+                                  na * tb * 512, &full[r.s], policy);
+                    if (GIDX) {
+                        bulk_g2s(st + p.off_gi, p.g_idx + 64 * a0, na * 256, &full[r.s]);
+                    } else {
+                        tma_load_2d(st + p.off_sc, &tmap_sc, band * kBandRows, g_first, &full[r.s]);
+                        if (p.zeros) tma_load_2d(st + p.off_zr, &tmap_zr, band * kBandRows, g_first, &full[r.s]);
+                    }
+                    if (i >= S) {
+                        tma_load_3d(st + p.off_x, &tmap_x, 0, 0, a0, &full[r.s]);
+                        if (p.s_inv) bulk_g2s(st + p.off_si, p.s_inv + 64 * a0, na * 256, &full[r.s]);
+                    }
+                }
+                if (i == pro - 1) {
+                    // the activations of the first stages, once the preceding grid is done
+                    pdl_wait();
+                    int k = 0;
+                    for (int pj = 0; pj < it.count() && k < pro; ++pj) {
+                        const int bj = it.band(pj);
+                        const int qs = max(u0, bj * p.KU), qe = min(u1, (bj + 1) * p.KU);
+                        for (int sj = 0; UPS * sj < qe - qs && k < pro; ++sj, ++k) {
+                            int aj, nj;
+                            stage_atoms<UPS>(p, bj, qs, qe, sj, aj, nj);
+                            unsigned char* sk = smem + k * p.stage_bytes;
+                            if (lane == 0) {
+                                tma_load_3d(sk + p.off_x, &tmap_x, 0, 0, aj, &full[k]);
+                                if (p.s_inv) bulk_g2s(sk + p.off_si, p.s_inv + 64 * aj, nj * 256, &full[k]);
+                            }
+                        }
+                    }
+                }
             }
-            __syncwarp();
-            u += na;
         }
-        // On abort, wait (bounded) for the copies already issued before leaving.
-        if (*s_abort && lane == 0)
-            for (int k = (i > S ? i - S : 0); k < i; ++k) (void)mbar_wait(&full[k % S], (k / S) & 1);
-    } else {
-        // ------------------------------------------------------------ consumers
-        pdl_wait();   // before any store to Y or the workspace
-        const int w = warp - 1;
-        const int ctid = threadIdx.x - 32;
-        const int q = lane & 3, g8 = lane >> 2;
-        const int rl0 = 16 * w + g8, rl1 = rl0 + 8;
-        // activation fragment offsets inside a 128B-swizzled box: row g8 (+8 per token
-        // tile), k pairs 8j+q (b0) and 8j+4+q (b1) of the 16-deep step j
-        const uint32_t xrow = g8 * 128;
-        int xlo[4], xhi[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            xlo[j] = (((2 * j) ^ g8) << 4) + 4 * q;
-            xhi[j] = (((2 * j + 1) ^ g8) << 4) + 4 * q;
+        // On abort, wait (bounded) for the copies already issued before leaving (an abort
+        // can only happen at i >= S, after every prologue copy went out).
+        if (abort && lane == 0) {
+            Ring q;
+            for (int k = 0; k < i; ++k, q.next(S))
+                if (k >= i - S) (void)mbar_wait(&full[q.s], q.ph);
         }
-        const bool g32 = (g == 32);
-        // symmetric format: the implicit zero point 8 never changes
-        const ZeroConsts zc_sym = zero_consts_h<BF16>(0x4800u, 0x4800u);
-        float acc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-        // stage coordinates advance incrementally (one division per CTA)
-        int band = (u0 < u1) ? u0 / p.KA : 0;
-        int a0 = u0 - band * p.KA;
-        int cur_band = (u0 < u1) ? band : -1;
-        int gcur = (64 * a0) / g;          // group of the next column to process
-        int next_b = (gcur + 1) * g;       // first column of the following group
+        __syncwarp();
+    } else if (warp <= C::xw) {
+        // ------------------------------------------------------------ activation warps
+        const int xw = warp - 1;
         bool aborted = false;
-
-        int i = 0;
-        for (int u = u0; u < u1; ++i) {
-            const int na = min(kAtomsPerStage, min(p.KA - a0, u1 - u));
-            const int s = i % S, ph = (i / S) & 1;
-            if (band != cur_band) {
-                flush_band<NT>(p, cur_band, u0, u1, cta, w, lane, ctid, aborted, acc, s_last);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-                cur_band = band;
-            }
-            if (!aborted) {
-                aborted = *s_abort || !mbar_wait(&full[s], ph);
-                if (aborted) *s_abort = 1;
-            }
-            unsigned char* st = smem + s * p.stage_bytes;
-            unsigned char* xb = st + p.off_x;
-            if (p.s_inv) {
-                // X' = X * s_inv rounded to the activation type, in place, once per stage
+        Ring r;
+        for (int pi = 0; pi < it.count(); ++pi) {
+            const int band = it.band(pi);
+            const int ps = max(u0, band * p.KU), pe = min(u1, (band + 1) * p.KU);
+            for (int stg = 0; UPS * stg < pe - ps; ++stg, r.next(S)) {
+                int a0, na;
+                stage_atoms<UPS>(p, band, ps, pe, stg, a0, na);
                 if (!aborted) {
-                    const float* si = reinterpret_cast<const float*>(st + p.off_si);
-                    const int per_box = p.M * 32;
-#pragma unroll
-                    for (int a = 0; a < kAtomsPerStage; ++a) {
-                        if (a < na) {
-                            for (int r = ctid; r < per_box; r += 32 * kWarps) {
-                                const int tok = r >> 5, kp = r & 31;
-                                uint32_t* px = reinterpret_cast<uint32_t*>(xb + a * C::xbox + xsw(tok, kp));
-                                const float2 v = unpack2<BF16>(*px);
-                                const float2 sv = *reinterpret_cast<const float2*>(si + 64 * a + 2 * kp);
-                                *px = pack2<BF16>(__fmul_rn(v.x, sv.x), __fmul_rn(v.y, sv.y));
-                            }
-                        }
-                    }
+                    aborted = *s_abort || !mbar_wait(&full[r.s], r.ph);
+                    if (aborted) *s_abort = 1;
                 }
-                named_bar_sync(1, 32 * kWarps);
-            }
-            const int tb = band_tiles(p, band);
-            if (!GIDX) {
-                // the group containing this stage's first column (the staged scale and
-                // zero-point rows start there)
-                while (64 * a0 >= next_b) {
-                    next_b += g;
-                    ++gcur;
-                }
-            }
-            if (!aborted && w < tb) {
-                if constexpr (!GIDX) {
-                    consume_stage<NT, BF16>(st, p.off_x, p.off_sc, p.off_zr, p.zeros != nullptr, na, a0,
-                                            tb, next_b, g, g32, w, lane, rl0, rl1, xrow, xlo, xhi,
-                                            zc_sym, acc);
-                } else {
-                    // act-order: every channel has its own group; fold the scale into an
-                    // fp16 weight (q - z) * scale before the MMA
-                    const int32_t* gis = reinterpret_cast<const int32_t*>(st + p.off_gi);
-                    const int n_r0 = band * kBandRows + rl0, n_r1 = n_r0 + 8;
-#pragma unroll
-                    for (int a = 0; a < kAtomsPerStage; ++a) {
-                        if (a < na) {
-                            const uint4 wq = *reinterpret_cast<const uint4*>(
-                                st + (a * tb + w) * 512 + lane * 16);
-                            const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-                            const unsigned char* xa = xb + a * C::xbox;
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const int kk = 64 * a + 16 * j + 2 * q;
-                                int gk[4] = {gis[kk], gis[kk + 1], gis[kk + 8], gis[kk + 9]};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    if (gk[e] < 0 || gk[e] >= p.G) {
-                                        atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
-                                        gk[e] = 0;
-                                    }
-                                uint32_t af[4];
-#pragma unroll
-                                for (int r = 0; r < 4; ++r) {
-                                    const int row = (r & 1) ? n_r1 : n_r0;
-                                    const int kl = (r & 2) ? 2 : 0;
-                                    const float qlo = (float)((wv[j] >> (4 * r)) & 0xF);
-                                    const float qhi = (float)((wv[j] >> (4 * (r + 4))) & 0xF);
-                                    const __half z_lo = p.zeros ? __ldg(p.zeros + (size_t)gk[kl] * p.N + row)
-                                                                : __float2half_rn(8.0f);
-                                    const __half z_hi = p.zeros ? __ldg(p.zeros + (size_t)gk[kl + 1] * p.N + row)
-                                                                : __float2half_rn(8.0f);
-                                    const __half2 ss = __halves2half2(__ldg(p.scales + (size_t)gk[kl] * p.N + row),
-                                                                      __ldg(p.scales + (size_t)gk[kl + 1] * p.N + row));
-                                    af[r] = h2_as_u32(__hmul2(
-                                        __hsub2(__floats2half2_rn(qlo, qhi), __halves2half2(z_lo, z_hi)), ss));
-                                }
-#pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    const uint32_t b0 = lds32(xa + xrow + nt * 1024 + xlo[j]);
-                                    const uint32_t b1 = lds32(xa + xrow + nt * 1024 + xhi[j]);
-                                    mma_16816<false>(acc[nt], af, b0, b1);
-                                }
-                            }
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-            u += na;
-            a0 += na;
-            if (a0 == p.KA) {
-                a0 = 0;
-                ++band;
-                gcur = 0;
-                next_b = g;
+                if (!aborted) prep_stage<NT, BF16, GIDX>(smem + r.s * p.stage_bytes, p, na, xw, lane);
+                mbar_arrive(&xready[r.s]);
             }
         }
-        if (cur_band >= 0)
-            flush_band<NT>(p, cur_band, u0, u1, cta, w, lane, ctid, aborted, acc, s_last);
+    } else {
+        // ------------------------------------------------------------ MMA warps
+        pdl_wait();   // before any store to Y or the workspace
+        constexpr int TPW = C::tpw;
+        const int cw = warp - 1 - C::xw;
+        const int grp = cw >> 3, w8 = cw & 7;          // stage group, warp within it
+        const int h = TPW == 2 ? (w8 >> 2) : 0;        // K half (two tiles per warp)
+        const int t0 = TPW == 2 ? 2 * (w8 & 3) : w8;
+        const int set = grp * (TPW == 2 ? 2 : 1) + h;  // partial-sum set at a flush
+        const Lane L = make_lane(lane, NT == 1 ? p.M : C::mpad);
+        float acc[TPW][NT][4];
+        zero_acc<NT, TPW>(acc);
+        bool aborted = false;
+        Ring r;
+        int i = 0;
+        for (int pi = 0; pi < it.count(); ++pi) {
+            const int band = it.band(pi);
+            const int ps = max(u0, band * p.KU), pe = min(u1, (band + 1) * p.KU);
+            const int tb = band_tiles(p, band);
+            for (int stg = 0; UPS * stg < pe - ps; ++stg, ++i, r.next(S)) {
+                if ((i % C::groups) != grp) continue;   // the other group's stage
+                int a0, na;
+                stage_atoms<UPS>(p, band, ps, pe, stg, a0, na);
+                if (!aborted) {
+                    aborted = *s_abort || !mbar_wait(&xready[r.s], r.ph);
+                    if (aborted) *s_abort = 1;
+                }
+                const int ab = TPW == 2 ? h * (C::aps / 2) : 0;
+                const int ae = TPW == 2 ? min(na, ab + C::aps / 2) : na;
+                if (!aborted && t0 < tb && ab < ae) {
+                    unsigned char* st = smem + r.s * p.stage_bytes;
+                    StageView v;
+                    v.codes = st;
+                    v.x = st + p.off_xs;
+                    v.xstride = (NT == 1 ? p.M : C::mpad) * 128;
+                    v.sx = st + p.off_sx;
+                    v.sc = st + p.off_sc;
+                    v.zr = p.zeros ? st + p.off_zr : nullptr;
+                    v.tb = tb;
+                    v.a0 = a0;
+                    v.gfirst = GIDX ? 0 : (64 * a0) / g;
+                    v.r0 = GIDX ? 0 : 64 * a0 - v.gfirst * g;
+                    if constexpr (GIDX) consume_gidx<NT, TPW>(v, p, L, band, t0, ab, ae, st + p.off_gi, acc);
+                    else consume<NT, TPW, BF16, MODE>(v, L, t0, ab, ae, g, acc);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[r.s]);
+            }
+            flush_part<NT, TPW>(p, xchg, band, ps, pe, cta, set, t0, L, aborted, acc);
+            zero_acc<NT, TPW>(acc);
+        }
     }
 }
 

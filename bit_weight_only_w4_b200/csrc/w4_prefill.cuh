@@ -162,8 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const PrefillParams p) {
     extern __shared__ unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled operand tiles
-    unsigned char* smem = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* smem = align_smem_1024(smem_raw);
     using L = SmemLayout;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::bars);
     uint64_t* deq = full + kStages;

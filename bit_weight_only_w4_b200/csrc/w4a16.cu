@@ -16,7 +16,6 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kDecodeMaxM = 64;
-constexpr int kDecodeMaxCtasPerSm = 2;
 constexpr int kQuantMaxGroups = 1536;
 constexpr int64_t kMaxBands = 8192;                       // N <= 1,048,576 (fix-up counters)
 
@@ -68,15 +67,23 @@ bool ensure_smem(Kernel k, int bytes, std::once_flag (&flags)[kMaxDevices], int 
 // ---------------------------------------------------------------- decode launch plan
 int decode_tiles_for(int64_t M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 
-// Split-K fix-up counters live in a fixed region at the start of the workspace, one per
-// 128-row band, so that every call -- whatever its N -- finds its counters where earlier
-// calls left them at zero; the partial-sum slots follow the region.
+// Workspace layout (caller-owned, zero-filled once):
+//   [0, 32 KB)                 a fixed region kept at zero (the original counter region;
+//                              kept so the layout of the rest is stable);
+//   [32 KB, 32 KB + R)         the decode kernel's split-K partial words, one slot of
+//                              8 tiles x NT token tiles x 4 x 32 {value, flag} words per CTA
+//                              (one CTA per SM).  R is sized for the largest NT (8), so
+//                              every decode call -- whatever its M -- finds its slots in the
+//                              same place; every call leaves each flag it read at zero;
+//   [32 KB + R, ...)           prefill scratch (the activations scaled by s_inv), which
+//                              therefore never touches a flag.
 constexpr size_t kCounterBytes = (size_t)kMaxBands * 4;   // 32 KB
 
+size_t decode_slot_bytes(int NT, int sms) { return (size_t)sms * w4d::kTilesPerBand * NT * 4 * 32 * 8; }
+size_t slot_region_bytes(int sms) { return decode_slot_bytes(8, sms); }
+
 size_t decode_workspace_bytes(int64_t M, int sms) {
-    const int Mp = 8 * decode_tiles_for(M);
-    const size_t partials = (size_t)sms * kDecodeMaxCtasPerSm * 2 * w4d::kBandRows * Mp * 4;
-    return kCounterBytes + partials;
+    return kCounterBytes + decode_slot_bytes(decode_tiles_for(M), sms);
 }
 
 int smem_per_sm(int dev) {
@@ -154,43 +161,51 @@ bool make_meta_map(CUtensorMap* map, const void* base, int64_t G, int64_t N, int
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NT, bool BF16, bool GIDX>
+template <int NT, bool BF16, int MODE>
 w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
                         cudaStream_t stream) {
     using C = w4d::Cfg<NT>;
+    constexpr bool GIDX = MODE == w4d::kModeGidx;
+    auto kernel = w4d::decode_kernel<NT, BF16, MODE>;
     static std::once_flag flags[kMaxDevices];
     constexpr int kMaxSmem = 227 * 1024;
     bool attr_ok = true;
     std::call_once(flags[dev], [&] {
-        attr_ok = cudaFuncSetAttribute(w4d::decode_kernel<NT, BF16, GIDX>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kMaxSmem) == cudaSuccess;
+        attr_ok = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) ==
+                  cudaSuccess;
     });
     if (!attr_ok) return W4_ERR_CUDA;
-    // stage layout: codes | activation boxes | s_inv | scale rows | zero rows | g_idx
+    // stage layout: codes | activation box (M rows) | X' | activation sums | s_inv |
+    // scale rows | zero-point rows | g_idx
     const int g = p.group_size;
-    p.ngs = GIDX ? 0 : (g == 32 ? 8 : std::min(p.G, (256 + 2 * g - 65) / g));
-    p.off_x = w4d::kAtomsPerStage * w4d::kWarps * 512;
-    p.off_si = p.off_x + w4d::kAtomsPerStage * C::xbox;
-    p.off_sc = p.off_si + (p.s_inv ? 1024 : 0);
+    const int span = 64 * C::aps;   // input channels per stage
+    const int xrows = NT == 1 ? p.M : C::mpad;
+    auto up = [](int v, int a) { return (v + a - 1) / a * a; };
+    p.ngs = GIDX ? 0 : (g == 32 ? span / 32 : std::min(p.G, (span + 2 * g - 65) / g));
+    p.off_x = C::aps * w4d::kTilesPerBand * 512;
+    p.off_xs = p.off_x + up(C::aps * p.M * 128, 1024);
+    p.off_sx = p.off_xs + up(C::aps * xrows * 128, 128);
+    p.off_si = p.off_sx + (GIDX ? 0 : C::sx_floats * 4);
+    p.off_sc = p.off_si + (p.s_inv ? C::aps * 256 : 0);
     p.off_zr = p.off_sc + p.ngs * 256;
     p.off_gi = p.off_zr + (p.zeros ? p.ngs * 256 : 0);
-    p.stage_bytes = (p.off_gi + (GIDX ? 1024 : 0) + 1023) / 1024 * 1024;
-    const int smem = C::stages * p.stage_bytes + 2 * C::stages * 8 + 16 + 1024;
-    if (smem > kMaxSmem) return W4_ERR_UNSUPPORTED;
-    int per_sm = NT >= 8 ? 1 : std::min(kDecodeMaxCtasPerSm, smem_per_sm(dev) / (smem + 1024));
-    if (per_sm < 1) per_sm = 1;
-    const int bands = (p.tiles + w4d::kWarps - 1) / w4d::kWarps;
-    p.units = bands * p.KA;
-    int P = sm_count(dev) * per_sm;
+    p.stage_bytes = (p.off_gi + (GIDX ? C::aps * 256 : 0) + 1023) / 1024 * 1024;
+    // as many stages as fit: the CTA fills the SM's shared memory, one CTA per SM
+    const int fixed = C::xchg_bytes + 3 * w4d::kMaxStages * 8 + 16 + 1024;
+    p.stages = std::min(w4d::kMaxStages, (kMaxSmem - fixed) / p.stage_bytes);
+    if (p.stages < 2) return W4_ERR_UNSUPPORTED;
+    const int smem = p.stages * p.stage_bytes + fixed;
+    const int bands = (p.tiles + w4d::kTilesPerBand - 1) / w4d::kTilesPerBand;
+    p.KU = (p.KA + 1) / 2;
+    p.units = bands * p.KU;
+    int P = sm_count(dev);
     if (P <= 0) return W4_ERR_CUDA;
     if (P > p.units) P = p.units;
     p.base = p.units / P;
     p.rem = p.units % P;
-    p.counters = reinterpret_cast<unsigned*>(ws);
-    p.partials = reinterpret_cast<float*>(ws + kCounterBytes);
+    p.slots = reinterpret_cast<unsigned long long*>(ws + kCounterBytes);
     CUtensorMap map_x, map_sc, map_zr;
-    if (!make_act_blocks_map(&map_x, X, BF16, p.M, p.K, C::mpad, w4d::kAtomsPerStage)) return W4_ERR_CUDA;
+    if (!make_act_blocks_map(&map_x, X, BF16, p.M, p.K, p.M, C::aps)) return W4_ERR_CUDA;
     map_sc = map_x;
     map_zr = map_x;
     if (!GIDX) {
@@ -201,7 +216,7 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     // the tail of the preceding kernel on the stream
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)P);
-    cfg.blockDim = dim3(w4d::kThreads);
+    cfg.blockDim = dim3(C::threads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -209,20 +224,41 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, w4d::decode_kernel<NT, BF16, GIDX>, map_x, map_sc, map_zr, p) !=
-        cudaSuccess)
-        return W4_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kernel, map_x, map_sc, map_zr, p) != cudaSuccess) return W4_ERR_CUDA;
     return launch_status();
 }
 
-template <bool BF16, bool GIDX>
-w4_status dispatch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
+// Group handling: one fold per 128-channel half stage when groups are whole multiples of
+// 128 channels and K holds whole 128-channel units; a fold per 32 channels for g = 32;
+// folds at 64-channel boundaries otherwise.
+int decode_mode(int64_t K, int32_t g, bool gidx) {
+    if (gidx) return w4d::kModeGidx;
+    if (g % 128 == 0 && (K / 64) % 2 == 0) return w4d::kModeHalf;
+    if (g == 32) return w4d::kModeG32;
+    return w4d::kModeAtom;
+}
+
+template <int NT, bool BF16>
+w4_status dispatch_mode(int mode, w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
+                        cudaStream_t s) {
+    if constexpr (!BF16) {
+        if (mode == w4d::kModeGidx) return launch_decode<NT, false, w4d::kModeGidx>(p, X, ws, dev, s);
+    } else {
+        if (mode == w4d::kModeGidx) return W4_ERR_UNSUPPORTED;
+    }
+    if (mode == w4d::kModeHalf) return launch_decode<NT, BF16, w4d::kModeHalf>(p, X, ws, dev, s);
+    if (mode == w4d::kModeG32) return launch_decode<NT, BF16, w4d::kModeG32>(p, X, ws, dev, s);
+    return launch_decode<NT, BF16, w4d::kModeAtom>(p, X, ws, dev, s);
+}
+
+template <bool BF16>
+w4_status dispatch_decode(int mode, w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
                           cudaStream_t s) {
     switch (decode_tiles_for(p.M)) {
-        case 1: return launch_decode<1, BF16, GIDX>(p, X, ws, dev, s);
-        case 2: return launch_decode<2, BF16, GIDX>(p, X, ws, dev, s);
-        case 4: return launch_decode<4, BF16, GIDX>(p, X, ws, dev, s);
-        default: return launch_decode<8, BF16, GIDX>(p, X, ws, dev, s);
+        case 1: return dispatch_mode<1, BF16>(mode, p, X, ws, dev, s);
+        case 2: return dispatch_mode<2, BF16>(mode, p, X, ws, dev, s);
+        case 4: return dispatch_mode<4, BF16>(mode, p, X, ws, dev, s);
+        default: return dispatch_mode<8, BF16>(mode, p, X, ws, dev, s);
     }
 }
 
@@ -314,8 +350,8 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size
     const int sms = dev >= 0 ? sm_count(dev) : 0;
     if (sms <= 0) return 0;
     if (M <= kDecodeMaxM) return decode_workspace_bytes(M, sms);
-    // prefill: scaled activations, behind the counter region (which must stay zero)
-    return kCounterBytes + (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
+    // prefill: scaled activations, behind the zero region and the decode slot region
+    return kCounterBytes + slot_region_bytes(sms) + (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
 }
 
 w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
@@ -364,16 +400,16 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
         p.KA = (int)(K / 64);
         p.tiles = (int)(N / 16);
         unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
-        if (bf16) return dispatch_decode<true, false>(p, X, ws, dev, strm);
-        return gidx ? dispatch_decode<false, true>(p, X, ws, dev, strm)
-                    : dispatch_decode<false, false>(p, X, ws, dev, strm);
+        const int mode = decode_mode(K, group_size, gidx);
+        if (bf16) return dispatch_decode<true>(mode, p, X, ws, dev, strm);
+        return dispatch_decode<false>(mode, p, X, ws, dev, strm);
     }
 
     const void* Xeff = X;
     if (s_inv) {
         const size_t pairs = (size_t)M * (size_t)K / 2;
         const unsigned blocks = (unsigned)((pairs + 255) / 256 < 65535 * 8 ? (pairs + 255) / 256 : 65535 * 8);
-        void* xp = reinterpret_cast<unsigned char*>(workspace) + kCounterBytes;
+        void* xp = reinterpret_cast<unsigned char*>(workspace) + kCounterBytes + slot_region_bytes(sm_count(dev));
         if (bf16) w4p::scale_acts_kernel<true><<<blocks, 256, 0, strm>>>(X, s_inv, xp, (int)M, (int)K);
         else w4p::scale_acts_kernel<false><<<blocks, 256, 0, strm>>>(X, s_inv, xp, (int)M, (int)K);
         if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
@@ -471,13 +507,14 @@ struct NoAllocScratch {
 NoAllocScratch g_noalloc[kMaxDevices];
 
 // Set-up on the first call per device (that device current): look up the array's device
-// address and zero its counter region, the part that every call expects to find at zero.
+// address and zero it (every call expects the split-K flags it reads to start at zero and
+// leaves them at zero).
 void* noalloc_scratch(int dev) {
     NoAllocScratch& s = g_noalloc[dev];
     std::call_once(s.once, [&] {
         void* p = nullptr;
         s.err = cudaGetSymbolAddress(&p, g_w4_noalloc_scratch);
-        if (s.err == cudaSuccess) s.err = cudaMemset(p, 0, kCounterBytes);
+        if (s.err == cudaSuccess) s.err = cudaMemset(p, 0, kNoAllocScratchBytes);
         if (s.err == cudaSuccess) s.err = cudaDeviceSynchronize();
         if (s.err == cudaSuccess) s.ptr = p;
     });
@@ -530,7 +567,7 @@ extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64
     p.KA = (int)(K / 64);
     p.tiles = (int)(N / 16);
     cudaStream_t strm = as_stream(stream);
-    if (bf16) return dispatch_decode<true, false>(p, X, ws, dev, strm);
-    return gidx ? dispatch_decode<false, true>(p, X, ws, dev, strm)
-                : dispatch_decode<false, false>(p, X, ws, dev, strm);
+    const int mode = decode_mode(K, group_size, gidx);
+    if (bf16) return dispatch_decode<true>(mode, p, X, ws, dev, strm);
+    return dispatch_decode<false>(mode, p, X, ws, dev, strm);
 }
