@@ -77,6 +77,7 @@ struct DecodeParams {
     const __half* zeros;      // [G,N] or null
     const int32_t* g_idx;     // [K] or null
     const float* s_inv;       // [K] or null
+    const void* X;            // [M,K] activations (read directly when X' is resident)
     void* Y;                  // [M,N]
     unsigned long long* slots;   // split-K partials: [P][8 tiles][NT][4][32] {fp32 bits, flag}
     int M, N, K, group_size, G, out_dtype;
@@ -87,8 +88,13 @@ struct DecodeParams {
     int base, rem;            // units per CTA: base (+1 for the first rem CTAs)
     int ngs;                  // group rows staged per stage (scale / zero-point box height)
     int stages;               // ring depth (<= kMaxStages)
+    int xres;                 // 1: X' and its sums are prepared once per CTA and stay resident
+    int off_res;              // byte offset of the resident X' (after the ring and exchange)
+    int off_res_s;            // byte offset of the resident sums: [K/32 | K/64 | K/128][sstride]
+    int sstride;              // tokens per row of the activation sums
+    int off_xchg;             // byte offset of the MMA-warp exchange buffer
     // byte offsets inside one stage
-    int off_x, off_xs, off_sx, off_si, off_sc, off_zr, off_gi, stage_bytes;
+    int off_x, off_xs, off_sx, off_si, off_sc, off_zr, off_gi, off_desc, stage_bytes;
 };
 
 W4_DEV int unit_begin(const DecodeParams& p, int c) { return c * p.base + min(c, p.rem); }
@@ -228,23 +234,26 @@ W4_DEV RowFold row_fold(uint32_t sc_bits, uint32_t z_bits) {
 // Per-lane constants of an MMA warp.
 struct Lane {
     int lane, g8, q;
+    int st;                  // token offset of this lane's activation-sum pair
     int xlo[4], xhi[4];      // activation fragment byte offsets of the 16-deep steps
 };
 
-// xrows: token rows stored per column block of X'; with fewer than 8 rows, lanes of token
-// rows >= M read row M-1 instead (their products land in accumulator columns that are
-// never stored).
-W4_DEV Lane make_lane(int lane, int xrows) {
+// X' is stored [token row][column block][128 B], each 128-byte line swizzled by its row
+// (16-byte chunk c at (c ^ (row & 7)) * 16), `rs` bytes per row.  xrows: token rows
+// stored; with fewer than 8, lanes of token rows >= M read row M-1 instead (their
+// products land in accumulator columns that are never stored).
+W4_DEV Lane make_lane(int lane, int xrows, int sstride, int rs) {
     Lane L;
     L.lane = lane;
     L.g8 = lane >> 2;
     L.q = lane & 3;
+    L.st = min(2 * L.q, sstride - 2);   // token pairs beyond the stored ones: never stored
     const int row = min(L.g8, xrows - 1);
     // row `row` of a 128B-swizzled line, k pairs 8j+q (b0) and 8j+4+q (b1) of step j
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        L.xlo[j] = row * 128 + ((((2 * j) ^ row) & 7) << 4) + 4 * L.q;
-        L.xhi[j] = row * 128 + ((((2 * j + 1) ^ row) & 7) << 4) + 4 * L.q;
+        L.xlo[j] = row * rs + ((((2 * j) ^ row) & 7) << 4) + 4 * L.q;
+        L.xhi[j] = row * rs + ((((2 * j + 1) ^ row) & 7) << 4) + 4 * L.q;
     }
     return L;
 }
@@ -254,12 +263,14 @@ W4_DEV Lane make_lane(int lane, int xrows) {
 struct StageView {
     const unsigned char* codes;   // the stage's packed tiles: [atom][tile][512 B]
     const unsigned char* x;       // activations X': [column block][token row][128 B swizzled]
-    const unsigned char* sx;      // activation sums: [segment][token] fp32
+    const unsigned char* sx32;    // activation sums over 32 / 64 / 128 channels from the
+    const unsigned char* sx64;    // stage's first channel: [segment][sstride] fp32
+    const unsigned char* sx128;
+    int sstride;
     const unsigned char* sc;      // scale rows: [group row][128] fp16
     const unsigned char* zr;      // zero-point rows, or null (symmetric)
-    int xstride;                  // bytes per column block of X' (token rows x 128)
     int tb, a0, gfirst;
-    int r0;                       // (64 * a0) mod group size: offset of the stage in its group
+    int kin, grow;                // first consumed atom: offset in its group, staged group row
 };
 
 // D(16x8, fp32) = A(16x16) * B(16x8), no accumulator input.
@@ -287,8 +298,8 @@ W4_DEV void mma_step(const uint32_t (&wj)[TPW], const unsigned char* xa, int xl,
     uint32_t b0[NT], b1[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-        b0[nt] = ld_u32(xa + nt * 1024 + xl);
-        b1[nt] = ld_u32(xa + nt * 1024 + xh);
+        b0[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + xl);
+        b1[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + xh);
     }
 #pragma unroll
     for (int tt = 0; tt < TPW; ++tt) {
@@ -303,9 +314,9 @@ W4_DEV void mma_step(const uint32_t (&wj)[TPW], const unsigned char* xa, int xl,
 }
 
 template <int NT>
-W4_DEV void load_sums(const unsigned char* sx, int seg, const Lane& L, float2 (&S)[NT]) {
+W4_DEV void load_sums(const unsigned char* sx, int seg, int sstride, const Lane& L, float2 (&S)[NT]) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) S[nt] = ld_f2(sx + (seg * 8 * NT + 8 * nt + 2 * L.q) * 4);
+    for (int nt = 0; nt < NT; ++nt) S[nt] = ld_f2(sx + (seg * sstride + 8 * nt + L.st) * 4);
 }
 
 // Fold the partial sums c of one group (staged group row `grow`) into acc:
@@ -352,40 +363,63 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
                     float (&acc)[TPW][NT][4]) {
     const unsigned char* wl = v.codes + t0 * 512 + L.lane * 16;
     if constexpr (MODE == kModeHalf) {
-        // atoms come in pairs, each pair inside one group; with one token tile the odd
-        // 16-deep steps accumulate into a second register set so consecutive MMAs of a
-        // tile do not wait on each other
+        // atoms come in pairs, each pair inside one group (at most two pairs per call).
+        // Every address below is a per-call pointer plus a compile-time offset.  With one
+        // token tile the odd 16-deep steps accumulate into a second register set so
+        // consecutive MMAs of a tile do not wait on each other.
         constexpr int CH = NT == 1 ? 2 : 1;
+        constexpr int NTOFF = 8 * Cfg<NT>::aps * 128;   // token tiles of the staged X'
+        const unsigned char* xb = v.x + ab * 128;
+        const unsigned char* xq[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            xq[2 * j] = xb + L.xlo[j];
+            xq[2 * j + 1] = xb + L.xhi[j];
+        }
+        const int wstride = v.tb * 512;
+        const unsigned char* wp[4];
+        wp[0] = v.codes + ab * wstride + t0 * 512 + L.lane * 16;
+#pragma unroll
+        for (int k = 1; k < 4; ++k) wp[k] = wp[k - 1] + wstride;
+        const unsigned char* scp = v.sc + (16 * t0 + L.g8) * 2;
+        const unsigned char* zrp = v.zr + (16 * t0 + L.g8) * 2;
+        const unsigned char* sxp = v.sx128 + ((ab >> 1) * v.sstride + L.st) * 4;
         // staged group row of the first pair and the pair's offset inside its group
-        int kin = v.r0 + 64 * ab;
-        int grow = kin / g;
-        kin -= grow * g;
-#pragma unroll 1
-        for (int a = ab; a < ae; a += 2) {
+        int kin = v.kin;
+        int grow = v.grow;
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+            if (ab + 2 * pr >= ae) break;
             uint4 w[2][TPW];
 #pragma unroll
             for (int aa = 0; aa < 2; ++aa)
 #pragma unroll
-                for (int tt = 0; tt < TPW; ++tt) w[aa][tt] = ld_u128(wl + ((a + aa) * v.tb + tt) * 512);
+                for (int tt = 0; tt < TPW; ++tt) w[aa][tt] = ld_u128(wp[2 * pr + aa] + tt * 512);
             float c[TPW][NT][4], c2[TPW][NT][4];
 #pragma unroll
-            for (int aa = 0; aa < 2; ++aa) {
-                const unsigned char* xa = v.x + (a + aa) * v.xstride;
+            for (int aa = 0; aa < 2; ++aa)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    uint32_t wj[TPW];
+                    const int xo = (2 * pr + aa) * 128;
+                    uint32_t b0[NT], b1[NT];
 #pragma unroll
-                    for (int tt = 0; tt < TPW; ++tt) wj[tt] = word_j<TPW>(w[aa][tt], j);
+                    for (int nt = 0; nt < NT; ++nt) {
+                        b0[nt] = ld_u32(xq[2 * j] + xo + nt * NTOFF);
+                        b1[nt] = ld_u32(xq[2 * j + 1] + xo + nt * NTOFF);
+                    }
                     const int st = 4 * aa + j;
-                    if (CH == 2 && (st & 1)) {
-                        if (st == 1) mma_step<NT, TPW, BF16, true>(wj, xa, L.xlo[j], L.xhi[j], c2);
-                        else mma_step<NT, TPW, BF16, false>(wj, xa, L.xlo[j], L.xhi[j], c2);
-                    } else {
-                        if (st == 0) mma_step<NT, TPW, BF16, true>(wj, xa, L.xlo[j], L.xhi[j], c);
-                        else mma_step<NT, TPW, BF16, false>(wj, xa, L.xlo[j], L.xhi[j], c);
+#pragma unroll
+                    for (int tt = 0; tt < TPW; ++tt) {
+                        uint32_t af[4];
+                        unpack_biased<BF16>(word_j<TPW>(w[aa][tt], j), af);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            float (&d)[4] = (CH == 2 && (st & 1)) ? c2[tt][nt] : c[tt][nt];
+                            if (st < CH) mma_16816_z<BF16>(d, af, b0[nt], b1[nt]);
+                            else mma_16816<BF16>(d, af, b0[nt], b1[nt]);
+                        }
                     }
                 }
-            }
             if constexpr (CH == 2) {
 #pragma unroll
                 for (int tt = 0; tt < TPW; ++tt)
@@ -395,8 +429,24 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
                         for (int e = 0; e < 4; ++e) c[tt][nt][e] += c2[tt][nt][e];
             }
             float2 S[NT];
-            load_sums<NT>(v.sx, Cfg<NT>::sx128 + (a >> 1), L, S);
-            fold<NT, TPW, BF16>(v, L, t0, grow, S, c, acc);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) S[nt] = ld_f2(sxp + (pr * v.sstride + 8 * nt) * 4);
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt) {
+                const int o = grow * 256 + tt * 32;
+                const uint32_t sc0 = ld_u16(scp + o), sc1 = ld_u16(scp + o + 16);
+                const uint32_t z0 = v.zr ? ld_u16(zrp + o) : 0x4800u;   // symmetric: z = 8
+                const uint32_t z1 = v.zr ? ld_u16(zrp + o + 16) : 0x4800u;
+                const RowFold f0 = row_fold<BF16, false>(sc0, z0);
+                const RowFold f1 = row_fold<BF16, true>(sc1, z1);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    acc[tt][nt][0] = fmaf(f0.scp, fmaf(f0.bz, S[nt].x, c[tt][nt][0]), acc[tt][nt][0]);
+                    acc[tt][nt][1] = fmaf(f0.scp, fmaf(f0.bz, S[nt].y, c[tt][nt][1]), acc[tt][nt][1]);
+                    acc[tt][nt][2] = fmaf(f1.scp, fmaf(f1.bz, S[nt].x, c[tt][nt][2]), acc[tt][nt][2]);
+                    acc[tt][nt][3] = fmaf(f1.scp, fmaf(f1.bz, S[nt].y, c[tt][nt][3]), acc[tt][nt][3]);
+                }
+            }
             kin += 128;
             if (kin >= g) {
                 kin -= g;
@@ -415,7 +465,7 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
             uint4 w[TPW];
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt) w[tt] = ld_u128(wl + (a * v.tb + tt) * 512);
-            const unsigned char* xa = v.x + a * v.xstride;
+            const unsigned char* xa = v.x + a * 128;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 uint32_t wj[TPW];
@@ -425,7 +475,7 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
                 if constexpr (MODE == kModeG32) {
                     if (j & 1) {
                         float2 S32[NT];
-                        load_sums<NT>(v.sx, Cfg<NT>::sx32 + 2 * a + (j >> 1), L, S32);
+                        load_sums<NT>(v.sx32, 2 * a + (j >> 1), v.sstride, L, S32);
                         fold<NT, TPW, BF16>(v, L, t0, 2 * a + (j >> 1), S32, c, acc);
                         zero_acc<NT, TPW>(c);
                     }
@@ -433,7 +483,7 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
             }
             if constexpr (MODE == kModeAtom) {
                 float2 S64[NT];
-                load_sums<NT>(v.sx, Cfg<NT>::sx64 + a, L, S64);
+                load_sums<NT>(v.sx64, a, v.sstride, L, S64);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     S[nt].x += S64[nt].x;
@@ -458,7 +508,7 @@ W4_DEV void consume_gidx(const StageView& v, const DecodeParams& p, const Lane& 
     const unsigned char* wl = v.codes + t0 * 512 + L.lane * 16;
 #pragma unroll 1
     for (int a = ab; a < ae; ++a) {
-        const unsigned char* xa = v.x + a * v.xstride;
+        const unsigned char* xa = v.x + a * 128;
 #pragma unroll 1
         for (int j = 0; j < 4; ++j) {
             const int kk = 64 * a + 16 * j + 2 * L.q;
@@ -473,8 +523,8 @@ W4_DEV void consume_gidx(const StageView& v, const DecodeParams& p, const Lane& 
             uint32_t b0[NT], b1[NT];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                b0[nt] = ld_u32(xa + nt * 1024 + L.xlo[j]);
-                b1[nt] = ld_u32(xa + nt * 1024 + L.xhi[j]);
+                b0[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + L.xlo[j]);
+                b1[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + L.xhi[j]);
             }
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt) {
@@ -513,7 +563,6 @@ template <int NT, bool BF16, bool GIDX>
 W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw, int lane) {
     using C = Cfg<NT>;
     constexpr int CPT = 8 * C::aps;    // chunks per token
-    const int xrows = NT == 1 ? p.M : C::mpad;
     const unsigned char* xb = st + p.off_x;
     unsigned char* xs = st + p.off_xs;
     float* sx = reinterpret_cast<float*>(st + p.off_sx);
@@ -538,8 +587,8 @@ W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw,
                     w[i] = pack2<BF16>(__fmul_rn(f.x, sv[2 * i]), __fmul_rn(f.y, sv[2 * i + 1]));
                 }
             }
-            // X' rows: xrows per column block, swizzled by token row
-            *reinterpret_cast<uint4*>(xs + (blk * xrows + m) * 128 + ((ch ^ (m & 7)) << 4)) =
+            // X': [token row][column block][128 B], lines swizzled by token row
+            *reinterpret_cast<uint4*>(xs + m * (C::aps * 128) + blk * 128 + ((ch ^ (m & 7)) << 4)) =
                 make_uint4(w[0], w[1], w[2], w[3]);
             if constexpr (!GIDX) {
                 float2 f[4];
@@ -557,6 +606,60 @@ W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw,
             s += __shfl_xor_sync(0xffffffffu, s, 8);
             if ((lane & 15) == 0) sx[(C::sx128 + (c >> 4)) * C::mpad + m] = s;
         }
+    }
+}
+
+// Resident activations (one token tile, small M*K): X' = X * s_inv for the whole of K and
+// its sums over every 32, 64 and 128 channels, prepared once per CTA by the warps
+// [w0, w0 + nw) straight from global memory.  X' keeps the per-stage layout, M rows per
+// 64-channel block; sums are [segment][sstride].  Consecutive lanes take consecutive
+// 8-channel chunks, so the sums are warp shuffles.
+template <bool BF16>
+W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* xr, float* sr, int w,
+                          int nw, int lane) {
+    const int cpt = p.K / 8;                       // chunks per token
+    const int ss = p.sstride;
+    float* s32 = sr;
+    float* s64 = s32 + (p.K / 32) * ss;
+    float* s128 = s64 + (p.K / 64) * ss;
+    const uint4* x4 = reinterpret_cast<const uint4*>(X);
+    for (int base = 32 * w; base < p.M * cpt; base += 32 * nw) {
+        const int item = base + lane;
+        const bool valid = item < p.M * cpt;
+        const int m = valid ? item / cpt : 0;
+        const int c = valid ? item - m * cpt : 0;
+        float s = 0.0f;
+        if (valid) {
+            uint4 v = x4[(size_t)m * cpt + c];
+            uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            if (p.s_inv) {
+                const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c);
+                const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c + 1);
+                const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = unpack2<BF16>(wv[i]);
+                    wv[i] = pack2<BF16>(__fmul_rn(f.x, sv[2 * i]), __fmul_rn(f.y, sv[2 * i + 1]));
+                }
+            }
+            const int blk = c >> 3, ch = c & 7;
+            *reinterpret_cast<uint4*>(xr + m * (p.K / 64 * 128) + blk * 128 + ((ch ^ (m & 7)) << 4)) =
+                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            float2 f[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) f[i] = unpack2<BF16>(wv[i]);
+            s = ((f[0].x + f[0].y) + (f[1].x + f[1].y)) + ((f[2].x + f[2].y) + (f[3].x + f[3].y));
+        }
+        // groups of 4 / 8 / 16 consecutive chunks never straddle two tokens when K is a
+        // multiple of 32 / 64 / 128 channels (K is a multiple of 64; the 128-channel sums
+        // are only read when K is a multiple of 128)
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        if (valid && (lane & 3) == 0) s32[(c >> 2) * ss + m] = s;
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        if (valid && (lane & 7) == 0) s64[(c >> 3) * ss + m] = s;
+        s += __shfl_xor_sync(0xffffffffu, s, 8);
+        if (valid && (lane & 15) == 0 && (c >> 4) < p.K / 128) s128[(c >> 4) * ss + m] = s;
     }
 }
 
@@ -712,7 +815,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
     const int S = p.stages;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align_smem_1024(smem_raw);
-    unsigned char* xchg = smem + S * p.stage_bytes;
+    unsigned char* xchg = smem + p.off_xchg;
     uint64_t* full = reinterpret_cast<uint64_t*>(xchg + C::xchg_bytes);
     uint64_t* xready = full + kMaxStages;
     uint64_t* empty = xready + kMaxStages;
@@ -733,7 +836,11 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
         fence_mbar_init();
     }
     // activation sums and X' rows of tokens >= M are never written: start from zero
-    {
+    if (p.xres) {
+        const int words = (p.K / 32 + p.K / 64 + p.K / 128) * p.sstride;
+        for (int i = threadIdx.x; i < words; i += C::threads)
+            reinterpret_cast<float*>(smem + p.off_res_s)[i] = 0.0f;
+    } else {
         const int words = (p.off_si - p.off_xs) / 4;   // X' and sums of one stage
         for (int i = threadIdx.x; i < S * words; i += C::threads)
             reinterpret_cast<uint32_t*>(smem + (i / words) * p.stage_bytes + p.off_xs)[i % words] = 0u;
@@ -787,8 +894,17 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                 unsigned char* st = smem + r.s * p.stage_bytes;
                 const int g_first = GIDX ? 0 : (64 * a0) / g;
                 if (lane == 0) {
-                    uint32_t bytes = na * tb * 512 + C::aps * p.M * 128;
-                    if (p.s_inv) bytes += na * 256;
+                    // stage descriptor for the consumers: {a0, na, tiles, first group row}
+                    // and, for each half, the offset of its first atom in its group and
+                    // its staged group row
+                    const int r0 = 64 * a0 - g_first * g;
+                    const int k1 = r0 + 64 * (C::aps / 2);
+                    const int g1 = GIDX ? 0 : k1 / g;
+                    int4* desc = reinterpret_cast<int4*>(st + p.off_desc);
+                    desc[0] = make_int4(a0, na, tb, g_first);
+                    desc[1] = make_int4(r0, 0, k1 - g1 * g, g1);
+                    uint32_t bytes = na * tb * 512;
+                    if (!p.xres) bytes += C::aps * p.M * 128 + (p.s_inv ? na * 256 : 0);
                     if (GIDX) bytes += na * 256;
                     else bytes += p.ngs * 256 * (p.zeros ? 2 : 1);
                     mbar_arrive_expect_tx(&full[r.s], bytes);
@@ -800,12 +916,12 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                         tma_load_2d(st + p.off_sc, &tmap_sc, band * kBandRows, g_first, &full[r.s]);
                         if (p.zeros) tma_load_2d(st + p.off_zr, &tmap_zr, band * kBandRows, g_first, &full[r.s]);
                     }
-                    if (i >= S) {
+                    if (i >= S && !p.xres) {
                         tma_load_3d(st + p.off_x, &tmap_x, 0, 0, a0, &full[r.s]);
                         if (p.s_inv) bulk_g2s(st + p.off_si, p.s_inv + 64 * a0, na * 256, &full[r.s]);
                     }
                 }
-                if (i == pro - 1) {
+                if (i == pro - 1 && !p.xres) {
                     // the activations of the first stages, once the preceding grid is done
                     pdl_wait();
                     int k = 0;
@@ -833,8 +949,17 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                 if (k >= i - S) (void)mbar_wait(&full[q.s], q.ph);
         }
         __syncwarp();
-    } else if (warp <= C::xw) {
+    } else {
+    if (p.xres) {
+        // ------------------------------------------------------------ resident X'
+        pdl_wait();   // X may come from the preceding kernel
+        prep_resident<BF16>(p, p.X, smem + p.off_res, reinterpret_cast<float*>(smem + p.off_res_s),
+                            warp - 1, C::warps - 1, lane);
+        named_bar_sync(3, C::threads - 32);
+    }
+    if (warp <= C::xw) {
         // ------------------------------------------------------------ activation warps
+        if (p.xres) return;
         const int xw = warp - 1;
         bool aborted = false;
         Ring r;
@@ -861,7 +986,9 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
         const int h = TPW == 2 ? (w8 >> 2) : 0;        // K half (two tiles per warp)
         const int t0 = TPW == 2 ? 2 * (w8 & 3) : w8;
         const int set = grp * (TPW == 2 ? 2 : 1) + h;  // partial-sum set at a flush
-        const Lane L = make_lane(lane, NT == 1 ? p.M : C::mpad);
+        const int xrows = NT == 1 ? p.M : C::mpad;
+        const int sstride = p.xres ? p.sstride : C::mpad;
+        const Lane L = make_lane(lane, xrows, sstride, p.xres ? p.K / 64 * 128 : C::aps * 128);
         float acc[TPW][NT][4];
         zero_acc<NT, TPW>(acc);
         bool aborted = false;
@@ -873,27 +1000,39 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
             const int tb = band_tiles(p, band);
             for (int stg = 0; UPS * stg < pe - ps; ++stg, ++i, r.next(S)) {
                 if ((i % C::groups) != grp) continue;   // the other group's stage
-                int a0, na;
-                stage_atoms<UPS>(p, band, ps, pe, stg, a0, na);
                 if (!aborted) {
-                    aborted = *s_abort || !mbar_wait(&xready[r.s], r.ph);
+                    aborted = *s_abort || !mbar_wait(p.xres ? &full[r.s] : &xready[r.s], r.ph);
                     if (aborted) *s_abort = 1;
                 }
+                unsigned char* st = smem + r.s * p.stage_bytes;
+                const int4 d0 = *reinterpret_cast<const int4*>(st + p.off_desc);
+                const int4 d1 = *reinterpret_cast<const int4*>(st + p.off_desc + 16);
+                const int a0 = d0.x, na = d0.y;
                 const int ab = TPW == 2 ? h * (C::aps / 2) : 0;
                 const int ae = TPW == 2 ? min(na, ab + C::aps / 2) : na;
                 if (!aborted && t0 < tb && ab < ae) {
-                    unsigned char* st = smem + r.s * p.stage_bytes;
                     StageView v;
                     v.codes = st;
-                    v.x = st + p.off_xs;
-                    v.xstride = (NT == 1 ? p.M : C::mpad) * 128;
-                    v.sx = st + p.off_sx;
+                    v.sstride = sstride;
+                    if (p.xres) {
+                        const unsigned char* rs = smem + p.off_res_s;
+                        v.x = smem + p.off_res + a0 * 128;
+                        v.sx32 = rs + (2 * a0) * sstride * 4;
+                        v.sx64 = rs + (p.K / 32 + a0) * sstride * 4;
+                        v.sx128 = rs + (p.K / 32 + p.K / 64 + a0 / 2) * sstride * 4;
+                    } else {
+                        v.x = st + p.off_xs;
+                        v.sx32 = st + p.off_sx + C::sx32 * C::mpad * 4;
+                        v.sx64 = st + p.off_sx + C::sx64 * C::mpad * 4;
+                        v.sx128 = st + p.off_sx + C::sx128 * C::mpad * 4;
+                    }
                     v.sc = st + p.off_sc;
                     v.zr = p.zeros ? st + p.off_zr : nullptr;
                     v.tb = tb;
                     v.a0 = a0;
-                    v.gfirst = GIDX ? 0 : (64 * a0) / g;
-                    v.r0 = GIDX ? 0 : 64 * a0 - v.gfirst * g;
+                    v.gfirst = d0.w;
+                    v.kin = ab == 0 ? d1.x : d1.z;
+                    v.grow = ab == 0 ? d1.y : d1.w;
                     if constexpr (GIDX) consume_gidx<NT, TPW>(v, p, L, band, t0, ab, ae, st + p.off_gi, acc);
                     else consume<NT, TPW, BF16, MODE>(v, L, t0, ab, ae, g, acc);
                 }
@@ -903,6 +1042,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
             flush_part<NT, TPW>(p, xchg, band, ps, pe, cta, set, t0, L, aborted, acc);
             zero_acc<NT, TPW>(acc);
         }
+    }
     }
 }
 

@@ -175,26 +175,40 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
                   cudaSuccess;
     });
     if (!attr_ok) return W4_ERR_CUDA;
+    // X' resident (one token tile, small M*K): X' and its sums are prepared once per CTA;
+    // the ring then carries only codes and group metadata.
+    auto up = [](int v, int a) { return (v + a - 1) / a * a; };
+    const int sstride_res = std::max(2, (int)((p.M + 1) / 2 * 2));
+    const int res_x = up(p.M * p.K * 2, 128);
+    const int res_s = up((p.K / 32 + p.K / 64 + p.K / 128) * sstride_res * 4, 128);
+    p.xres = (NT == 1 && !GIDX && res_x + res_s <= 80 * 1024) ? 1 : 0;
+    p.sstride = p.xres ? sstride_res : C::mpad;
     // stage layout: codes | activation box (M rows) | X' | activation sums | s_inv |
-    // scale rows | zero-point rows | g_idx
+    // scale rows | zero-point rows | g_idx   (no activation parts when X' is resident)
     const int g = p.group_size;
     const int span = 64 * C::aps;   // input channels per stage
     const int xrows = NT == 1 ? p.M : C::mpad;
-    auto up = [](int v, int a) { return (v + a - 1) / a * a; };
+    const bool staged_x = !p.xres;
     p.ngs = GIDX ? 0 : (g == 32 ? span / 32 : std::min(p.G, (span + 2 * g - 65) / g));
     p.off_x = C::aps * w4d::kTilesPerBand * 512;
-    p.off_xs = p.off_x + up(C::aps * p.M * 128, 1024);
-    p.off_sx = p.off_xs + up(C::aps * xrows * 128, 128);
-    p.off_si = p.off_sx + (GIDX ? 0 : C::sx_floats * 4);
-    p.off_sc = p.off_si + (p.s_inv ? C::aps * 256 : 0);
+    p.off_xs = p.off_x + (staged_x ? up(C::aps * p.M * 128, 1024) : 0);
+    p.off_sx = p.off_xs + (staged_x ? up(C::aps * xrows * 128, 128) : 0);
+    p.off_si = p.off_sx + (staged_x && !GIDX ? C::sx_floats * 4 : 0);
+    p.off_sc = p.off_si + (staged_x && p.s_inv ? C::aps * 256 : 0);
     p.off_zr = p.off_sc + p.ngs * 256;
     p.off_gi = p.off_zr + (p.zeros ? p.ngs * 256 : 0);
-    p.stage_bytes = (p.off_gi + (GIDX ? C::aps * 256 : 0) + 1023) / 1024 * 1024;
+    p.off_desc = p.off_gi + (GIDX ? C::aps * 256 : 0);
+    p.stage_bytes = (p.off_desc + 32 + 1023) / 1024 * 1024;
     // as many stages as fit: the CTA fills the SM's shared memory, one CTA per SM
-    const int fixed = C::xchg_bytes + 3 * w4d::kMaxStages * 8 + 16 + 1024;
+    const int resident = p.xres ? res_x + res_s : 0;
+    const int fixed = resident + C::xchg_bytes + 3 * w4d::kMaxStages * 8 + 16 + 1024;
     p.stages = std::min(w4d::kMaxStages, (kMaxSmem - fixed) / p.stage_bytes);
     if (p.stages < 2) return W4_ERR_UNSUPPORTED;
+    p.off_res = p.stages * p.stage_bytes;
+    p.off_res_s = p.off_res + res_x;
+    p.off_xchg = p.off_res + resident;
     const int smem = p.stages * p.stage_bytes + fixed;
+    p.X = X;
     const int bands = (p.tiles + w4d::kTilesPerBand - 1) / w4d::kTilesPerBand;
     p.KU = (p.KA + 1) / 2;
     p.units = bands * p.KU;
