@@ -109,6 +109,15 @@ W4_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_depend
 // Wait until the preceding grid has completed and its memory operations are visible.
 W4_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// One lane of a converged warp (the same lane for every caller in the warp).
+W4_DEV bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // ---------------------------------------------------------------- named barriers
 W4_DEV void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -137,6 +137,14 @@ W4_DEV uint32_t mma_idesc(bool bf16) {
            ((uint32_t)(BN >> 4) << 24);
 }
 
+// Store four 8x8 16-bit matrices from the MMA fragment layout to shared memory; each
+// lane gives the address of one 16-byte row (lanes 8i..8i+7: rows of matrix i).
+W4_DEV void stmatrix_x4(uint32_t saddr, const uint32_t (&r)[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+
 // byte offset of element (row, k) in a 128B-swizzled K-major tile (k < 64, 2-byte elems)
 W4_DEV uint32_t sw128_off(int row, int k) {
     return (uint32_t)(row * 128 + ((((k >> 3) ^ (row & 7)) & 7) << 4) + ((k & 7) << 1));
@@ -237,47 +245,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        {
+            // the whole warp runs the loop (its values stay warp-uniform); one elected lane
+            // issues each MMA and commit
+            const bool leader = elect_one();
             const uint32_t idesc = mma_idesc(BF16 && !GIDX);
-            int grp_i = -1, pb = 0;
+            // descriptors of ring slot 0; slot s is s * 16 KB further (s * 1024 in the
+            // descriptors' 16-byte address units) and each 16-channel step 32 bytes (2)
+            const uint64_t a_desc0 = sw128_desc(smem_u32(smem + L::a));
+            const uint64_t b_desc0 = sw128_desc(smem_u32(smem + L::b));
+            // group boundaries: every spg stages (g a multiple of 64), twice per stage
+            // (g = 32) or never (act-order: one partial sum over the whole K)
+            const int spg = GIDX ? KT : (g >= BK ? g / BK : 1);
+            const bool two_per_stage = !GIDX && g == 32;
+            int grp_i = -1, sig = 0;   // group counter, stage index inside the group
             bool ok = true;
-            for (int kt = 0; kt < KT && ok; ++kt) {
-                const int s = kt % kStages, ph = (kt / kStages) & 1;
-                ok = wait_or_abort(&full[s], ph, abort_flag) &&
-                     wait_or_abort(&deq[s], ph, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t a_base = smem_u32(smem + L::a + s * kABytes);
-                const uint32_t b_base = smem_u32(smem + L::b + s * kBBytes);
+            for (int kt0 = 0; kt0 < KT && ok; kt0 += kStages) {
+                const uint32_t ph = (uint32_t)((kt0 / kStages) & 1);
 #pragma unroll
-                for (int j = 0; j < BK / 16; ++j) {
-                    const int kabs = kt * BK + 16 * j;
-                    bool first, last;
-                    if (GIDX) {
-                        first = (kabs == 0);
-                        last = (kabs + 16 == p.K);
-                    } else {
-                        first = (kabs % g) == 0;
-                        last = ((kabs + 16) % g) == 0;
-                    }
-                    if (first) {
-                        ++grp_i;
-                        pb = grp_i & 1;
-                        if (grp_i >= 2) {
-                            ok = wait_or_abort(&pempty[pb], ((grp_i >> 1) - 1) & 1, abort_flag);
-                            if (!ok) break;
-                            tc_fence_after();
+                for (int s = 0; s < kStages; ++s) {
+                    const int kt = kt0 + s;
+                    if (kt >= KT) break;
+                    ok = wait_or_abort(&full[s], ph, abort_flag) && wait_or_abort(&deq[s], ph, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t ad = a_desc0 + (uint64_t)(s * (kABytes >> 4));
+                    const uint64_t bd = b_desc0 + (uint64_t)(s * (kBBytes >> 4));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        // h: 32-channel half of the stage
+                        const bool starts = two_per_stage ? true : (h == 0 && sig == 0);
+                        if (starts) {
+                            ++grp_i;
+                            if (grp_i >= 2) {
+                                ok = wait_or_abort(&pempty[grp_i & 1], ((grp_i >> 1) - 1) & 1, abort_flag);
+                                ok = __all_sync(0xffffffffu, ok);
+                                if (!ok) break;
+                                tc_fence_after();
+                            }
                         }
+                        const uint32_t dcol = tmem_base + (uint32_t)((grp_i & 1) * BM);
+                        if (leader) {
+                            tc_mma(dcol, ad + 4 * h, bd + 4 * h, idesc, starts ? 0u : 1u);
+                            tc_mma(dcol, ad + 4 * h + 2, bd + 4 * h + 2, idesc, 1u);
+                        }
+                        const bool ends = two_per_stage ? true : (h == 1 && sig == spg - 1);
+                        if (ends && leader) tc_commit(&pfull[grp_i & 1]);
                     }
-                    tc_mma(tmem_base + (uint32_t)(pb * BM), sw128_desc(a_base + 32 * j),
-                           sw128_desc(b_base + 32 * j), idesc, first ? 0u : 1u);
-                    if (last) tc_commit(&pfull[pb]);
+                    if (!ok) break;
+                    if (leader) tc_commit(&empty[s]);
+                    if (++sig == spg) sig = 0;
                 }
-                if (!ok) break;
-                tc_commit(&empty[s]);
             }
-            // every MMA this thread issued has finished once mma_done completes
-            tc_commit(mma_done);
+            // every MMA this warp issued has finished once mma_done completes
+            if (leader) tc_commit(mma_done);
             (void)mbar_wait(mma_done, 0);
         }
         __syncwarp();
@@ -285,12 +307,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ dequant warps
         const int dq = warp - 2;                 // handles row tiles 2dq, 2dq+1
         const int gq = lane >> 2, c = 2 * (lane & 3);
+        // stmatrix.x4 row addresses: lane l gives row (l & 7) of 8x8 matrix l >> 3, the
+        // matrices being (rows 0-7 | 8-15) x (channels 0-7 | 8-15) of a 16x16 step, i.e.
+        // the order of the MMA A fragment the unpack produces
+        const int mi = lane >> 3, rr = lane & 7;
         for (int kt = 0; kt < KT; ++kt) {
             const int s = kt % kStages, ph = (kt / kStages) & 1;
             if (!wait_or_abort(&full[s], ph, abort_flag)) break;
             unsigned char* a_tile = smem + L::a + s * kABytes;
+            const uint32_t a_u32 = smem_u32(a_tile);
             const unsigned char* pk = smem + L::pk + s * kPBytes;
-            const __half* zs = reinterpret_cast<const __half*>(smem + L::zr + s * kZBytes);
+            const unsigned char* zs = smem + L::zr + s * kZBytes;
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
                 const int t = 2 * dq + tt;
@@ -299,21 +326,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
                 const int r0 = 16 * t + gq, r1 = r0 + 8;       // rows within the tile
                 const int nr0 = n0 + r0, nr1 = n0 + r1;        // output rows
+                const uint32_t row_addr = a_u32 + (uint32_t)((16 * t + rr + 8 * (mi & 1)) * 128);
+                // zero-point constants of this stage's group(s) (two groups when g = 32)
+                ZeroConsts zc[2];
+                if constexpr (!GIDX) {
+#pragma unroll
+                    for (int zg = 0; zg < 2; ++zg) {
+                        const int zo = (g == 32 ? zg : 0) * BN * 2;
+                        const uint32_t z0 = p.zeros ? *reinterpret_cast<const unsigned short*>(zs + zo + 2 * r0) : 0x4800u;
+                        const uint32_t z1 = p.zeros ? *reinterpret_cast<const unsigned short*>(zs + zo + 2 * r1) : 0x4800u;
+                        zc[zg] = zero_consts_h<BF16>(z0, z1);
+                    }
+                }
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int kk = 16 * j + c;                 // column within the stage
                     const int kabs = kt * BK + kk;
                     uint32_t af[4];
                     if constexpr (!GIDX) {
-                        // zero points of this stage's group(s), staged by the producer
-                        const int zg = (g == 32) ? (j >> 1) : 0;
-                        float z0 = 8.0f, z1 = 8.0f;
-                        if (p.zeros) {
-                            z0 = __half2float(zs[zg * BN + r0]);
-                            z1 = __half2float(zs[zg * BN + r1]);
-                        }
-                        const ZeroConsts zc = BF16 ? zero_consts_bf16(z0, z1) : zero_consts_f16(z0, z1);
-                        unpack_word<BF16>(wv[j], zc, af);
+                        unpack_word<BF16>(wv[j], zc[j >> 1], af);
                     } else {
                         int gk[4] = {__ldg(p.g_idx + kabs), __ldg(p.g_idx + kabs + 1),
                                      __ldg(p.g_idx + kabs + 8), __ldg(p.g_idx + kabs + 9)};
@@ -339,10 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 __hsub2(__floats2half2_rn(qlo, qhi), __halves2half2(z_lo, z_hi)), ss));
                         }
                     }
-                    *reinterpret_cast<uint32_t*>(a_tile + sw128_off(r0, kk)) = af[0];
-                    *reinterpret_cast<uint32_t*>(a_tile + sw128_off(r1, kk)) = af[1];
-                    *reinterpret_cast<uint32_t*>(a_tile + sw128_off(r0, kk + 8)) = af[2];
-                    *reinterpret_cast<uint32_t*>(a_tile + sw128_off(r1, kk + 8)) = af[3];
+                    // 128B-swizzled K-major rows: chunk (2j + mi/2) of row r at (chunk ^ (r & 7))
+                    stmatrix_x4(row_addr + (uint32_t)((((2 * j + (mi >> 1)) ^ rr) & 7) << 4), af);
                 }
             }
             fence_proxy_async_smem();
