@@ -157,8 +157,10 @@ W4_DEV void store_out(const PrefillParams& p, int m, int n, float v) {
     else reinterpret_cast<__half*>(p.Y)[idx] = __float2half_rn(v);
 }
 
-// bounded wait that also honours the CTA's abort flag
+// bounded wait that also honours the CTA's abort flag (read only when the phase is not
+// already complete)
 W4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (mbar_wait(bar, parity)) return true;
     *abort_flag = 1;
@@ -406,10 +408,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&pempty[pb]);
         }
-        if (ok && row_ok) {
+        // Y tile through shared memory (the A ring is idle once the last group's MMAs
+        // are done): thread `row` writes column `row` of the [BM tokens][BN rows] tile,
+        // then the four warps copy it out in 16-byte pieces along N
+        const int esz = p.out_dtype == 2 ? 4 : 2;
+        unsigned char* yt = smem + L::a;
+        if (ok) {
 #pragma unroll
-            for (int i = 0; i < BM; ++i)
-                if (m0 + i < p.M) store_out(p, m0 + i, n, acc[i]);
+            for (int i = 0; i < BM; ++i) {
+                unsigned char* e = yt + (i * BN + row) * esz;
+                if (p.out_dtype == 2) *reinterpret_cast<float*>(e) = acc[i];
+                else if (p.out_dtype == 1) *reinterpret_cast<__nv_bfloat16*>(e) = __float2bfloat16_rn(acc[i]);
+                else *reinterpret_cast<__half*>(e) = __float2half_rn(acc[i]);
+            }
+        }
+        named_bar_sync(1, 128);
+        if (ok) {
+            const int cpr = BN * esz / 16;               // 16-byte pieces per token row
+            const int ncols = min(BN, p.N - n0);         // a multiple of 16 (N % 16 == 0)
+            for (int c = 32 * quad + lane; c < BM * cpr; c += 128) {
+                const int m = c / cpr, pc = c - m * cpr;
+                if (m0 + m >= p.M || pc * 16 >= ncols * esz) continue;
+                const uint4 v = *reinterpret_cast<const uint4*>(yt + m * BN * esz + pc * 16);
+                *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(p.Y) +
+                                          ((size_t)(m0 + m) * p.N + n0) * esz + pc * 16) = v;
+            }
         }
     }
 
