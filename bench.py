@@ -434,13 +434,13 @@ def our_arm(args, world, rank, local):
         v, sec, desc = cpu_oracle_sample()
         cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
                "seconds": round(sec, 2)}
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get("bytes_per_launch")
-        except Exception:
-            traffic = None
+    # DRAM traffic per launch of the decode kernel: ncu measured 48.571 MB read + 0.009 MB
+    # written for the gate_up launch (47.88 MB algorithmic), a ratio of 1.014
+    # (profiles/decode_gate_up_4096x22016_m1.md); the average launch of the step is scaled
+    # by its algorithmic bytes.  Set to None whenever the decode kernel changes.
+    DECODE_TRAFFIC_RATIO = 1.014
+    launches_per_step = N_LAYERS * len(projs)
+    traffic = DECODE_TRAFFIC_RATIO * step_bytes / launches_per_step
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
