@@ -116,10 +116,13 @@ w4_status w4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K
  * w4a16_gemm -- fused dequantise-GEMM:  Y[M,N] = X'[M,K] * What[N,K]^T, with
  *   X'[m,k]   = X[m,k] * s_inv[k]   (s_inv NULL: X' = X)   -- AWQ eq. 1, right factor
  *   What[n,k] = (q[n,k] - z[group(k),n]) * scale[group(k),n]
- * accumulated in fp32.  Without g_idx the (q - z) products are exact integers fed to
- * the tensor cores and each group's fp32 partial sum is multiplied by its scale; with
- * g_idx the scale is folded into an fp16 weight before the MMA (fp16 activations only).
- * With s_inv, X' is rounded to the activation dtype before the MMA.
+ * accumulated in fp32.  Without g_idx the codes reach the tensor cores as exact small
+ * integers and each group's fp32 partial sum is multiplied by its scale: the prefill
+ * kernel multiplies (q - z); the decode kernel multiplies the biased codes the AND/OR
+ * unpack yields (1024 + q or 1024 + 16 q in fp16, 128 + q in bf16) and removes the bias
+ * and the zero point per group with the group's activation sum, in fp32.  With g_idx the
+ * scale is folded into an fp16 weight before the MMA (fp16 activations only).  With
+ * s_inv, X' is rounded to the activation dtype before the MMA.
  *
  *   X          device [M,K] row-major, act_dtype W4_F16 or W4_BF16
  *   qweight, scales, zeros, g_idx, group_size: as produced by w4_quantize_pack
@@ -142,7 +145,7 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
                      w4_stream_t stream);
 
 /*
- * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 16 (M <= 64 where the scratch fits)
+ * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 32 (M <= 64 where the scratch fits)
  * without a caller-supplied workspace.  The pages have no counterpart to this call; it
  * exists for callers that cannot allocate device memory where they run the GEMM, such as
  * plug-ins of inference runtimes that forbid allocation after their set-up phase, or C
@@ -151,10 +154,10 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
  *
  * Arguments, layouts and results are those of w4a16_gemm minus the workspace.  The
  * scratch is one fixed 8 MiB array in device memory that every GPU loading this library
- * holds until the process exits.  Calls whose scratch would exceed it (M above 16 on a
+ * holds until the process exits.  Calls whose scratch would exceed it (M above 32 on a
  * 148-SM B200; any M > 64) return W4_ERR_UNSUPPORTED; use w4a16_gemm for them.  The
- * first call on a device sets up that device (looks up the array's address, zeroes its
- * counters and synchronises the device); make that first call before any stream
+ * first call on a device sets up that device (looks up the array's address, zeroes the
+ * array and synchronises the device); make that first call before any stream
  * capture.  Every call on a device shares the one array: calls that may overlap on the
  * GPU (different streams without ordering) race and give wrong results.  The call
  * allocates nothing and frees nothing.
