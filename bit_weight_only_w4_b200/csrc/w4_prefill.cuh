@@ -44,7 +44,8 @@ struct SmemLayout {
     static constexpr int b = a + kStages * kABytes;          // kStages x 16 KB
     static constexpr int pk = b + kStages * kBBytes;         // kStages x 4 KB
     static constexpr int zr = pk + kStages * kPBytes;        // kStages x 512 B
-    static constexpr int bars = zr + kStages * kZBytes;      // barriers
+    static constexpr int y = zr + kStages * kZBytes;         // Y tile staging, BM x BN fp32
+    static constexpr int bars = y + BM * BN * 4;             // barriers
     static constexpr int nbars = 3 * kStages + 4 + 1;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int flags = tmem_slot + 8;
@@ -184,11 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::flags);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN;       // first output row of the tile
-    const int m0 = blockIdx.y * BM;       // first token of the tile
-    const int KT = p.K / BK;              // stages along K
+    const int KT = p.K / BK;              // stages along K per tile
     const int g = p.group_size;
     const int ngroups = GIDX ? 1 : p.K / g;
+    // persistent tiles: tile t covers tokens [m0, m0+BM) of m-block t / nbands and output
+    // rows [n0, n0+BN) of band t % nbands, so the CTAs running at one time share their
+    // activation tiles (L2 reuse); a CTA takes tiles blockIdx.x, + gridDim.x, ...
+    const int nbands = (p.N + BN - 1) / BN;
+    const int ntiles = nbands * ((p.M + BM - 1) / BM);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -220,90 +224,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // this CTA's 128 rows are band blockIdx.x; its codes for column block kt are
-            // one contiguous run of tiles x 512 bytes
-            const int band = blockIdx.x;
-            const int tiles = min(BN / 16, p.tiles - n0 / 16);
-            const int zgroups = (!GIDX && p.zeros) ? (g == 32 ? 2 : 1) : 0;
-            const uint32_t bytes = kBBytes + tiles * 512 + zgroups * tiles * 32;
-            int issued = 0;
-            for (int kt = 0; kt < KT; ++kt, ++issued) {
-                const int s = kt % kStages, ph = (kt / kStages) & 1;
-                if (kt >= kStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&full[s], bytes);
-                bulk_g2s(smem + L::pk + s * kPBytes,
-                         p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)kt * tiles), tiles * 512,
-                         &full[s]);
-                for (int zg = 0; zg < zgroups; ++zg)
-                    bulk_g2s(smem + L::zr + s * kZBytes + zg * BN * 2,
-                             p.zeros + (size_t)((kt * BK) / g + zg) * p.N + n0, tiles * 32, &full[s]);
-                if (kt == 0) pdl_wait();   // activations may come from the preceding kernel
-                tma_load_2d(smem + L::b + s * kBBytes, &tmap_x, kt * BK, m0, &full[s]);
+            // the codes of band b for column block kt are one contiguous run of
+            // tiles x 512 bytes
+            int gst = 0;   // stage counter across this CTA's tiles (ring slot, phase)
+            bool waited = false;
+            for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+                const int band = t % nbands;
+                const int n0 = band * BN, m0 = (t / nbands) * BM;
+                const int tiles = min(BN / 16, p.tiles - n0 / 16);
+                const int zgroups = (!GIDX && p.zeros) ? (g == 32 ? 2 : 1) : 0;
+                const uint32_t bytes = kBBytes + tiles * 512 + zgroups * tiles * 32;
+                for (int kt = 0; kt < KT; ++kt, ++gst) {
+                    const int s = gst % kStages, ph = (gst / kStages) & 1;
+                    if (gst >= kStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    bulk_g2s(smem + L::pk + s * kPBytes,
+                             p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)kt * tiles), tiles * 512,
+                             &full[s]);
+                    for (int zg = 0; zg < zgroups; ++zg)
+                        bulk_g2s(smem + L::zr + s * kZBytes + zg * BN * 2,
+                                 p.zeros + (size_t)((kt * BK) / g + zg) * p.N + n0, tiles * 32, &full[s]);
+                    if (!waited) {
+                        pdl_wait();   // activations may come from the preceding kernel
+                        waited = true;
+                    }
+                    tma_load_2d(smem + L::b + s * kBBytes, &tmap_x, kt * BK, m0, &full[s]);
+                }
             }
             if (*abort_flag)
-                for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+                for (int i = (gst > kStages ? gst - kStages : 0); i < gst; ++i)
                     (void)mbar_wait(&full[i % kStages], (i / kStages) & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        {
-            // the whole warp runs the loop (its values stay warp-uniform); one elected lane
-            // issues each MMA and commit
-            const bool leader = elect_one();
-            const uint32_t idesc = mma_idesc(BF16 && !GIDX);
-            // descriptors of ring slot 0; slot s is s * 16 KB further (s * 1024 in the
-            // descriptors' 16-byte address units) and each 16-channel step 32 bytes (2)
-            const uint64_t a_desc0 = sw128_desc(smem_u32(smem + L::a));
-            const uint64_t b_desc0 = sw128_desc(smem_u32(smem + L::b));
-            // group boundaries: every spg stages (g a multiple of 64), twice per stage
-            // (g = 32) or never (act-order: one partial sum over the whole K)
-            const int spg = GIDX ? KT : (g >= BK ? g / BK : 1);
-            const bool two_per_stage = !GIDX && g == 32;
-            int grp_i = -1, sig = 0;   // group counter, stage index inside the group
-            bool ok = true;
-            for (int kt0 = 0; kt0 < KT && ok; kt0 += kStages) {
-                const uint32_t ph = (uint32_t)((kt0 / kStages) & 1);
-#pragma unroll
-                for (int s = 0; s < kStages; ++s) {
-                    const int kt = kt0 + s;
-                    if (kt >= KT) break;
-                    ok = wait_or_abort(&full[s], ph, abort_flag) && wait_or_abort(&deq[s], ph, abort_flag);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint64_t ad = a_desc0 + (uint64_t)(s * (kABytes >> 4));
-                    const uint64_t bd = b_desc0 + (uint64_t)(s * (kBBytes >> 4));
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        // h: 32-channel half of the stage
-                        const bool starts = two_per_stage ? true : (h == 0 && sig == 0);
-                        if (starts) {
-                            ++grp_i;
-                            if (grp_i >= 2) {
-                                ok = wait_or_abort(&pempty[grp_i & 1], ((grp_i >> 1) - 1) & 1, abort_flag);
-                                ok = __all_sync(0xffffffffu, ok);
-                                if (!ok) break;
-                                tc_fence_after();
-                            }
-                        }
-                        const uint32_t dcol = tmem_base + (uint32_t)((grp_i & 1) * BM);
-                        if (leader) {
-                            tc_mma(dcol, ad + 4 * h, bd + 4 * h, idesc, starts ? 0u : 1u);
-                            tc_mma(dcol, ad + 4 * h + 2, bd + 4 * h + 2, idesc, 1u);
-                        }
-                        const bool ends = two_per_stage ? true : (h == 1 && sig == spg - 1);
-                        if (ends && leader) tc_commit(&pfull[grp_i & 1]);
-                    }
-                    if (!ok) break;
-                    if (leader) tc_commit(&empty[s]);
-                    if (++sig == spg) sig = 0;
+        // the whole warp runs the loop (its values stay warp-uniform); one elected lane
+        // issues each MMA and commit
+        const bool leader = elect_one();
+        const uint32_t idesc = mma_idesc(BF16 && !GIDX);
+        // descriptors of ring slot 0; slot s is s * 16 KB further (s * 1024 in the
+        // descriptors' 16-byte address units) and each 16-channel step 32 bytes (2)
+        const uint64_t a_desc0 = sw128_desc(smem_u32(smem + L::a));
+        const uint64_t b_desc0 = sw128_desc(smem_u32(smem + L::b));
+        // group boundaries: every spg stages (g a multiple of 64), twice per stage
+        // (g = 32) or once per tile (act-order: one partial sum over the whole K)
+        const int spg = GIDX ? KT : (g >= BK ? g / BK : 1);
+        const bool two_per_stage = !GIDX && g == 32;
+        int grp_i = -1;   // group counter across this CTA's tiles (partial buffer, phase)
+        int gst = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            int sig = 0;   // stage index inside the current group
+            for (int kt = 0; kt < KT; ++kt, ++gst) {
+                const int s = gst % kStages;
+                const uint32_t ph = (uint32_t)((gst / kStages) & 1);
+                // the dequant warps arrive on deq[s] only after full[s] completed (its
+                // activation tile landed), so deq[s] alone orders the MMA after both
+                ok = wait_or_abort(&deq[s], ph, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                const uint64_t ad = a_desc0 + (uint64_t)(s * (kABytes >> 4));
+                const uint64_t bd = b_desc0 + (uint64_t)(s * (kBBytes >> 4));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    // h: 32-channel half of the stage
+                    const bool starts = two_per_stage ? true : (h == 0 && sig == 0);
+                    if (starts) {
+                        ++grp_i;
+                        if (grp_i >= 2) {
+                            ok = wait_or_abort(&pempty[grp_i & 1], ((grp_i >> 1) - 1) & 1, abort_flag);
+                            ok = __all_sync(0xffffffffu, ok);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                    }
+                    const uint32_t dcol = tmem_base + (uint32_t)((grp_i & 1) * BM);
+                    if (leader) {
+                        tc_mma(dcol, ad + 4 * h, bd + 4 * h, idesc, starts ? 0u : 1u);
+                        tc_mma(dcol, ad + 4 * h + 2, bd + 4 * h + 2, idesc, 1u);
+                    }
+                    const bool ends = two_per_stage ? true : (h == 1 && sig == spg - 1);
+                    if (ends && leader) tc_commit(&pfull[grp_i & 1]);
+                }
+                if (!ok) break;
+                if (leader) tc_commit(&empty[s]);
+                if (++sig == spg) sig = 0;
             }
-            // every MMA this warp issued has finished once mma_done completes
-            if (leader) tc_commit(mma_done);
-            (void)mbar_wait(mma_done, 0);
         }
+        // every MMA this warp issued has finished once mma_done completes
+        if (leader) tc_commit(mma_done);
+        (void)mbar_wait(mma_done, 0);
         __syncwarp();
     } else if (warp < 6) {
         // ------------------------------------------------------------ dequant warps
@@ -313,9 +326,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // matrices being (rows 0-7 | 8-15) x (channels 0-7 | 8-15) of a 16x16 step, i.e.
         // the order of the MMA A fragment the unpack produces
         const int mi = lane >> 3, rr = lane & 7;
-        for (int kt = 0; kt < KT; ++kt) {
-            const int s = kt % kStages, ph = (kt / kStages) & 1;
-            if (!wait_or_abort(&full[s], ph, abort_flag)) break;
+        int gst = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const int n0 = (t % nbands) * BN;
+        for (int kt = 0; kt < KT; ++kt, ++gst) {
+            const int s = gst % kStages, ph = (gst / kStages) & 1;
+            if (!wait_or_abort(&full[s], ph, abort_flag)) {
+                ok = false;
+                break;
+            }
             unsigned char* a_tile = smem + L::a + s * kABytes;
             const uint32_t a_u32 = smem_u32(a_tile);
             const unsigned char* pk = smem + L::pk + s * kPBytes;
@@ -379,60 +399,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             mbar_arrive(&deq[s]);
         }
+        }
     } else {
         // ------------------------------------------------------------ epilogue warps
         pdl_wait();   // before any store to Y
         const int quad = warp & 3;                 // tensor-memory lanes 32*quad..
         const int row = 32 * quad + lane;          // output row within the tile
-        const int n = n0 + row;
-        const bool row_ok = n < p.N;
-        float acc[BM];
-#pragma unroll
-        for (int i = 0; i < BM; ++i) acc[i] = 0.0f;
-        bool ok = true;
-        for (int grp_i = 0; grp_i < ngroups && ok; ++grp_i) {
-            const int pb = grp_i & 1;
-            float sc = 1.0f;
-            if (!GIDX && row_ok) sc = __half2float(__ldg(p.scales + (size_t)grp_i * p.N + n));
-            ok = wait_or_abort(&pfull[pb], (grp_i >> 1) & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(pb * BM);
-#pragma unroll
-            for (int ch = 0; ch < BM / 32; ++ch) {
-                float v[32];
-                tmem_ld32(taddr + 32 * ch, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) acc[32 * ch + i] = fmaf(sc, v[i], acc[32 * ch + i]);
-            }
-            tc_fence_before();
-            mbar_arrive(&pempty[pb]);
-        }
-        // Y tile through shared memory (the A ring is idle once the last group's MMAs
-        // are done): thread `row` writes column `row` of the [BM tokens][BN rows] tile,
-        // then the four warps copy it out in 16-byte pieces along N
         const int esz = p.out_dtype == 2 ? 4 : 2;
-        unsigned char* yt = smem + L::a;
-        if (ok) {
+        unsigned char* yt = smem + L::y;
+        int ge = 0;   // group counter across this CTA's tiles (partial buffer, phase)
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            const int n0 = (t % nbands) * BN, m0 = (t / nbands) * BM;
+            const int n = n0 + row;
+            const bool row_ok = n < p.N;
+            float acc[BM];
 #pragma unroll
-            for (int i = 0; i < BM; ++i) {
-                unsigned char* e = yt + (i * BN + row) * esz;
-                if (p.out_dtype == 2) *reinterpret_cast<float*>(e) = acc[i];
-                else if (p.out_dtype == 1) *reinterpret_cast<__nv_bfloat16*>(e) = __float2bfloat16_rn(acc[i]);
-                else *reinterpret_cast<__half*>(e) = __float2half_rn(acc[i]);
+            for (int i = 0; i < BM; ++i) acc[i] = 0.0f;
+            for (int grp = 0; grp < ngroups && ok; ++grp, ++ge) {
+                const int pb = ge & 1;
+                float sc = 1.0f;
+                if (!GIDX && row_ok) sc = __half2float(__ldg(p.scales + (size_t)grp * p.N + n));
+                ok = wait_or_abort(&pfull[pb], (ge >> 1) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(pb * BM);
+#pragma unroll
+                for (int ch = 0; ch < BM / 32; ++ch) {
+                    float v[32];
+                    tmem_ld32(taddr + 32 * ch, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[32 * ch + i] = fmaf(sc, v[i], acc[32 * ch + i]);
+                }
+                tc_fence_before();
+                mbar_arrive(&pempty[pb]);
             }
-        }
-        named_bar_sync(1, 128);
-        if (ok) {
-            const int cpr = BN * esz / 16;               // 16-byte pieces per token row
-            const int ncols = min(BN, p.N - n0);         // a multiple of 16 (N % 16 == 0)
-            for (int c = 32 * quad + lane; c < BM * cpr; c += 128) {
-                const int m = c / cpr, pc = c - m * cpr;
-                if (m0 + m >= p.M || pc * 16 >= ncols * esz) continue;
-                const uint4 v = *reinterpret_cast<const uint4*>(yt + m * BN * esz + pc * 16);
-                *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(p.Y) +
-                                          ((size_t)(m0 + m) * p.N + n0) * esz + pc * 16) = v;
+            // Y tile through its own shared buffer: thread `row` writes column `row` of the
+            // [BM tokens][BN rows] tile, then the four warps copy it out in 16-byte pieces
+            // along N.  The next tile's MMAs proceed meanwhile.
+            if (ok) {
+#pragma unroll
+                for (int i = 0; i < BM; ++i) {
+                    unsigned char* e = yt + (i * BN + row) * esz;
+                    if (p.out_dtype == 2) *reinterpret_cast<float*>(e) = acc[i];
+                    else if (p.out_dtype == 1) *reinterpret_cast<__nv_bfloat16*>(e) = __float2bfloat16_rn(acc[i]);
+                    else *reinterpret_cast<__half*>(e) = __float2half_rn(acc[i]);
+                }
             }
+            named_bar_sync(1, 128);
+            if (ok) {
+                const int cpr = BN * esz / 16;               // 16-byte pieces per token row
+                const int ncols = min(BN, p.N - n0);         // a multiple of 16 (N % 16 == 0)
+                for (int c = 32 * quad + lane; c < BM * cpr; c += 128) {
+                    const int m = c / cpr, pc = c - m * cpr;
+                    if (m0 + m >= p.M || pc * 16 >= ncols * esz) continue;
+                    const uint4 v = *reinterpret_cast<const uint4*>(yt + m * BN * esz + pc * 16);
+                    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(p.Y) +
+                                              ((size_t)(m0 + m) * p.N + n0) * esz + pc * 16) = v;
+                }
+            }
+            named_bar_sync(1, 128);   // the buffer is free for the next tile
         }
     }
 

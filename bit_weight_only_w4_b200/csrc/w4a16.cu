@@ -283,7 +283,11 @@ w4_status launch_prefill(const CUtensorMap& map, const w4p::PrefillParams& p, in
     static std::once_flag flags[kMaxDevices];
     auto k = w4p::prefill_kernel<BF16, GIDX>;
     if (!ensure_smem(k, w4p::SmemLayout::bytes, flags, dev)) return W4_ERR_CUDA;
-    const dim3 grid((unsigned)((p.N + w4p::BN - 1) / w4p::BN), (unsigned)((p.M + w4p::BM - 1) / w4p::BM));
+    // persistent: one CTA per SM (or per tile when there are fewer tiles)
+    const long long ntiles = (long long)((p.N + w4p::BN - 1) / w4p::BN) * ((p.M + w4p::BM - 1) / w4p::BM);
+    const int sms = sm_count(dev);
+    if (sms <= 0) return W4_ERR_CUDA;
+    const dim3 grid((unsigned)std::min<long long>(ntiles, sms));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(w4p::kThreads);
