@@ -26,26 +26,38 @@
 
 namespace w4p {
 
-constexpr int BN = 128;        // output rows per CTA (MMA M)
+constexpr int BN = 256;        // output rows per CTA: two 128-row halves (MMA M = 128 each)
+constexpr int BH = 128;        // rows per half
 constexpr int BM = 128;        // tokens per CTA (MMA N)
 constexpr int BK = 64;         // input channels per stage (one 128-byte swizzle row)
-constexpr int kStages = 4;
-constexpr int kThreads = 320;
-constexpr int kTmemCols = 256; // two fp32 partial buffers of BM columns
+constexpr int kStages = 3;
+constexpr int kThreads = 512;  // producer, MMA, 6 dequant, 8 epilogue warps (4 warpgroups)
+constexpr int kDequantWarps = 6;
+// Register split: launched with 128 registers a thread (512 x 128 = the SM's 65536);
+// warpgroups 0-1 (producer, MMA, dequant) give theirs down to kRegsLow, warpgroups 2-3
+// (epilogue: 128 fp32 accumulators a thread) take kRegsHigh.  2 x 128 x 88 + 2 x 128 x
+// 168 = 65536, exactly the launch's registers.
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsLow = 88;
+constexpr int kRegsHigh = 168;
+static_assert(2 * 128 * kRegsLow + 2 * 128 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
+constexpr int kTmemCols = 512; // two fp32 partial buffers x two halves x BM columns
+constexpr int kYChunk = 32;    // tokens per pass of the output staging buffer
 
-constexpr int kABytes = BN * BK * 2;   // 16 KB
+constexpr int kAHalf = BH * BK * 2;    // 16 KB: one half's dequantised operand tile
+constexpr int kABytes = 2 * kAHalf;    // 32 KB
 constexpr int kBBytes = BM * BK * 2;   // 16 KB
-constexpr int kPBytes = BN * BK / 2;   // 4 KB packed codes
+constexpr int kPBytes = BN * BK / 2;   // 8 KB packed codes (two 128-row bands)
 constexpr int kZBytes = 2 * BN * 2;    // zero-point rows of up to two groups
 constexpr int kStageBytes = kABytes + kBBytes + kPBytes + kZBytes;
 
 struct SmemLayout {
-    static constexpr int a = 0;                              // kStages x 16 KB (1024-aligned)
+    static constexpr int a = 0;                              // kStages x 32 KB (1024-aligned)
     static constexpr int b = a + kStages * kABytes;          // kStages x 16 KB
-    static constexpr int pk = b + kStages * kBBytes;         // kStages x 4 KB
-    static constexpr int zr = pk + kStages * kPBytes;        // kStages x 512 B
-    static constexpr int y = zr + kStages * kZBytes;         // Y tile staging, BM x BN fp32
-    static constexpr int bars = y + BM * BN * 4;             // barriers
+    static constexpr int pk = b + kStages * kBBytes;         // kStages x 8 KB
+    static constexpr int zr = pk + kStages * kPBytes;        // kStages x 1 KB
+    static constexpr int y = zr + kStages * kZBytes;         // output staging: kYChunk x BN fp32
+    static constexpr int bars = y + kYChunk * BN * 4;        // barriers
     static constexpr int nbars = 3 * kStages + 4 + 1;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int flags = tmem_slot + 8;
@@ -131,11 +143,23 @@ W4_DEV uint64_t sw128_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor: fp32 accumulator, A/B fp16 (0) or bf16 (1), both K-major,
-// N = BM, M = BN.
+// N = BM tokens, M = BH rows (one half; a single-CTA MMA is at most 128 rows).
 W4_DEV uint32_t mma_idesc(bool bf16) {
     const uint32_t fmt = bf16 ? 1u : 0u;
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(BM >> 3) << 17) |
-           ((uint32_t)(BN >> 4) << 24);
+           ((uint32_t)(BH >> 4) << 24);
+}
+
+// Per-warpgroup register limits (executed by all 128 threads of a warpgroup).  An increase
+// waits until the registers are free, so the split must fit the launch's registers; the
+// host launches the kernel only when it was compiled with kLaunchRegs registers a thread.
+template <uint32_t N>
+W4_DEV void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+W4_DEV void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Store four 8x8 16-bit matrices from the MMA fragment layout to shared memory; each
@@ -189,20 +213,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = p.group_size;
     const int ngroups = GIDX ? 1 : p.K / g;
     // persistent tiles: tile t covers tokens [m0, m0+BM) of m-block t / nbands and output
-    // rows [n0, n0+BN) of band t % nbands, so the CTAs running at one time share their
-    // activation tiles (L2 reuse); a CTA takes tiles blockIdx.x, + gridDim.x, ...
+    // rows [n0, n0+BN) of row block t % nbands, so the CTAs running at one time share
+    // their activation tiles (L2 reuse); a CTA takes tiles blockIdx.x, + gridDim.x, ...
     const int nbands = (p.N + BN - 1) / BN;
     const int ntiles = nbands * ((p.M + BM - 1) / BM);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&deq[s], 128);
+            mbar_init(&deq[s], 32 * kDequantWarps);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&pfull[b], 1);
-            mbar_init(&pempty[b], 128);
+            mbar_init(&pempty[b], 256);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -220,30 +244,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     // The next kernel may be scheduled while this grid runs; codes and zero points, read
     // before pdl_wait(), are never written by the kernels of this library.
     pdl_launch_dependents();
-
+    if (warp < 8) {
+    // warpgroups 0-1: producer, MMA issuer, dequant warps (few registers each)
+    setmaxnreg_dec<kRegsLow>();
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // the codes of band b for column block kt are one contiguous run of
-            // tiles x 512 bytes
+            // the codes of one 128-row band for column block kt are one contiguous run of
+            // tiles x 512 bytes; a tile of BN rows spans two bands
             int gst = 0;   // stage counter across this CTA's tiles (ring slot, phase)
             bool waited = false;
             for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
-                const int band = t % nbands;
-                const int n0 = band * BN, m0 = (t / nbands) * BM;
-                const int tiles = min(BN / 16, p.tiles - n0 / 16);
+                const int rb = t % nbands;
+                const int n0 = rb * BN, m0 = (t / nbands) * BM;
+                int th[2];                                   // tiles of each half
+                for (int h = 0; h < 2; ++h) th[h] = max(0, min(BH / 16, p.tiles - (n0 + h * BH) / 16));
                 const int zgroups = (!GIDX && p.zeros) ? (g == 32 ? 2 : 1) : 0;
-                const uint32_t bytes = kBBytes + tiles * 512 + zgroups * tiles * 32;
+                const uint32_t bytes = kBBytes + (th[0] + th[1]) * (512 + zgroups * 32);
                 for (int kt = 0; kt < KT; ++kt, ++gst) {
                     const int s = gst % kStages, ph = (gst / kStages) & 1;
                     if (gst >= kStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
                     mbar_arrive_expect_tx(&full[s], bytes);
-                    bulk_g2s(smem + L::pk + s * kPBytes,
-                             p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)kt * tiles), tiles * 512,
-                             &full[s]);
-                    for (int zg = 0; zg < zgroups; ++zg)
-                        bulk_g2s(smem + L::zr + s * kZBytes + zg * BN * 2,
-                                 p.zeros + (size_t)((kt * BK) / g + zg) * p.N + n0, tiles * 32, &full[s]);
+                    for (int h = 0; h < 2; ++h) {
+                        if (th[h] == 0) continue;
+                        const int band = 2 * rb + h;
+                        bulk_g2s(smem + L::pk + s * kPBytes + h * (kPBytes / 2),
+                                 p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)kt * th[h]), th[h] * 512,
+                                 &full[s]);
+                        for (int zg = 0; zg < zgroups; ++zg)
+                            bulk_g2s(smem + L::zr + s * kZBytes + zg * BN * 2 + h * BH * 2,
+                                     p.zeros + (size_t)((kt * BK) / g + zg) * p.N + n0 + h * BH, th[h] * 32,
+                                     &full[s]);
+                    }
                     if (!waited) {
                         pdl_wait();   // activations may come from the preceding kernel
                         waited = true;
@@ -259,11 +291,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         // the whole warp runs the loop (its values stay warp-uniform); one elected lane
-        // issues each MMA and commit
+        // issues each MMA and commit.  Per 16-channel step: one 128x128x16 MMA per half,
+        // both against the same activation tile.
         const bool leader = elect_one();
         const uint32_t idesc = mma_idesc(BF16 && !GIDX);
-        // descriptors of ring slot 0; slot s is s * 16 KB further (s * 1024 in the
-        // descriptors' 16-byte address units) and each 16-channel step 32 bytes (2)
+        // descriptors of ring slot 0; slot s, half h and 16-channel step j are
+        // s * kABytes + h * kAHalf + 32 j bytes further (>> 4 in the descriptors)
         const uint64_t a_desc0 = sw128_desc(smem_u32(smem + L::a));
         const uint64_t b_desc0 = sw128_desc(smem_u32(smem + L::b));
         // group boundaries: every spg stages (g a multiple of 64), twice per stage
@@ -289,9 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t ad = a_desc0 + (uint64_t)(s * (kABytes >> 4));
                 const uint64_t bd = b_desc0 + (uint64_t)(s * (kBBytes >> 4));
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    // h: 32-channel half of the stage
-                    const bool starts = two_per_stage ? true : (h == 0 && sig == 0);
+                for (int hk = 0; hk < 2; ++hk) {
+                    // hk: 32-channel half of the stage
+                    const bool starts = two_per_stage ? true : (hk == 0 && sig == 0);
                     if (starts) {
                         ++grp_i;
                         if (grp_i >= 2) {
@@ -301,12 +334,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                         }
                     }
-                    const uint32_t dcol = tmem_base + (uint32_t)((grp_i & 1) * BM);
+                    const uint32_t dcol = tmem_base + (uint32_t)((grp_i & 1) * 2 * BM);
                     if (leader) {
-                        tc_mma(dcol, ad + 4 * h, bd + 4 * h, idesc, starts ? 0u : 1u);
-                        tc_mma(dcol, ad + 4 * h + 2, bd + 4 * h + 2, idesc, 1u);
+#pragma unroll
+                        for (int j = 0; j < 2; ++j)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                tc_mma(dcol + h * BM, ad + h * (kAHalf >> 4) + 4 * hk + 2 * j, bd + 4 * hk + 2 * j,
+                                       idesc, (starts && j == 0) ? 0u : 1u);
                     }
-                    const bool ends = two_per_stage ? true : (h == 1 && sig == spg - 1);
+                    const bool ends = two_per_stage ? true : (hk == 1 && sig == spg - 1);
                     if (ends && leader) tc_commit(&pfull[grp_i & 1]);
                 }
                 if (!ok) break;
@@ -318,9 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) tc_commit(mma_done);
         (void)mbar_wait(mma_done, 0);
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp < 8) {
         // ------------------------------------------------------------ dequant warps
-        const int dq = warp - 2;                 // handles row tiles 2dq, 2dq+1
+        const int dq = warp - 2;                 // row tiles dq, dq + 6, dq + 12 of the 16
         const int gq = lane >> 2, c = 2 * (lane & 3);
         // stmatrix.x4 row addresses: lane l gives row (l & 7) of 8x8 matrix l >> 3, the
         // matrices being (rows 0-7 | 8-15) x (channels 0-7 | 8-15) of a 16x16 step, i.e.
@@ -329,82 +366,87 @@ __global__ void __launch_bounds__(kThreads, 1)
         int gst = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const int n0 = (t % nbands) * BN;
-        for (int kt = 0; kt < KT; ++kt, ++gst) {
-            const int s = gst % kStages, ph = (gst / kStages) & 1;
-            if (!wait_or_abort(&full[s], ph, abort_flag)) {
-                ok = false;
-                break;
-            }
-            unsigned char* a_tile = smem + L::a + s * kABytes;
-            const uint32_t a_u32 = smem_u32(a_tile);
-            const unsigned char* pk = smem + L::pk + s * kPBytes;
-            const unsigned char* zs = smem + L::zr + s * kZBytes;
-#pragma unroll
-            for (int tt = 0; tt < 2; ++tt) {
-                const int t = 2 * dq + tt;
-                if (n0 / 16 + t >= p.tiles) continue;
-                const uint4 wq = *reinterpret_cast<const uint4*>(pk + t * 512 + lane * 16);
-                const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-                const int r0 = 16 * t + gq, r1 = r0 + 8;       // rows within the tile
-                const int nr0 = n0 + r0, nr1 = n0 + r1;        // output rows
-                const uint32_t row_addr = a_u32 + (uint32_t)((16 * t + rr + 8 * (mi & 1)) * 128);
-                // zero-point constants of this stage's group(s) (two groups when g = 32)
-                ZeroConsts zc[2];
-                if constexpr (!GIDX) {
-#pragma unroll
-                    for (int zg = 0; zg < 2; ++zg) {
-                        const int zo = (g == 32 ? zg : 0) * BN * 2;
-                        const uint32_t z0 = p.zeros ? *reinterpret_cast<const unsigned short*>(zs + zo + 2 * r0) : 0x4800u;
-                        const uint32_t z1 = p.zeros ? *reinterpret_cast<const unsigned short*>(zs + zo + 2 * r1) : 0x4800u;
-                        zc[zg] = zero_consts_h<BF16>(z0, z1);
-                    }
+            const int n0 = (t % nbands) * BN;
+            const int tt_end = max(0, min(BN / 16, p.tiles - n0 / 16));   // tiles of the tile
+            for (int kt = 0; kt < KT; ++kt, ++gst) {
+                const int s = gst % kStages, ph = (gst / kStages) & 1;
+                if (!wait_or_abort(&full[s], ph, abort_flag)) {
+                    ok = false;
+                    break;
                 }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int kk = 16 * j + c;                 // column within the stage
-                    const int kabs = kt * BK + kk;
-                    uint32_t af[4];
+#pragma unroll 1
+                for (int ti = dq; ti < BN / 16; ti += kDequantWarps) {
+                    if (ti >= tt_end) break;
+                    const int hh = ti >> 3, tt = ti & 7;          // half, tile within the half
+                    const uint32_t a_u32 = smem_u32(smem + L::a + s * kABytes + hh * kAHalf);
+                    const unsigned char* pk = smem + L::pk + s * kPBytes + hh * (kPBytes / 2);
+                    const unsigned char* zs = smem + L::zr + s * kZBytes + hh * BH * 2;
+                    const uint4 wq = *reinterpret_cast<const uint4*>(pk + tt * 512 + lane * 16);
+                    const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+                    const int r0 = 16 * tt + gq, r1 = r0 + 8;      // rows within the half
+                    const int nr0 = n0 + hh * BH + r0, nr1 = nr0 + 8;  // output rows
+                    const uint32_t row_addr = a_u32 + (uint32_t)((16 * tt + rr + 8 * (mi & 1)) * 128);
+                    // zero-point constants of this stage's group(s) (two groups when g = 32)
+                    ZeroConsts zc[2];
                     if constexpr (!GIDX) {
-                        unpack_word<BF16>(wv[j], zc[j >> 1], af);
-                    } else {
-                        int gk[4] = {__ldg(p.g_idx + kabs), __ldg(p.g_idx + kabs + 1),
-                                     __ldg(p.g_idx + kabs + 8), __ldg(p.g_idx + kabs + 9)};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if (gk[e] < 0 || gk[e] >= p.G) {
-                                atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
-                                gk[e] = 0;
-                            }
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int row = (r & 1) ? nr1 : nr0;
-                            const int kl = (r & 2) ? 2 : 0;
-                            const float qlo = (float)((wv[j] >> (4 * r)) & 0xF);
-                            const float qhi = (float)((wv[j] >> (4 * (r + 4))) & 0xF);
-                            const __half z_lo = p.zeros ? __ldg(p.zeros + (size_t)gk[kl] * p.N + row)
-                                                        : __float2half_rn(8.0f);
-                            const __half z_hi = p.zeros ? __ldg(p.zeros + (size_t)gk[kl + 1] * p.N + row)
-                                                        : __float2half_rn(8.0f);
-                            const __half2 ss = __halves2half2(__ldg(p.scales + (size_t)gk[kl] * p.N + row),
-                                                              __ldg(p.scales + (size_t)gk[kl + 1] * p.N + row));
-                            af[r] = h2_as_u32(__hmul2(
-                                __hsub2(__floats2half2_rn(qlo, qhi), __halves2half2(z_lo, z_hi)), ss));
+                        for (int zg = 0; zg < 2; ++zg) {
+                            const int zo = (g == 32 ? zg : 0) * BN * 2;
+                            const uint32_t z0 = p.zeros ? *reinterpret_cast<const unsigned short*>(zs + zo + 2 * r0) : 0x4800u;
+                            const uint32_t z1 = p.zeros ? *reinterpret_cast<const unsigned short*>(zs + zo + 2 * r1) : 0x4800u;
+                            zc[zg] = zero_consts_h<BF16>(z0, z1);
                         }
                     }
-                    // 128B-swizzled K-major rows: chunk (2j + mi/2) of row r at (chunk ^ (r & 7))
-                    stmatrix_x4(row_addr + (uint32_t)((((2 * j + (mi >> 1)) ^ rr) & 7) << 4), af);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int kk = 16 * j + c;                 // column within the stage
+                        const int kabs = kt * BK + kk;
+                        uint32_t af[4];
+                        if constexpr (!GIDX) {
+                            unpack_word<BF16>(wv[j], zc[j >> 1], af);
+                        } else {
+                            int gk[4] = {__ldg(p.g_idx + kabs), __ldg(p.g_idx + kabs + 1),
+                                         __ldg(p.g_idx + kabs + 8), __ldg(p.g_idx + kabs + 9)};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                if (gk[e] < 0 || gk[e] >= p.G) {
+                                    atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
+                                    gk[e] = 0;
+                                }
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) {
+                                const int row = (r & 1) ? nr1 : nr0;
+                                const int kl = (r & 2) ? 2 : 0;
+                                const float qlo = (float)((wv[j] >> (4 * r)) & 0xF);
+                                const float qhi = (float)((wv[j] >> (4 * (r + 4))) & 0xF);
+                                const __half z_lo = p.zeros ? __ldg(p.zeros + (size_t)gk[kl] * p.N + row)
+                                                            : __float2half_rn(8.0f);
+                                const __half z_hi = p.zeros ? __ldg(p.zeros + (size_t)gk[kl + 1] * p.N + row)
+                                                            : __float2half_rn(8.0f);
+                                const __half2 ss = __halves2half2(__ldg(p.scales + (size_t)gk[kl] * p.N + row),
+                                                                  __ldg(p.scales + (size_t)gk[kl + 1] * p.N + row));
+                                af[r] = h2_as_u32(__hmul2(
+                                    __hsub2(__floats2half2_rn(qlo, qhi), __halves2half2(z_lo, z_hi)), ss));
+                            }
+                        }
+                        // 128B-swizzled K-major rows: chunk (2j + mi/2) of row r at (chunk ^ (r & 7))
+                        stmatrix_x4(row_addr + (uint32_t)((((2 * j + (mi >> 1)) ^ rr) & 7) << 4), af);
+                    }
                 }
+                fence_proxy_async_smem();
+                mbar_arrive(&deq[s]);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&deq[s]);
         }
-        }
+    }
     } else {
         // ------------------------------------------------------------ epilogue warps
+        // warpgroups 2-3: 128 fp32 accumulators a thread
+        setmaxnreg_inc<kRegsHigh>();
         pdl_wait();   // before any store to Y
+        const int e = warp - 8;
         const int quad = warp & 3;                 // tensor-memory lanes 32*quad..
-        const int row = 32 * quad + lane;          // output row within the tile
+        const int h = e >> 2;                      // half
+        const int row = h * BH + 32 * quad + lane; // output row within the tile
         const int esz = p.out_dtype == 2 ? 4 : 2;
         unsigned char* yt = smem + L::y;
         int ge = 0;   // group counter across this CTA's tiles (partial buffer, phase)
@@ -423,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = wait_or_abort(&pfull[pb], (ge >> 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(pb * BM);
+                const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(pb * 2 * BM + h * BM);
 #pragma unroll
                 for (int ch = 0; ch < BM / 32; ++ch) {
                     float v[32];
@@ -434,31 +476,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&pempty[pb]);
             }
-            // Y tile through its own shared buffer: thread `row` writes column `row` of the
-            // [BM tokens][BN rows] tile, then the four warps copy it out in 16-byte pieces
-            // along N.  The next tile's MMAs proceed meanwhile.
-            if (ok) {
+            // Y tile through a staging buffer of kYChunk tokens: thread `row` writes column
+            // `row` of a [kYChunk tokens][BN rows] block, then the eight warps copy it out in
+            // 16-byte pieces along N.  The next tile's MMAs proceed meanwhile.
+            const int cpr = BN * esz / 16;               // 16-byte pieces per token row
+            const int ncols = min(BN, p.N - n0);         // a multiple of 16 (N % 16 == 0)
 #pragma unroll
-                for (int i = 0; i < BM; ++i) {
-                    unsigned char* e = yt + (i * BN + row) * esz;
-                    if (p.out_dtype == 2) *reinterpret_cast<float*>(e) = acc[i];
-                    else if (p.out_dtype == 1) *reinterpret_cast<__nv_bfloat16*>(e) = __float2bfloat16_rn(acc[i]);
-                    else *reinterpret_cast<__half*>(e) = __float2half_rn(acc[i]);
+            for (int ck = 0; ck < BM / kYChunk; ++ck) {
+                if (ok) {
+#pragma unroll
+                    for (int i = 0; i < kYChunk; ++i) {
+                        unsigned char* ep = yt + (i * BN + row) * esz;
+                        const float v = acc[ck * kYChunk + i];
+                        if (p.out_dtype == 2) *reinterpret_cast<float*>(ep) = v;
+                        else if (p.out_dtype == 1) *reinterpret_cast<__nv_bfloat16*>(ep) = __float2bfloat16_rn(v);
+                        else *reinterpret_cast<__half*>(ep) = __float2half_rn(v);
+                    }
                 }
-            }
-            named_bar_sync(1, 128);
-            if (ok) {
-                const int cpr = BN * esz / 16;               // 16-byte pieces per token row
-                const int ncols = min(BN, p.N - n0);         // a multiple of 16 (N % 16 == 0)
-                for (int c = 32 * quad + lane; c < BM * cpr; c += 128) {
-                    const int m = c / cpr, pc = c - m * cpr;
-                    if (m0 + m >= p.M || pc * 16 >= ncols * esz) continue;
-                    const uint4 v = *reinterpret_cast<const uint4*>(yt + m * BN * esz + pc * 16);
-                    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(p.Y) +
-                                              ((size_t)(m0 + m) * p.N + n0) * esz + pc * 16) = v;
+                named_bar_sync(1, 256);
+                if (ok) {
+                    for (int cc = 32 * e + lane; cc < kYChunk * cpr; cc += 256) {
+                        const int m = cc / cpr, pc = cc - m * cpr;
+                        const int mm = m0 + ck * kYChunk + m;
+                        if (mm >= p.M || pc * 16 >= ncols * esz) continue;
+                        const uint4 v = *reinterpret_cast<const uint4*>(yt + m * BN * esz + pc * 16);
+                        *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(p.Y) +
+                                                  ((size_t)mm * p.N + n0) * esz + pc * 16) = v;
+                    }
                 }
+                named_bar_sync(1, 256);   // the buffer is free for the next block
             }
-            named_bar_sync(1, 128);   // the buffer is free for the next tile
         }
     }
 

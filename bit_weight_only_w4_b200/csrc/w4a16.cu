@@ -283,6 +283,15 @@ w4_status launch_prefill(const CUtensorMap& map, const w4p::PrefillParams& p, in
     static std::once_flag flags[kMaxDevices];
     auto k = w4p::prefill_kernel<BF16, GIDX>;
     if (!ensure_smem(k, w4p::SmemLayout::bytes, flags, dev)) return W4_ERR_CUDA;
+    // the kernel's per-warpgroup register split assumes this many registers a thread at
+    // launch; any other build would make its register increase wait forever
+    static int regs[kMaxDevices];
+    static std::once_flag rflags[kMaxDevices];
+    std::call_once(rflags[dev], [&] {
+        cudaFuncAttributes a;
+        regs[dev] = cudaFuncGetAttributes(&a, k) == cudaSuccess ? a.numRegs : -1;
+    });
+    if (regs[dev] != w4p::kLaunchRegs) return W4_ERR_UNSUPPORTED;
     // persistent: one CTA per SM (or per tile when there are fewer tiles)
     const long long ntiles = (long long)((p.N + w4p::BN - 1) / w4p::BN) * ((p.M + w4p::BM - 1) / w4p::BM);
     const int sms = sm_count(dev);
