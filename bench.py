@@ -344,28 +344,34 @@ def time_quantize(w4, torch, projs, iters=3):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def cpu_oracle_sample(target_s=12.0, rows_per_layer=None):
+def cpu_oracle_sample(target_s=12.0, rows_per_layer=256):
     """Time the oracle's online path (X*s_inv, dequantise, fp32 product) for M=1 on a
-    seeded sample of output rows of every decode layer; returns (GB/s of effective weight
-    bytes processed, seconds, description)."""
+    seeded sample of output rows of every decode layer, each layer's product repeated until
+    about target_s / 4 seconds of CPU work; returns (GB/s of effective weight bytes
+    processed, seconds, description)."""
     import oracle
     wl = workloads.workload(DECODE_CFG)
     rng = np.random.default_rng(0)
-    total_bytes, total_s, n_rows = 0, 0.0, 0
-    rows_per_layer = rows_per_layer or 256
+    total_bytes, total_s, n_rows, reps = 0, 0.0, 0, []
     for i, L in enumerate(wl.layers):
         li = workloads.make_layer(wl, i, M=1, with_weights=False)
         # a fresh seeded sample of rows (weights regenerated only for those rows)
         ns = np.sort(rng.choice(L.N, size=rows_per_layer, replace=False))
         Wr = workloads.gen_weights(L.N, L.K, 0, wl.config_id, i)[ns]
         q, sc, zr = oracle.quantize_weights(Wr.view(np.uint16), li.s, 128)
-        t0 = time.perf_counter()
-        oracle.reference_y(li.X, li.s_inv, q, sc, zr, 128)
-        total_s += time.perf_counter() - t0
-        total_bytes += workloads.effective_weight_bytes(rows_per_layer, L.K, 128, False, False)
+        layer_s, r = 0.0, 0
+        while r == 0 or layer_s < target_s / len(wl.layers):
+            t0 = time.perf_counter()
+            oracle.reference_y(li.X, li.s_inv, q, sc, zr, 128)
+            layer_s += time.perf_counter() - t0
+            r += 1
+        total_s += layer_s
+        total_bytes += r * workloads.effective_weight_bytes(rows_per_layer, L.K, 128, False, False)
         n_rows += rows_per_layer
-    desc = (f"M=1, {rows_per_layer} seeded output rows of each of the 4 layers "
-            f"({n_rows} rows, {total_bytes / 1e6:.1f} MB effective weights), single thread")
+        reps.append(r)
+    desc = (f"M=1, {rows_per_layer} seeded output rows of each of the 4 layers ({n_rows} rows), "
+            f"each layer's product repeated {reps} times ({total_bytes / 1e6:.0f} MB of effective "
+            f"weights in {total_s:.1f} s), single thread")
     return total_bytes / total_s / 1e9, total_s, desc
 
 
@@ -376,10 +382,12 @@ def reference_arm(args, world, rank):
     oracle.lib()
     vals = []
     desc = ""
+    # each step a bounded sample, so that the whole run takes about two minutes
+    per_step = max(0.5, min(12.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_oracle_sample(rows_per_layer=64)
+        cpu_oracle_sample(target_s=per_step)
     for _ in range(args.steps):
-        v, s, desc = cpu_oracle_sample(rows_per_layer=256)
+        v, s, desc = cpu_oracle_sample(target_s=per_step)
         vals.append(v)
     value = statistics.median(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
@@ -434,13 +442,13 @@ def our_arm(args, world, rank, local):
         v, sec, desc = cpu_oracle_sample()
         cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
                "seconds": round(sec, 2)}
-    # DRAM traffic per launch of the decode kernel: ncu measured 48.571 MB read + 0.009 MB
-    # written for the gate_up launch (47.88 MB algorithmic), a ratio of 1.014
-    # (profiles/decode_gate_up_4096x22016_m1.md); the average launch of the step is scaled
-    # by its algorithmic bytes.  Set to None whenever the decode kernel changes.
-    DECODE_TRAFFIC_RATIO = 1.014
+    # DRAM traffic per launch of the decode kernel, as a ratio to its algorithmic bytes from
+    # one ncu capture of the gate_up launch (profiles/decode_gate_up_4096x22016_m1.md); the
+    # average launch of the step is scaled by its algorithmic bytes.  None until the current
+    # kernel has been captured.
+    DECODE_TRAFFIC_RATIO = None
     launches_per_step = N_LAYERS * len(projs)
-    traffic = DECODE_TRAFFIC_RATIO * step_bytes / launches_per_step
+    traffic = (DECODE_TRAFFIC_RATIO * step_bytes / launches_per_step) if DECODE_TRAFFIC_RATIO else None
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,

@@ -41,7 +41,6 @@ namespace w4d {
 
 constexpr int kBandRows = 128;
 constexpr int kTilesPerBand = 8;
-constexpr int kMmaWarps = 8;
 
 // Group handling of the MMA warps.
 enum : int {
@@ -56,16 +55,23 @@ struct Cfg {
     static constexpr int tpw = NT <= 2 ? 2 : 1;          // row tiles per MMA warp
     static constexpr int aps = NT <= 2 ? 8 : 4;          // atoms (64-channel blocks) per stage
     static constexpr int xw = NT == 1 ? 1 : NT <= 4 ? 2 : 4;   // activation warps
-    static constexpr int mma_warps = NT <= 4 ? 16 : 8;   // two stage groups (one when 8)
+    static constexpr int mma_warps = NT <= 4 ? 16 : 8;
     static constexpr int groups = mma_warps / 8;         // stage-parity groups
+    static constexpr int stage_warps = mma_warps / groups;   // MMA warps sharing a stage
+    static constexpr int tsets = 8 / tpw;                // row-tile sets of a band
+    static constexpr int kparts = stage_warps / tsets;   // K slices of a stage
+    static constexpr int apk = aps / kparts;             // atoms per K slice
     static constexpr int warps = 1 + xw + mma_warps;
     static constexpr int threads = 32 * warps;
     static constexpr int mpad = 8 * NT;                  // token rows per activation box slot
     // activation sums of one stage: per token, over 32, 64 and 128 consecutive channels
     static constexpr int sx32 = 0, sx64 = 2 * aps, sx128 = 3 * aps;
     static constexpr int sx_floats = 4 * aps * mpad;
-    // partial-sum sets per row tile at a flush: stage groups x K halves
-    static constexpr int nset = groups * (tpw == 2 ? 2 : 1);
+    // partial-sum sets per row tile at a flush: stage groups x K slices
+    static constexpr int nset = groups * kparts;
+    // the producer warp sums the contributors' shares of a completed band ahead of the
+    // flush (into [M][128] fp32 of shared memory) when that buffer is small
+    static constexpr bool pgather = NT <= 2;
     // MMA-warp exchange buffer: [nset-1][8 tiles][NT][4][32 lanes] fp32
     static constexpr int xchg_bytes = (nset - 1) * 8 * NT * 4 * 32 * 4;
 };
@@ -93,6 +99,7 @@ struct DecodeParams {
     int off_res_s;            // byte offset of the resident sums: [K/32 | K/64 | K/128][sstride]
     int sstride;              // tokens per row of the activation sums
     int off_xchg;             // byte offset of the MMA-warp exchange buffer
+    int off_gsum;             // byte offset of the contributors' sums of the completed band: [M][128] fp32
     // byte offsets inside one stage
     int off_x, off_xs, off_sx, off_si, off_sc, off_zr, off_gi, off_desc, stage_bytes;
 };
@@ -108,20 +115,23 @@ W4_DEV int band_tiles(const DecodeParams& p, int band) {
 
 // The parts of a CTA's unit range [u0,u1), one per band it touches, in processing order:
 // when the range ends inside a band, that (contributor) part comes first, so its partial
-// sums are published early; every other part either is a whole band or holds the band's
-// last unit and completes it.
+// sums are published early; the whole bands follow, and the first band of the range comes
+// last: when the range starts inside it, that part completes the band and has to wait for
+// the contributors' sums, which by then (each contributor publishes in its first part)
+// are normally out.
 struct PartIter {
     int b0, b1;
-    bool contrib_first;
+    int lead;   // 1 when the last band is a contributor part (processed first)
     W4_DEV PartIter(const DecodeParams& p, int u0, int u1) {
         b0 = u0 / p.KU;
         b1 = (u1 - 1) / p.KU;
-        contrib_first = u1 < (b1 + 1) * p.KU;
+        lead = (b1 > b0 && u1 < (b1 + 1) * p.KU) ? 1 : 0;
     }
     W4_DEV int count() const { return b1 - b0 + 1; }
     W4_DEV int band(int pi) const {
-        if (contrib_first) return pi == 0 ? b1 : b0 + pi - 1;
-        return b0 + pi;
+        if (pi == b1 - b0) return b0;
+        if (lead && pi == 0) return b1;
+        return b0 + 1 + pi - lead;
     }
 };
 
@@ -395,6 +405,16 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
             for (int aa = 0; aa < 2; ++aa)
 #pragma unroll
                 for (int tt = 0; tt < TPW; ++tt) w[aa][tt] = ld_u128(wp[2 * pr + aa] + tt * 512);
+            // scale and zero-point bits of rows r0 and r1 of each tile
+            uint32_t md[TPW][4];
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt) {
+                const int o = grow * 256 + tt * 32;
+                md[tt][0] = ld_u16(scp + o);
+                md[tt][1] = ld_u16(scp + o + 16);
+                md[tt][2] = v.zr ? ld_u16(zrp + o) : 0x4800u;   // symmetric: z = 8
+                md[tt][3] = v.zr ? ld_u16(zrp + o + 16) : 0x4800u;
+            }
             float c[TPW][NT][4], c2[TPW][NT][4];
 #pragma unroll
             for (int aa = 0; aa < 2; ++aa)
@@ -433,12 +453,8 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
             for (int nt = 0; nt < NT; ++nt) S[nt] = ld_f2(sxp + (pr * v.sstride + 8 * nt) * 4);
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt) {
-                const int o = grow * 256 + tt * 32;
-                const uint32_t sc0 = ld_u16(scp + o), sc1 = ld_u16(scp + o + 16);
-                const uint32_t z0 = v.zr ? ld_u16(zrp + o) : 0x4800u;   // symmetric: z = 8
-                const uint32_t z1 = v.zr ? ld_u16(zrp + o + 16) : 0x4800u;
-                const RowFold f0 = row_fold<BF16, false>(sc0, z0);
-                const RowFold f1 = row_fold<BF16, true>(sc1, z1);
+                const RowFold f0 = row_fold<BF16, false>(md[tt][0], md[tt][2]);
+                const RowFold f1 = row_fold<BF16, true>(md[tt][1], md[tt][3]);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     acc[tt][nt][0] = fmaf(f0.scp, fmaf(f0.bz, S[nt].x, c[tt][nt][0]), acc[tt][nt][0]);
@@ -666,13 +682,106 @@ W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* x
 // ---------------------------------------------------------------- end of a part
 // Combine, then store, publish or complete the band's sums.  Slot entry of (tile t, token
 // tile nt, element e, lane) is ((t * NT + nt) * 4 + e) * 32 + lane.
+
+// Slot index of entry x of a band's shares, entries ordered by (channel in the band, token).
+template <int NT>
+W4_DEV int share_slot(int x, int M) {
+    const int m = x % M, nl = x / M;
+    const int r = nl & 15;
+    return (((nl >> 4) * NT + (m >> 3)) * 4 + 2 * (r >> 3) + (m & 1)) * 32 + 4 * (r & 7) + ((m & 7) >> 1);
+}
+
+// Producer warp, once its copies are out: sum the shares that CTAs [c_first, cta) published
+// for `band` (CTA order per entry) into gsum[m][n - band start], for the MMA warps'
+// completing flush.  Entries are spread over the lanes four at a time, and the loads of two
+// contributors of those entries go out together.  False on a timed-out wait.
+template <int NT>
+W4_DEV bool gather_shares(const DecodeParams& p, float* gsum, int band, int cta, int lane) {
+    constexpr int kSlot = kTilesPerBand * NT * 4 * 32;
+    const int n_ent = band_tiles(p, band) * 16 * p.M;
+    const int c_first = cta_of_unit(p, band * p.KU);
+    for (int x0 = 0; x0 < n_ent; x0 += 128) {
+        int j[4];
+        float tot[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int x = x0 + 32 * k + lane;
+            j[k] = x < n_ent ? share_slot<NT>(x, p.M) : -1;
+            tot[k] = 0.0f;
+        }
+        for (int c0 = c_first; c0 < cta; c0 += 2) {
+            unsigned long long v[4][2];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+                    v[k][b] = j[k] >= 0 && c0 + b < cta ? slot_get(p.slots + (size_t)(c0 + b) * kSlot + j[k]) : 0ull;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    if (j[k] < 0 || c0 + b >= cta) continue;
+                    unsigned long long* a = p.slots + (size_t)(c0 + b) * kSlot + j[k];
+                    float val = __uint_as_float((uint32_t)v[k][b]);
+                    if ((v[k][b] >> 32) == 0 && !slot_wait(a, val)) return false;
+                    tot[k] += val;
+                    slot_clear(a);
+                }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int x = x0 + 32 * k + lane;
+            if (x < n_ent) gsum[(x % p.M) * kBandRows + x / p.M] = tot[k];
+        }
+    }
+    return true;
+}
+
+// MMA thread mt of nthr: for each entry x = mt, mt + nthr, ... of the band, xc[slot] = the
+// sum of the shares CTAs [c_first, cta) published, in CTA order; the loads of up to eight
+// contributors of an entry go out together.  False on a timed-out wait.
+template <int NT>
+W4_DEV bool sum_shares(const DecodeParams& p, float* xc, int band, int c_first, int cta, int mt, int nthr) {
+    constexpr int kSlot = kTilesPerBand * NT * 4 * 32;
+    const int n_ent = band_tiles(p, band) * 16 * p.M;
+    for (int x = mt; x < n_ent; x += nthr) {
+        const int j = share_slot<NT>(x, p.M);
+        float tot = 0.0f;
+        for (int c0 = c_first; c0 < cta; c0 += 8) {
+            unsigned long long v[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+                v[b] = c0 + b < cta ? slot_get(p.slots + (size_t)(c0 + b) * kSlot + j) : 0ull;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                if (c0 + b >= cta) break;
+                unsigned long long* a = p.slots + (size_t)(c0 + b) * kSlot + j;
+                float val = __uint_as_float((uint32_t)v[b]);
+                if ((v[b] >> 32) == 0 && !slot_wait(a, val)) return false;
+                tot += val;
+                slot_clear(a);
+            }
+        }
+        xc[j] = tot;
+    }
+    return true;
+}
+
+// Who adds the contributors' shares when a part completes a band with `ncon` contributors:
+// the producer warp ahead of time (few contributors, small buffer) or all MMA warps
+// together after the last stage.
+constexpr int kFewShares = 2;
+template <int NT>
+W4_DEV bool producer_sums(int ncon) {
+    return Cfg<NT>::pgather && ncon <= kFewShares;
+}
+
+// Combine the partial sums of a row tile's sets (stage groups x K slices) in shared memory:
+// set 0 adds the others in a fixed order.  Every MMA warp takes part (named barriers).
 template <int NT, int TPW>
-W4_DEV void flush_part(const DecodeParams& p, unsigned char* xchg, int band, int ps, int pe, int cta,
-                       int set, int t0, const Lane& L, bool aborted, float (&acc)[TPW][NT][4]) {
+W4_DEV void combine_sets(unsigned char* xchg, int set, int t0, const Lane& L, float (&acc)[TPW][NT][4]) {
     using C = Cfg<NT>;
     if constexpr (C::nset > 1) {
-        // the partial sums of a row tile (stage groups x K halves) meet in shared memory;
-        // set 0 adds the others in a fixed order
         float* xc = reinterpret_cast<float*>(xchg);
         constexpr int kSet = 8 * NT * 4 * 32;
         if (set > 0) {
@@ -697,14 +806,34 @@ W4_DEV void flush_part(const DecodeParams& p, unsigned char* xchg, int band, int
                             acc[tt][nt][e] += xc[(k - 1) * kSet + (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane];
         }
         named_bar_sync(2, 32 * C::mma_warps);
-        if (set > 0) return;
     }
-    if (aborted) return;
+}
+
+template <int NT, int TPW>
+W4_DEV void store_rows(const DecodeParams& p, int band, int t0, const Lane& L, const float (&acc)[TPW][NT][4]) {
     const int tb = band_tiles(p, band);
-    const int bu0 = band * p.KU, bu1 = bu0 + p.KU;
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+        if (t0 + tt >= tb) continue;
+        const int n0 = band * kBandRows + 16 * (t0 + tt) + L.g8;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int m = 8 * nt + 2 * L.q + (e & 1);
+                if (m < p.M) store_out(p, m, n0 + ((e >> 1) << 3), acc[tt][nt][e]);
+            }
+    }
+}
+
+// A part that does not complete its band (set-0 threads, after combine_sets): a whole band
+// is stored; a contributor part publishes this CTA's share into its slots.
+template <int NT, int TPW>
+W4_DEV void flush_part(const DecodeParams& p, int band, int pe, int cta, int t0, const Lane& L,
+                       const float (&acc)[TPW][NT][4]) {
     constexpr int kSlot = kTilesPerBand * NT * 4 * 32;
-    if (pe < bu1) {
-        // contributor: publish this CTA's share of the band
+    const int tb = band_tiles(p, band);
+    if (pe < (band + 1) * p.KU) {
         unsigned long long* base = p.slots + (size_t)cta * kSlot;
 #pragma unroll
         for (int tt = 0; tt < TPW; ++tt) {
@@ -718,68 +847,59 @@ W4_DEV void flush_part(const DecodeParams& p, unsigned char* xchg, int band, int
         }
         return;
     }
-    if (ps > bu0) {
-        // the band's last unit: add the contributors' shares (CTA order) before this one's
-        float tot[TPW][NT][4];
-#pragma unroll
-        for (int tt = 0; tt < TPW; ++tt)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) tot[tt][nt][e] = 0.0f;
-        const int c_first = cta_of_unit(p, bu0);
-        bool ok = true;
-        for (int c = c_first; c < cta && ok; ++c) {
-            unsigned long long* base = p.slots + (size_t)c * kSlot;
-            unsigned long long w[TPW][NT][4];
+    store_rows<NT, TPW>(p, band, t0, L, acc);
+}
+
+// The CTA's last part holds the band's last unit and started inside the band: add the
+// contributors' shares (CTA order) before this CTA's own, then store.  Runs after the part
+// loop, on every MMA warp (named barriers on the shared path).
+template <int NT, int TPW>
+W4_DEV void complete_band(const DecodeParams& p, unsigned char* smem, unsigned char* xchg, volatile int* s_abort,
+                          const float* gsum, uint64_t* gready, int band, int cta, int set, int t0, const Lane& L,
+                          bool aborted, float (&acc)[TPW][NT][4]) {
+    using C = Cfg<NT>;
+    const int tb = band_tiles(p, band);
+    const int c_first = cta_of_unit(p, band * p.KU);
+    if (!producer_sums<NT>(cta - c_first)) {
+        // the MMA threads share the band's entries, summing the contributors' shares into a
+        // slot-layout buffer (the exchange buffer, or with a single set the first ring stage,
+        // idle once every MMA warp is past the last stage); set 0 adds them
+        float* xc = reinterpret_cast<float*>(C::nset > 1 ? xchg : smem);
+        if constexpr (C::nset == 1) named_bar_sync(1, 32 * C::mma_warps);
+        const int mt = threadIdx.x - 32 * (1 + C::xw);
+        if (!aborted && !sum_shares<NT>(p, xc, band, c_first, cta, mt, 32 * C::mma_warps)) *s_abort = 1;
+        named_bar_sync(1, 32 * C::mma_warps);
+        if (set == 0) {
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const bool valid = t0 + tt < tb && 8 * nt + 2 * L.q + (e & 1) < p.M;
-                        w[tt][nt][e] = valid ? slot_get(base + (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane)
-                                             : (1ull << 32);
-                    }
-#pragma unroll
-            for (int tt = 0; tt < TPW; ++tt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const bool valid = t0 + tt < tb && 8 * nt + 2 * L.q + (e & 1) < p.M;
-                        if (!valid || !ok) continue;
-                        unsigned long long* a = base + (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane;
-                        float v = __uint_as_float((uint32_t)w[tt][nt][e]);
-                        if ((w[tt][nt][e] >> 32) == 0 && !slot_wait(a, v)) {
-                            ok = false;
-                            continue;
-                        }
-                        tot[tt][nt][e] += v;
-                        slot_clear(a);
+                        const int j = (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane;
+                        if (t0 + tt < tb && 8 * nt + 2 * L.q + (e & 1) < p.M) acc[tt][nt][e] = xc[j] + acc[tt][nt][e];
                     }
         }
-        if (!ok) return;
+        named_bar_sync(2, 32 * C::mma_warps);
+    } else {
+        if (set > 0 || aborted) return;
+        // the producer warp has summed the contributors' shares into gsum
+        if (!mbar_wait(gready, 0)) *s_abort = 1;
+        if (!*s_abort) {
 #pragma unroll
-        for (int tt = 0; tt < TPW; ++tt)
+            for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc[tt][nt][e] = tot[tt][nt][e] + acc[tt][nt][e];
+                    for (int e = 0; e < 4; ++e) {
+                        const int m = 8 * nt + 2 * L.q + (e & 1);
+                        const int nl = 16 * (t0 + tt) + L.g8 + 8 * (e >> 1);
+                        if (m < p.M && t0 + tt < tb) acc[tt][nt][e] = gsum[m * kBandRows + nl] + acc[tt][nt][e];
+                    }
+        }
     }
-#pragma unroll
-    for (int tt = 0; tt < TPW; ++tt) {
-        if (t0 + tt >= tb) continue;
-        const int n0 = band * kBandRows + 16 * (t0 + tt) + L.g8;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int m = 8 * nt + 2 * L.q + (e & 1);
-                if (m < p.M) store_out(p, m, n0 + ((e >> 1) << 3), acc[tt][nt][e]);
-            }
-    }
+    if (set > 0 || aborted || *s_abort) return;
+    store_rows<NT, TPW>(p, band, t0, L, acc);
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -820,6 +940,8 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
     uint64_t* xready = full + kMaxStages;
     uint64_t* empty = xready + kMaxStages;
     volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
+    uint64_t* gready = empty + kMaxStages + 1;   // contributors' sums in gsum
+    float* gsum = reinterpret_cast<float*>(smem + p.off_gsum);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
@@ -830,8 +952,9 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&xready[s], 32 * C::xw);
-            mbar_init(&empty[s], kMmaWarps);
+            mbar_init(&empty[s], C::stage_warps);
         }
+        mbar_init(gready, 1);
         *s_abort = 0;
         fence_mbar_init();
     }
@@ -895,14 +1018,21 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                 const int g_first = GIDX ? 0 : (64 * a0) / g;
                 if (lane == 0) {
                     // stage descriptor for the consumers: {a0, na, tiles, first group row}
-                    // and, for each half, the offset of its first atom in its group and
+                    // and, for each K slice, the offset of its first atom in its group and
                     // its staged group row
-                    const int r0 = 64 * a0 - g_first * g;
-                    const int k1 = r0 + 64 * (C::aps / 2);
-                    const int g1 = GIDX ? 0 : k1 / g;
+                    int kg[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                    if (!GIDX) {
+#pragma unroll
+                        for (int k = 0; k < C::kparts; ++k) {
+                            const int off = 64 * a0 - g_first * g + 64 * C::apk * k;
+                            kg[2 * k + 1] = off / g;
+                            kg[2 * k] = off - kg[2 * k + 1] * g;
+                        }
+                    }
                     int4* desc = reinterpret_cast<int4*>(st + p.off_desc);
                     desc[0] = make_int4(a0, na, tb, g_first);
-                    desc[1] = make_int4(r0, 0, k1 - g1 * g, g1);
+                    desc[1] = make_int4(kg[0], kg[1], kg[2], kg[3]);
+                    desc[2] = make_int4(kg[4], kg[5], kg[6], kg[7]);
                     uint32_t bytes = na * tb * 512;
                     if (!p.xres) bytes += C::aps * p.M * 128 + (p.s_inv ? na * 256 : 0);
                     if (GIDX) bytes += na * 256;
@@ -949,6 +1079,18 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                 if (k >= i - S) (void)mbar_wait(&full[q.s], q.ph);
         }
         __syncwarp();
+        if constexpr (C::pgather) {
+            // the last part completes band b0 when the range starts inside it: sum the
+            // earlier CTAs' shares while the MMA warps work through the last stages
+            const int bu0 = it.b0 * p.KU;
+            if (u0 > bu0 && u1 >= bu0 + p.KU && producer_sums<NT>(cta - cta_of_unit(p, bu0))) {
+                pdl_wait();   // the shares are this grid's, the slots cleared by the preceding one
+                const bool ok = !abort && gather_shares<NT>(p, gsum, it.b0, cta, lane);
+                if (!ok) *s_abort = 1;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(gready);
+            }
+        }
     } else {
     if (p.xres) {
         // ------------------------------------------------------------ resident X'
@@ -982,10 +1124,10 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
         pdl_wait();   // before any store to Y or the workspace
         constexpr int TPW = C::tpw;
         const int cw = warp - 1 - C::xw;
-        const int grp = cw >> 3, w8 = cw & 7;          // stage group, warp within it
-        const int h = TPW == 2 ? (w8 >> 2) : 0;        // K half (two tiles per warp)
-        const int t0 = TPW == 2 ? 2 * (w8 & 3) : w8;
-        const int set = grp * (TPW == 2 ? 2 : 1) + h;  // partial-sum set at a flush
+        const int grp = cw / C::stage_warps, ws = cw % C::stage_warps;   // stage group, warp in it
+        const int kp = ws / C::tsets;                  // K slice of the stage
+        const int t0 = TPW * (ws % C::tsets);          // first row tile
+        const int set = grp * C::kparts + kp;          // partial-sum set at a flush
         const int xrows = NT == 1 ? p.M : C::mpad;
         const int sstride = p.xres ? p.sstride : C::mpad;
         const Lane L = make_lane(lane, xrows, sstride, p.xres ? p.K / 64 * 128 : C::aps * 128);
@@ -1006,10 +1148,10 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                 }
                 unsigned char* st = smem + r.s * p.stage_bytes;
                 const int4 d0 = *reinterpret_cast<const int4*>(st + p.off_desc);
-                const int4 d1 = *reinterpret_cast<const int4*>(st + p.off_desc + 16);
+                const int2 kg = *reinterpret_cast<const int2*>(st + p.off_desc + 16 + 8 * kp);
                 const int a0 = d0.x, na = d0.y;
-                const int ab = TPW == 2 ? h * (C::aps / 2) : 0;
-                const int ae = TPW == 2 ? min(na, ab + C::aps / 2) : na;
+                const int ab = kp * C::apk;
+                const int ae = min(na, ab + C::apk);
                 if (!aborted && t0 < tb && ab < ae) {
                     StageView v;
                     v.codes = st;
@@ -1031,17 +1173,22 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                     v.tb = tb;
                     v.a0 = a0;
                     v.gfirst = d0.w;
-                    v.kin = ab == 0 ? d1.x : d1.z;
-                    v.grow = ab == 0 ? d1.y : d1.w;
+                    v.kin = kg.x;
+                    v.grow = kg.y;
                     if constexpr (GIDX) consume_gidx<NT, TPW>(v, p, L, band, t0, ab, ae, st + p.off_gi, acc);
                     else consume<NT, TPW, BF16, MODE>(v, L, t0, ab, ae, g, acc);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[r.s]);
             }
-            flush_part<NT, TPW>(p, xchg, band, ps, pe, cta, set, t0, L, aborted, acc);
+            combine_sets<NT, TPW>(xchg, set, t0, L, acc);
+            // the part that completes its band is the last one: finished after the loop
+            if (pe == (band + 1) * p.KU && ps > band * p.KU) continue;
+            if (set == 0 && !aborted) flush_part<NT, TPW>(p, band, pe, cta, t0, L, acc);
             zero_acc<NT, TPW>(acc);
         }
+        if (u0 > it.b0 * p.KU && u1 >= (it.b0 + 1) * p.KU)
+            complete_band<NT, TPW>(p, smem, xchg, s_abort, gsum, gready, it.b0, cta, set, t0, L, aborted, acc);
     }
     }
 }
