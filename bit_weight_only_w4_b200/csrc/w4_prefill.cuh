@@ -35,11 +35,12 @@ constexpr int kThreads = 512;  // producer, MMA, 6 dequant, 8 epilogue warps (4 
 constexpr int kDequantWarps = 6;
 // Register split: launched with 128 registers a thread (512 x 128 = the SM's 65536);
 // warpgroups 0-1 (producer, MMA, dequant) give theirs down to kRegsLow, warpgroups 2-3
-// (epilogue: 128 fp32 accumulators a thread) take kRegsHigh.  2 x 128 x 88 + 2 x 128 x
-// 168 = 65536, exactly the launch's registers.
+// (epilogue: 128 fp32 accumulators plus a 32-column tensor-memory load a thread) take
+// kRegsHigh.  2 x 128 x 80 + 2 x 128 x 176 = 65536, exactly the launch's registers; with
+// 168 for the epilogue its per-group loop spilled to local memory.
 constexpr int kLaunchRegs = 128;
-constexpr int kRegsLow = 88;
-constexpr int kRegsHigh = 168;
+constexpr int kRegsLow = 80;
+constexpr int kRegsHigh = 176;
 static_assert(2 * 128 * kRegsLow + 2 * 128 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
 constexpr int kTmemCols = 512; // two fp32 partial buffers x two halves x BM columns
 constexpr int kYChunk = 32;    // tokens per pass of the output staging buffer
