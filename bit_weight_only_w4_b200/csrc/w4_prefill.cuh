@@ -9,12 +9,13 @@
 //
 // One CTA computes a 128 (output rows) x 128 (tokens) tile of Y^T = What * X'^T:
 //   warp 0      TMA: activation tile (2-D tensor map, 128B swizzle) + packed weight tiles
-//               (1-D bulk copies) into a 4-stage ring;
+//               (1-D bulk copies) + zero-point rows into a 5-slot load ring;
 //   warp 1      allocates tensor memory and issues tcgen05.mma (one thread): A = the
 //               dequantised weights (128 x 64 per stage, K-major, 128B swizzle, shared
 //               memory), B = the activations, D = fp32 in tensor memory;
 //   warps 2-5   unpack the packed tile into exact integers q - z (fp16/bf16) in the
-//               swizzled A layout;
+//               swizzled A layout, into a 2-slot ring of its own (the load ring runs
+//               further ahead than the dequantised tiles need to);
 //   warps 6-9   epilogue: after each quantisation group the MMA warp hands over that
 //               group's fp32 partial tile (two tensor-memory buffers, ping-pong); each
 //               thread owns one output row, multiplies the partial by the row's group
@@ -30,7 +31,8 @@ constexpr int BN = 256;        // output rows per CTA: two 128-row halves (MMA M
 constexpr int BH = 128;        // rows per half
 constexpr int BM = 128;        // tokens per CTA (MMA N)
 constexpr int BK = 64;         // input channels per stage (one 128-byte swizzle row)
-constexpr int kStages = 3;
+constexpr int kLoadStages = 5;  // activations, codes, zero points: the copies run this far ahead
+constexpr int kDeqStages = 2;   // dequantised weight tiles (double-buffered)
 constexpr int kThreads = 512;  // producer, MMA, 6 dequant, 8 epilogue warps (4 warpgroups)
 constexpr int kDequantWarps = 6;
 // Register split: launched with 128 registers a thread (512 x 128 = the SM's 65536);
@@ -53,13 +55,13 @@ constexpr int kZBytes = 2 * BN * 2;    // zero-point rows of up to two groups
 constexpr int kStageBytes = kABytes + kBBytes + kPBytes + kZBytes;
 
 struct SmemLayout {
-    static constexpr int a = 0;                              // kStages x 32 KB (1024-aligned)
-    static constexpr int b = a + kStages * kABytes;          // kStages x 16 KB
-    static constexpr int pk = b + kStages * kBBytes;         // kStages x 8 KB
-    static constexpr int zr = pk + kStages * kPBytes;        // kStages x 1 KB
-    static constexpr int y = zr + kStages * kZBytes;         // output staging: kYChunk x BN fp32
+    static constexpr int a = 0;                              // kDeqStages x 32 KB (1024-aligned)
+    static constexpr int b = a + kDeqStages * kABytes;       // kLoadStages x 16 KB
+    static constexpr int pk = b + kLoadStages * kBBytes;     // kLoadStages x 8 KB
+    static constexpr int zr = pk + kLoadStages * kPBytes;    // kLoadStages x 1 KB
+    static constexpr int y = zr + kLoadStages * kZBytes;     // output staging: kYChunk x BN fp32
     static constexpr int bars = y + kYChunk * BN * 4;        // barriers
-    static constexpr int nbars = 3 * kStages + 4 + 1;
+    static constexpr int nbars = 2 * kLoadStages + 2 * kDeqStages + 4 + 1;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int flags = tmem_slot + 8;
     static constexpr int bytes = flags + 16 + 1024;          // + alignment slack
@@ -201,9 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char* smem = align_smem_1024(smem_raw);
     using L = SmemLayout;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::bars);
-    uint64_t* deq = full + kStages;
-    uint64_t* empty = deq + kStages;
-    uint64_t* pfull = empty + kStages;       // [2]
+    uint64_t* empty = full + kLoadStages;    // load slot free (its stage's MMAs are done)
+    uint64_t* deq = empty + kLoadStages;     // dequantised tile written
+    uint64_t* wempty = deq + kDeqStages;     // dequantised tile consumed by the MMAs
+    uint64_t* pfull = wempty + kDeqStages;   // [2]
     uint64_t* pempty = pfull + 2;            // [2]
     uint64_t* mma_done = pempty + 2;         // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::tmem_slot);
@@ -220,10 +223,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ntiles = nbands * ((p.M + BM - 1) / BM);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kLoadStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&deq[s], 32 * kDequantWarps);
             mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < kDeqStages; ++s) {
+            mbar_init(&deq[s], 32 * kDequantWarps);
+            mbar_init(&wempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&pfull[b], 1);
@@ -263,8 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int zgroups = (!GIDX && p.zeros) ? (g == 32 ? 2 : 1) : 0;
                 const uint32_t bytes = kBBytes + (th[0] + th[1]) * (512 + zgroups * 32);
                 for (int kt = 0; kt < KT; ++kt, ++gst) {
-                    const int s = gst % kStages, ph = (gst / kStages) & 1;
-                    if (gst >= kStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
+                    const int s = gst % kLoadStages, ph = (gst / kLoadStages) & 1;
+                    if (gst >= kLoadStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
                     mbar_arrive_expect_tx(&full[s], bytes);
                     for (int h = 0; h < 2; ++h) {
                         if (th[h] == 0) continue;
@@ -285,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (*abort_flag)
-                for (int i = (gst > kStages ? gst - kStages : 0); i < gst; ++i)
-                    (void)mbar_wait(&full[i % kStages], (i / kStages) & 1);
+                for (int i = (gst > kLoadStages ? gst - kLoadStages : 0); i < gst; ++i)
+                    (void)mbar_wait(&full[i % kLoadStages], (i / kLoadStages) & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -296,8 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // both against the same activation tile.
         const bool leader = elect_one();
         const uint32_t idesc = mma_idesc(BF16 && !GIDX);
-        // descriptors of ring slot 0; slot s, half h and 16-channel step j are
-        // s * kABytes + h * kAHalf + 32 j bytes further (>> 4 in the descriptors)
+        // descriptors of slot 0 of each ring; slot s, half h and 16-channel step j are
+        // s * (tile bytes) + h * kAHalf + 32 j bytes further (>> 4 in the descriptors)
         const uint64_t a_desc0 = sw128_desc(smem_u32(smem + L::a));
         const uint64_t b_desc0 = sw128_desc(smem_u32(smem + L::b));
         // group boundaries: every spg stages (g a multiple of 64), twice per stage
@@ -310,17 +316,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             int sig = 0;   // stage index inside the current group
             for (int kt = 0; kt < KT; ++kt, ++gst) {
-                const int s = gst % kStages;
-                const uint32_t ph = (uint32_t)((gst / kStages) & 1);
-                // the dequant warps arrive on deq[s] only after full[s] completed (its
-                // activation tile landed), so deq[s] alone orders the MMA after both
-                ok = wait_or_abort(&deq[s], ph, abort_flag);
+                const int s = gst % kLoadStages, ds = gst % kDeqStages;
+                const uint32_t ph = (uint32_t)((gst / kDeqStages) & 1);
+                // the dequant warps arrive on deq[ds] only after full[s] completed (the
+                // activation tile landed), so deq[ds] alone orders the MMA after both
+                ok = wait_or_abort(&deq[ds], ph, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t ad = a_desc0 + (uint64_t)(s * (kABytes >> 4));
+                const uint64_t ad = a_desc0 + (uint64_t)(ds * (kABytes >> 4));
                 const uint64_t bd = b_desc0 + (uint64_t)(s * (kBBytes >> 4));
 #pragma unroll
                 for (int hk = 0; hk < 2; ++hk) {
@@ -348,7 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (ends && leader) tc_commit(&pfull[grp_i & 1]);
                 }
                 if (!ok) break;
-                if (leader) tc_commit(&empty[s]);
+                if (leader) {
+                    tc_commit(&empty[s]);      // the load slot (activations) is free
+                    tc_commit(&wempty[ds]);    // and so is the dequantised tile
+                }
                 if (++sig == spg) sig = 0;
             }
         }
@@ -370,8 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n0 = (t % nbands) * BN;
             const int tt_end = max(0, min(BN / 16, p.tiles - n0 / 16));   // tiles of the tile
             for (int kt = 0; kt < KT; ++kt, ++gst) {
-                const int s = gst % kStages, ph = (gst / kStages) & 1;
-                if (!wait_or_abort(&full[s], ph, abort_flag)) {
+                const int s = gst % kLoadStages, ph = (gst / kLoadStages) & 1;
+                const int ds = gst % kDeqStages, dph = (gst / kDeqStages) & 1;
+                // the stage's copies have landed and the MMAs are done with the tile slot
+                if (!wait_or_abort(&full[s], ph, abort_flag) ||
+                    (gst >= kDeqStages && !wait_or_abort(&wempty[ds], dph ^ 1, abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -379,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int ti = dq; ti < BN / 16; ti += kDequantWarps) {
                     if (ti >= tt_end) break;
                     const int hh = ti >> 3, tt = ti & 7;          // half, tile within the half
-                    const uint32_t a_u32 = smem_u32(smem + L::a + s * kABytes + hh * kAHalf);
+                    const uint32_t a_u32 = smem_u32(smem + L::a + ds * kABytes + hh * kAHalf);
                     const unsigned char* pk = smem + L::pk + s * kPBytes + hh * (kPBytes / 2);
                     const unsigned char* zs = smem + L::zr + s * kZBytes + hh * BH * 2;
                     const uint4 wq = *reinterpret_cast<const uint4*>(pk + tt * 512 + lane * 16);
@@ -435,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(&deq[s]);
+                mbar_arrive(&deq[ds]);
             }
         }
     }
