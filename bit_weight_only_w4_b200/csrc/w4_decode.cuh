@@ -53,7 +53,7 @@ enum : int {
 template <int NT>
 struct Cfg {
     static constexpr int tpw = NT <= 2 ? 2 : 1;          // row tiles per MMA warp
-    static constexpr int aps = NT <= 2 ? 8 : 4;          // atoms (64-channel blocks) per stage
+    static constexpr int aps = NT == 1 ? 8 : 4;          // atoms (64-channel blocks) per stage
     static constexpr int xw = NT == 1 ? 1 : NT <= 4 ? 2 : 4;   // activation warps
     static constexpr int mma_warps = NT <= 4 ? 16 : 8;
     static constexpr int groups = mma_warps / 8;         // stage-parity groups
@@ -629,7 +629,8 @@ W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw,
 // its sums over every 32, 64 and 128 channels, prepared once per CTA by the warps
 // [w0, w0 + nw) straight from global memory.  X' keeps the per-stage layout, M rows per
 // 64-channel block; sums are [segment][sstride].  Consecutive lanes take consecutive
-// 8-channel chunks, so the sums are warp shuffles.
+// 8-channel chunks, so the sums are warp shuffles; a lane takes its chunk for every token
+// (M <= 8 here), loading the chunk's s_inv once and all M activation chunks together.
 template <bool BF16>
 W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* xr, float* sr, int w,
                           int nw, int lane) {
@@ -639,43 +640,54 @@ W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* x
     float* s64 = s32 + (p.K / 32) * ss;
     float* s128 = s64 + (p.K / 64) * ss;
     const uint4* x4 = reinterpret_cast<const uint4*>(X);
-    for (int base = 32 * w; base < p.M * cpt; base += 32 * nw) {
-        const int item = base + lane;
-        const bool valid = item < p.M * cpt;
-        const int m = valid ? item / cpt : 0;
-        const int c = valid ? item - m * cpt : 0;
-        float s = 0.0f;
-        if (valid) {
-            uint4 v = x4[(size_t)m * cpt + c];
-            uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-            if (p.s_inv) {
-                const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c);
-                const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c + 1);
-                const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    for (int base = 32 * w; base < cpt; base += 32 * nw) {
+        const int c = base + lane;
+        const bool valid = c < cpt;
+        float sv[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = unpack2<BF16>(wv[i]);
-                    wv[i] = pack2<BF16>(__fmul_rn(f.x, sv[2 * i]), __fmul_rn(f.y, sv[2 * i + 1]));
-                }
-            }
-            const int blk = c >> 3, ch = c & 7;
-            *reinterpret_cast<uint4*>(xr + m * (p.K / 64 * 128) + blk * 128 + ((ch ^ (m & 7)) << 4)) =
-                make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            float2 f[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) f[i] = unpack2<BF16>(wv[i]);
-            s = ((f[0].x + f[0].y) + (f[1].x + f[1].y)) + ((f[2].x + f[2].y) + (f[3].x + f[3].y));
+        for (int i = 0; i < 8; ++i) sv[i] = 1.0f;
+        if (p.s_inv && valid) {
+            const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c);
+            const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c + 1);
+            sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+            sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
         }
-        // groups of 4 / 8 / 16 consecutive chunks never straddle two tokens when K is a
-        // multiple of 32 / 64 / 128 channels (K is a multiple of 64; the 128-channel sums
-        // are only read when K is a multiple of 128)
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        if (valid && (lane & 3) == 0) s32[(c >> 2) * ss + m] = s;
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
-        if (valid && (lane & 7) == 0) s64[(c >> 3) * ss + m] = s;
-        s += __shfl_xor_sync(0xffffffffu, s, 8);
-        if (valid && (lane & 15) == 0 && (c >> 4) < p.K / 128) s128[(c >> 4) * ss + m] = s;
+        uint4 v[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+            v[m] = (valid && m < p.M) ? x4[(size_t)m * cpt + c] : make_uint4(0u, 0u, 0u, 0u);
+        const int blk = c >> 3, ch = c & 7;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            if (m >= p.M) break;
+            float s = 0.0f;
+            if (valid) {
+                uint32_t wv[4] = {v[m].x, v[m].y, v[m].z, v[m].w};
+                if (p.s_inv) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 f = unpack2<BF16>(wv[i]);
+                        wv[i] = pack2<BF16>(__fmul_rn(f.x, sv[2 * i]), __fmul_rn(f.y, sv[2 * i + 1]));
+                    }
+                }
+                *reinterpret_cast<uint4*>(xr + m * (p.K / 64 * 128) + blk * 128 + ((ch ^ (m & 7)) << 4)) =
+                    make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                float2 f[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) f[i] = unpack2<BF16>(wv[i]);
+                s = ((f[0].x + f[0].y) + (f[1].x + f[1].y)) + ((f[2].x + f[2].y) + (f[3].x + f[3].y));
+            }
+            // groups of 4 / 8 / 16 consecutive chunks are aligned to 32 / 64 / 128 channels
+            // (K is a multiple of 64; the 128-channel sums are only read when K is a
+            // multiple of 128)
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            if (valid && (lane & 3) == 0) s32[(c >> 2) * ss + m] = s;
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            if (valid && (lane & 7) == 0) s64[(c >> 3) * ss + m] = s;
+            s += __shfl_xor_sync(0xffffffffu, s, 8);
+            if (valid && (lane & 15) == 0 && (c >> 4) < p.K / 128) s128[(c >> 4) * ss + m] = s;
+        }
     }
 }
 
@@ -768,12 +780,12 @@ W4_DEV bool sum_shares(const DecodeParams& p, float* xc, int band, int c_first, 
 }
 
 // Who adds the contributors' shares when a part completes a band with `ncon` contributors:
-// the producer warp ahead of time (few contributors, small buffer) or all MMA warps
-// together after the last stage.
+// the producer warp ahead of time (few contributors and at most two tokens: one warp's
+// loads) or all MMA warps together after the last stage.
 constexpr int kFewShares = 2;
 template <int NT>
-W4_DEV bool producer_sums(int ncon) {
-    return Cfg<NT>::pgather && ncon <= kFewShares;
+W4_DEV bool producer_sums(const DecodeParams& p, int ncon) {
+    return Cfg<NT>::pgather && ncon <= kFewShares && p.M <= 2;
 }
 
 // Combine the partial sums of a row tile's sets (stage groups x K slices) in shared memory:
@@ -860,7 +872,7 @@ W4_DEV void complete_band(const DecodeParams& p, unsigned char* smem, unsigned c
     using C = Cfg<NT>;
     const int tb = band_tiles(p, band);
     const int c_first = cta_of_unit(p, band * p.KU);
-    if (!producer_sums<NT>(cta - c_first)) {
+    if (!producer_sums<NT>(p, cta - c_first)) {
         // the MMA threads share the band's entries, summing the contributors' shares into a
         // slot-layout buffer (the exchange buffer, or with a single set the first ring stage,
         // idle once every MMA warp is past the last stage); set 0 adds them
@@ -1083,7 +1095,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
             // the last part completes band b0 when the range starts inside it: sum the
             // earlier CTAs' shares while the MMA warps work through the last stages
             const int bu0 = it.b0 * p.KU;
-            if (u0 > bu0 && u1 >= bu0 + p.KU && producer_sums<NT>(cta - cta_of_unit(p, bu0))) {
+            if (u0 > bu0 && u1 >= bu0 + p.KU && producer_sums<NT>(p, cta - cta_of_unit(p, bu0))) {
                 pdl_wait();   // the shares are this grid's, the slots cleared by the preceding one
                 const bool ok = !abort && gather_shares<NT>(p, gsum, it.b0, cta, lane);
                 if (!ok) *s_abort = 1;
