@@ -69,9 +69,6 @@ struct Cfg {
     static constexpr int sx_floats = 4 * aps * mpad;
     // partial-sum sets per row tile at a flush: stage groups x K slices
     static constexpr int nset = groups * kparts;
-    // the producer warp sums the contributors' shares of a completed band ahead of the
-    // flush (into [M][128] fp32 of shared memory) when that buffer is small
-    static constexpr bool pgather = NT <= 2;
     // MMA-warp exchange buffer: [nset-1][8 tiles][NT][4][32 lanes] fp32
     static constexpr int xchg_bytes = (nset - 1) * 8 * NT * 4 * 32 * 4;
 };
@@ -99,7 +96,6 @@ struct DecodeParams {
     int off_res_s;            // byte offset of the resident sums: [K/32 | K/64 | K/128][sstride]
     int sstride;              // tokens per row of the activation sums
     int off_xchg;             // byte offset of the MMA-warp exchange buffer
-    int off_gsum;             // byte offset of the contributors' sums of the completed band: [M][128] fp32
     // byte offsets inside one stage
     int off_x, off_xs, off_sx, off_si, off_sc, off_zr, off_gi, off_desc, stage_bytes;
 };
@@ -703,52 +699,6 @@ W4_DEV int share_slot(int x, int M) {
     return (((nl >> 4) * NT + (m >> 3)) * 4 + 2 * (r >> 3) + (m & 1)) * 32 + 4 * (r & 7) + ((m & 7) >> 1);
 }
 
-// Producer warp, once its copies are out: sum the shares that CTAs [c_first, cta) published
-// for `band` (CTA order per entry) into gsum[m][n - band start], for the MMA warps'
-// completing flush.  Entries are spread over the lanes four at a time, and the loads of two
-// contributors of those entries go out together.  False on a timed-out wait.
-template <int NT>
-W4_DEV bool gather_shares(const DecodeParams& p, float* gsum, int band, int cta, int lane) {
-    constexpr int kSlot = kTilesPerBand * NT * 4 * 32;
-    const int n_ent = band_tiles(p, band) * 16 * p.M;
-    const int c_first = cta_of_unit(p, band * p.KU);
-    for (int x0 = 0; x0 < n_ent; x0 += 128) {
-        int j[4];
-        float tot[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int x = x0 + 32 * k + lane;
-            j[k] = x < n_ent ? share_slot<NT>(x, p.M) : -1;
-            tot[k] = 0.0f;
-        }
-        for (int c0 = c_first; c0 < cta; c0 += 2) {
-            unsigned long long v[4][2];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-                for (int b = 0; b < 2; ++b)
-                    v[k][b] = j[k] >= 0 && c0 + b < cta ? slot_get(p.slots + (size_t)(c0 + b) * kSlot + j[k]) : 0ull;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-                for (int b = 0; b < 2; ++b) {
-                    if (j[k] < 0 || c0 + b >= cta) continue;
-                    unsigned long long* a = p.slots + (size_t)(c0 + b) * kSlot + j[k];
-                    float val = __uint_as_float((uint32_t)v[k][b]);
-                    if ((v[k][b] >> 32) == 0 && !slot_wait(a, val)) return false;
-                    tot[k] += val;
-                    slot_clear(a);
-                }
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int x = x0 + 32 * k + lane;
-            if (x < n_ent) gsum[(x % p.M) * kBandRows + x / p.M] = tot[k];
-        }
-    }
-    return true;
-}
-
 // MMA thread mt of nthr: for each entry x = mt, mt + nthr, ... of the band, xc[slot] = the
 // sum of the shares CTAs [c_first, cta) published, in CTA order; the loads of up to eight
 // contributors of an entry go out together.  False on a timed-out wait.
@@ -779,17 +729,6 @@ W4_DEV bool sum_shares(const DecodeParams& p, float* xc, int band, int c_first, 
     return true;
 }
 
-// Who adds the contributors' shares when a part completes a band with `ncon` contributors:
-// the producer warp ahead of time (few contributors and at most two tokens: one warp's
-// loads) or all MMA warps together after the last stage.
-constexpr int kFewShares = 2;
-template <int NT>
-W4_DEV bool producer_sums(const DecodeParams& p, int ncon) {
-    return Cfg<NT>::pgather && ncon <= kFewShares && p.M <= 2;
-}
-
-// Combine the partial sums of a row tile's sets (stage groups x K slices) in shared memory:
-// set 0 adds the others in a fixed order.  Every MMA warp takes part (named barriers).
 template <int NT, int TPW>
 W4_DEV void combine_sets(unsigned char* xchg, int set, int t0, const Lane& L, float (&acc)[TPW][NT][4]) {
     using C = Cfg<NT>;
@@ -867,49 +806,31 @@ W4_DEV void flush_part(const DecodeParams& p, int band, int pe, int cta, int t0,
 // loop, on every MMA warp (named barriers on the shared path).
 template <int NT, int TPW>
 W4_DEV void complete_band(const DecodeParams& p, unsigned char* smem, unsigned char* xchg, volatile int* s_abort,
-                          const float* gsum, uint64_t* gready, int band, int cta, int set, int t0, const Lane& L,
-                          bool aborted, float (&acc)[TPW][NT][4]) {
+                          int band, int cta, int set, int t0, const Lane& L, bool aborted,
+                          float (&acc)[TPW][NT][4]) {
     using C = Cfg<NT>;
     const int tb = band_tiles(p, band);
     const int c_first = cta_of_unit(p, band * p.KU);
-    if (!producer_sums<NT>(p, cta - c_first)) {
-        // the MMA threads share the band's entries, summing the contributors' shares into a
-        // slot-layout buffer (the exchange buffer, or with a single set the first ring stage,
-        // idle once every MMA warp is past the last stage); set 0 adds them
-        float* xc = reinterpret_cast<float*>(C::nset > 1 ? xchg : smem);
-        if constexpr (C::nset == 1) named_bar_sync(1, 32 * C::mma_warps);
-        const int mt = threadIdx.x - 32 * (1 + C::xw);
-        if (!aborted && !sum_shares<NT>(p, xc, band, c_first, cta, mt, 32 * C::mma_warps)) *s_abort = 1;
-        named_bar_sync(1, 32 * C::mma_warps);
-        if (set == 0) {
+    // the MMA threads share the band's entries, summing the contributors' shares into a
+    // slot-layout buffer (the exchange buffer, or with a single set the first ring stage,
+    // idle once every MMA warp is past the last stage); set 0 adds them
+    float* xc = reinterpret_cast<float*>(C::nset > 1 ? xchg : smem);
+    if constexpr (C::nset == 1) named_bar_sync(1, 32 * C::mma_warps);
+    const int mt = threadIdx.x - 32 * (1 + C::xw);
+    if (!aborted && !sum_shares<NT>(p, xc, band, c_first, cta, mt, 32 * C::mma_warps)) *s_abort = 1;
+    named_bar_sync(1, 32 * C::mma_warps);
+    if (set == 0) {
 #pragma unroll
-            for (int tt = 0; tt < TPW; ++tt)
+        for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane;
-                        if (t0 + tt < tb && 8 * nt + 2 * L.q + (e & 1) < p.M) acc[tt][nt][e] = xc[j] + acc[tt][nt][e];
-                    }
-        }
-        named_bar_sync(2, 32 * C::mma_warps);
-    } else {
-        if (set > 0 || aborted) return;
-        // the producer warp has summed the contributors' shares into gsum
-        if (!mbar_wait(gready, 0)) *s_abort = 1;
-        if (!*s_abort) {
-#pragma unroll
-            for (int tt = 0; tt < TPW; ++tt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int m = 8 * nt + 2 * L.q + (e & 1);
-                        const int nl = 16 * (t0 + tt) + L.g8 + 8 * (e >> 1);
-                        if (m < p.M && t0 + tt < tb) acc[tt][nt][e] = gsum[m * kBandRows + nl] + acc[tt][nt][e];
-                    }
-        }
+                for (int e = 0; e < 4; ++e) {
+                    const int j = (((t0 + tt) * NT + nt) * 4 + e) * 32 + L.lane;
+                    if (t0 + tt < tb && 8 * nt + 2 * L.q + (e & 1) < p.M) acc[tt][nt][e] = xc[j] + acc[tt][nt][e];
+                }
     }
+    named_bar_sync(2, 32 * C::mma_warps);
     if (set > 0 || aborted || *s_abort) return;
     store_rows<NT, TPW>(p, band, t0, L, acc);
 }
@@ -952,8 +873,6 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
     uint64_t* xready = full + kMaxStages;
     uint64_t* empty = xready + kMaxStages;
     volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
-    uint64_t* gready = empty + kMaxStages + 1;   // contributors' sums in gsum
-    float* gsum = reinterpret_cast<float*>(smem + p.off_gsum);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
@@ -966,7 +885,6 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
             mbar_init(&xready[s], 32 * C::xw);
             mbar_init(&empty[s], C::stage_warps);
         }
-        mbar_init(gready, 1);
         *s_abort = 0;
         fence_mbar_init();
     }
@@ -1091,18 +1009,6 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                 if (k >= i - S) (void)mbar_wait(&full[q.s], q.ph);
         }
         __syncwarp();
-        if constexpr (C::pgather) {
-            // the last part completes band b0 when the range starts inside it: sum the
-            // earlier CTAs' shares while the MMA warps work through the last stages
-            const int bu0 = it.b0 * p.KU;
-            if (u0 > bu0 && u1 >= bu0 + p.KU && producer_sums<NT>(p, cta - cta_of_unit(p, bu0))) {
-                pdl_wait();   // the shares are this grid's, the slots cleared by the preceding one
-                const bool ok = !abort && gather_shares<NT>(p, gsum, it.b0, cta, lane);
-                if (!ok) *s_abort = 1;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(gready);
-            }
-        }
     } else {
     if (p.xres) {
         // ------------------------------------------------------------ resident X'
@@ -1200,7 +1106,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
             zero_acc<NT, TPW>(acc);
         }
         if (u0 > it.b0 * p.KU && u1 >= (it.b0 + 1) * p.KU)
-            complete_band<NT, TPW>(p, smem, xchg, s_abort, gsum, gready, it.b0, cta, set, t0, L, aborted, acc);
+            complete_band<NT, TPW>(p, smem, xchg, s_abort, it.b0, cta, set, t0, L, aborted, acc);
     }
     }
 }

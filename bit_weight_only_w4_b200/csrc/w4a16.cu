@@ -201,14 +201,12 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     p.stage_bytes = (p.off_desc + 48 + 1023) / 1024 * 1024;
     // as many stages as fit: the CTA fills the SM's shared memory, one CTA per SM
     const int resident = p.xres ? res_x + res_s : 0;
-    const int gsum = C::pgather ? up(p.M * w4d::kBandRows * 4, 128) : 0;
-    const int fixed = resident + gsum + C::xchg_bytes + 3 * w4d::kMaxStages * 8 + 16 + 1024;
+    const int fixed = resident + C::xchg_bytes + 3 * w4d::kMaxStages * 8 + 16 + 1024;
     p.stages = std::min(w4d::kMaxStages, (kMaxSmem - fixed) / p.stage_bytes);
     if (p.stages < 2) return W4_ERR_UNSUPPORTED;
     p.off_res = p.stages * p.stage_bytes;
     p.off_res_s = p.off_res + res_x;
-    p.off_gsum = p.off_res + resident;
-    p.off_xchg = p.off_gsum + gsum;
+    p.off_xchg = p.off_res + resident;
     const int smem = p.stages * p.stage_bytes + fixed;
     p.X = X;
     const int bands = (p.tiles + w4d::kTilesPerBand - 1) / w4d::kTilesPerBand;
