@@ -54,7 +54,7 @@ template <int NT>
 struct Cfg {
     static constexpr int tpw = NT <= 2 ? 2 : 1;          // row tiles per MMA warp
     static constexpr int aps = NT == 1 ? 8 : 4;          // atoms (64-channel blocks) per stage
-    static constexpr int xw = NT == 1 ? 1 : NT <= 4 ? 2 : 4;   // activation warps
+    static constexpr int xw = NT == 1 ? 1 : NT <= 4 ? 3 : 4;   // activation warps
     static constexpr int mma_warps = NT <= 4 ? 16 : 8;
     static constexpr int groups = mma_warps / 8;         // stage-parity groups
     static constexpr int stage_warps = mma_warps / groups;   // MMA warps sharing a stage
@@ -579,44 +579,69 @@ W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw,
     unsigned char* xs = st + p.off_xs;
     float* sx = reinterpret_cast<float*>(st + p.off_sx);
     const float* si = reinterpret_cast<const float*>(st + p.off_si);
-    for (int base = 32 * xw; base < p.M * CPT; base += 32 * C::xw) {
-        const int m = base / CPT;
-        const int c = base % CPT + lane;
-        const int blk = c >> 3, ch = c & 7;
-        float s = 0.0f;
-        if (c < 8 * na) {
-            // the tensor box holds M rows per column block, 128B-swizzled by line index
-            const int line = blk * p.M + m;
-            const uint4 v = ld_u128(xb + line * 128 + ((ch ^ (line & 7)) << 4));
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            if (p.s_inv) {
-                const float4 s0 = *reinterpret_cast<const float4*>(si + 8 * c);
-                const float4 s1 = *reinterpret_cast<const float4*>(si + 8 * c + 4);
-                const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    // two passes (token-row chunks base and base + 32 * xw) per iteration, their loads
+    // issued together
+    for (int base = 32 * xw; base < p.M * CPT; base += 64 * C::xw) {
+        int mm[2], cc[2];
+        bool act[2], ld[2];
+        uint4 v[2];
+        float sv[2][8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = unpack2<BF16>(w[i]);
-                    w[i] = pack2<BF16>(__fmul_rn(f.x, sv[2 * i]), __fmul_rn(f.y, sv[2 * i + 1]));
+        for (int u = 0; u < 2; ++u) {
+            const int b = base + 32 * C::xw * u;
+            act[u] = b < p.M * CPT;
+            mm[u] = b / CPT;
+            cc[u] = b % CPT + lane;
+            ld[u] = act[u] && cc[u] < 8 * na;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sv[u][i] = 1.0f;
+            if (ld[u]) {
+                // the tensor box holds M rows per column block, 128B-swizzled by line index
+                const int line = (cc[u] >> 3) * p.M + mm[u];
+                v[u] = ld_u128(xb + line * 128 + (((cc[u] & 7) ^ (line & 7)) << 4));
+                if (p.s_inv) {
+                    const float4 s0 = *reinterpret_cast<const float4*>(si + 8 * cc[u]);
+                    const float4 s1 = *reinterpret_cast<const float4*>(si + 8 * cc[u] + 4);
+                    sv[u][0] = s0.x; sv[u][1] = s0.y; sv[u][2] = s0.z; sv[u][3] = s0.w;
+                    sv[u][4] = s1.x; sv[u][5] = s1.y; sv[u][6] = s1.z; sv[u][7] = s1.w;
                 }
             }
-            // X': [token row][column block][128 B], lines swizzled by token row
-            *reinterpret_cast<uint4*>(xs + m * (C::aps * 128) + blk * 128 + ((ch ^ (m & 7)) << 4)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-            if constexpr (!GIDX) {
-                float2 f[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) f[i] = unpack2<BF16>(w[i]);
-                s = ((f[0].x + f[0].y) + (f[1].x + f[1].y)) + ((f[2].x + f[2].y) + (f[3].x + f[3].y));
-            }
         }
-        if constexpr (!GIDX) {
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
-            if ((lane & 3) == 0) sx[(C::sx32 + (c >> 2)) * C::mpad + m] = s;
-            s += __shfl_xor_sync(0xffffffffu, s, 4);
-            if ((lane & 7) == 0) sx[(C::sx64 + (c >> 3)) * C::mpad + m] = s;
-            s += __shfl_xor_sync(0xffffffffu, s, 8);
-            if ((lane & 15) == 0) sx[(C::sx128 + (c >> 4)) * C::mpad + m] = s;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (!act[u]) break;
+            const int m = mm[u], c = cc[u];
+            const int blk = c >> 3, ch = c & 7;
+            float s = 0.0f;
+            if (ld[u]) {
+                uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                if (p.s_inv) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 f = unpack2<BF16>(w[i]);
+                        w[i] = pack2<BF16>(__fmul_rn(f.x, sv[u][2 * i]), __fmul_rn(f.y, sv[u][2 * i + 1]));
+                    }
+                }
+                // X': [token row][column block][128 B], lines swizzled by token row
+                *reinterpret_cast<uint4*>(xs + m * (C::aps * 128) + blk * 128 + ((ch ^ (m & 7)) << 4)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+                if constexpr (!GIDX) {
+                    float2 f[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) f[i] = unpack2<BF16>(w[i]);
+                    s = ((f[0].x + f[0].y) + (f[1].x + f[1].y)) + ((f[2].x + f[2].y) + (f[3].x + f[3].y));
+                }
+            }
+            if constexpr (!GIDX) {
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                if ((lane & 3) == 0) sx[(C::sx32 + (c >> 2)) * C::mpad + m] = s;
+                s += __shfl_xor_sync(0xffffffffu, s, 4);
+                if ((lane & 7) == 0) sx[(C::sx64 + (c >> 3)) * C::mpad + m] = s;
+                s += __shfl_xor_sync(0xffffffffu, s, 8);
+                if ((lane & 15) == 0) sx[(C::sx128 + (c >> 4)) * C::mpad + m] = s;
+            }
         }
     }
 }
@@ -893,7 +918,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
         const int words = (p.K / 32 + p.K / 64 + p.K / 128) * p.sstride;
         for (int i = threadIdx.x; i < words; i += C::threads)
             reinterpret_cast<float*>(smem + p.off_res_s)[i] = 0.0f;
-    } else {
+    } else if (p.M < C::mpad) {
         const int words = (p.off_si - p.off_xs) / 4;   // X' and sums of one stage
         for (int i = threadIdx.x; i < S * words; i += C::threads)
             reinterpret_cast<uint32_t*>(smem + (i / words) * p.stage_bytes + p.off_xs)[i % words] = 0u;
