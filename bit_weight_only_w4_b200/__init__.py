@@ -66,6 +66,14 @@ def lib():
         L.w4_selftest_expired_wait.restype = st
         L.w4_status_string.argtypes = [st]
         L.w4_status_string.restype = ctypes.c_char_p
+        L.w4_actorder_perm.argtypes = [vp, i64, i32, vp, vp]
+        L.w4_actorder_perm.restype = st
+        L.w4_quantize_pack_perm.argtypes = [vp, st, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp]
+        L.w4_quantize_pack_perm.restype = st
+        L.w4a16_gemm_perm.argtypes = [vp, st, i64, i64, i64, vp, vp, vp, vp, i32, vp, vp, st, vp, sz, vp]
+        L.w4a16_gemm_perm.restype = st
+        L.w4a16_workspace_bytes_perm.argtypes = [i64, i64, i64, i32]
+        L.w4a16_workspace_bytes_perm.restype = sz
         _lib = L
     return _lib
 
@@ -140,16 +148,36 @@ def w4a16_workspace_bytes(M, N, K, group_size):
     return int(lib().w4a16_workspace_bytes(int(M), int(N), int(K), int(group_size)))
 
 
+def w4_actorder_perm(g_idx, group_size, perm=None, stream=None):
+    """perm int32 [K]: the channels sorted by g_idx (ties in channel order), for packing
+    act-order weights with contiguous groups (every group must hold group_size channels;
+    otherwise w4_check_device_error() reports W4_ERR_DEVICE_ARG)."""
+    torch = _torch()
+    K = g_idx.shape[0]
+    dev = _need_cuda(g_idx, perm)
+    if g_idx.dtype != torch.int32:
+        raise TypeError("g_idx must be int32")
+    if perm is None:
+        perm = torch.empty(K, dtype=torch.int32, device=dev)
+    with _DeviceGuard(dev):
+        st = lib().w4_actorder_perm(_ptr(g_idx), K, int(group_size), _ptr(perm), _stream_handle(stream, dev))
+    _check(st, "w4_actorder_perm")
+    return perm
+
+
 def w4_quantize_pack(W, s=None, group_size=128, symmetric=False, g_idx=None,
-                     qweight=None, scales=None, zeros=None, stream=None):
+                     qweight=None, scales=None, zeros=None, stream=None, perm=None):
     """AWQ scaling + group-wise RTN INT4 + packing of W [N,K] (fp16/bf16, CUDA).
 
-    Returns (qweight uint32-as-int32 [N*K/8] device layout, scales fp16 [G,N],
-    zeros fp16 [G,N] or None when symmetric)."""
+    With perm (from w4_actorder_perm; g_idx then None) column k of the packed matrix is
+    channel perm[k] and groups are contiguous.  Returns (qweight uint32-as-int32 [N*K/8]
+    device layout, scales fp16 [G,N], zeros fp16 [G,N] or None when symmetric)."""
     torch = _torch()
     N, K = W.shape
     G = K // group_size
-    dev = _need_cuda(W, s, g_idx, qweight, scales, zeros)
+    if perm is not None and g_idx is not None:
+        raise ValueError("pass g_idx or perm, not both")
+    dev = _need_cuda(W, s, g_idx, qweight, scales, zeros, perm)
     if qweight is None:
         qweight = torch.empty(N * K // 8, dtype=torch.int32, device=dev)
     if scales is None:
@@ -160,10 +188,17 @@ def w4_quantize_pack(W, s=None, group_size=128, symmetric=False, g_idx=None,
         raise TypeError("s must be float32")
     if g_idx is not None and g_idx.dtype != torch.int32:
         raise TypeError("g_idx must be int32")
+    if perm is not None and perm.dtype != torch.int32:
+        raise TypeError("perm must be int32")
     with _DeviceGuard(dev):
-        st = lib().w4_quantize_pack(_ptr(W), _dtype_code(W.dtype), N, K, _ptr(s), int(group_size),
-                                    int(bool(symmetric)), _ptr(g_idx), _ptr(qweight),
-                                    _ptr(scales), _ptr(zeros), _stream_handle(stream, dev))
+        if perm is not None:
+            st = lib().w4_quantize_pack_perm(_ptr(W), _dtype_code(W.dtype), N, K, _ptr(s), int(group_size),
+                                             int(bool(symmetric)), _ptr(perm), _ptr(qweight),
+                                             _ptr(scales), _ptr(zeros), _stream_handle(stream, dev))
+        else:
+            st = lib().w4_quantize_pack(_ptr(W), _dtype_code(W.dtype), N, K, _ptr(s), int(group_size),
+                                        int(bool(symmetric)), _ptr(g_idx), _ptr(qweight),
+                                        _ptr(scales), _ptr(zeros), _stream_handle(stream, dev))
     _check(st, "w4_quantize_pack")
     return qweight, scales, zeros
 
@@ -186,25 +221,39 @@ def workspace_for(device, nbytes):
 
 
 def w4a16_gemm(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None,
-               out_dtype=None, Y=None, workspace=None, stream=None):
-    """Y[M,N] = (X * s_inv)[M,K] @ dequant(qweight, scales, zeros, g_idx)^T on the GPU."""
+               out_dtype=None, Y=None, workspace=None, stream=None, perm=None):
+    """Y[M,N] = (X * s_inv)[M,K] @ dequant(qweight, scales, zeros, g_idx)^T on the GPU.
+
+    With perm, the weights were packed with that permutation (w4_quantize_pack(perm=...))
+    and the activation columns are gathered through it (w4a16_gemm_perm)."""
     torch = _torch()
     M, K = X.shape
     N = scales.shape[1]
-    dev = _need_cuda(X, qweight, scales, zeros, g_idx, s_inv, Y, workspace)
+    if perm is not None and g_idx is not None:
+        raise ValueError("pass g_idx or perm, not both")
+    dev = _need_cuda(X, qweight, scales, zeros, g_idx, s_inv, Y, workspace, perm)
     out_dtype = out_dtype or X.dtype
     if Y is None:
         Y = torch.empty(M, N, dtype=out_dtype, device=dev)
     with _DeviceGuard(dev):
-        need = w4a16_workspace_bytes(M, N, K, group_size) if M > 0 else 0
+        if perm is not None:
+            need = lib().w4a16_workspace_bytes_perm(M, N, K, int(group_size)) if M > 0 else 0
+        else:
+            need = w4a16_workspace_bytes(M, N, K, group_size) if M > 0 else 0
         if workspace is None and need > 0:
             workspace = workspace_for(dev, need)
         ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-        st = lib().w4a16_gemm(_ptr(X), _dtype_code(X.dtype), M, N, K, _ptr(qweight), _ptr(scales),
-                              _ptr(zeros), _ptr(g_idx), int(group_size), _ptr(s_inv), _ptr(Y),
-                              _dtype_code(Y.dtype), _ptr(workspace), ws_bytes,
-                              _stream_handle(stream, dev))
-    _check(st, "w4a16_gemm")
+        if perm is not None:
+            st = lib().w4a16_gemm_perm(_ptr(X), _dtype_code(X.dtype), M, N, K, _ptr(qweight), _ptr(scales),
+                                       _ptr(zeros), _ptr(perm), int(group_size), _ptr(s_inv), _ptr(Y),
+                                       _dtype_code(Y.dtype), _ptr(workspace), ws_bytes,
+                                       _stream_handle(stream, dev))
+        else:
+            st = lib().w4a16_gemm(_ptr(X), _dtype_code(X.dtype), M, N, K, _ptr(qweight), _ptr(scales),
+                                  _ptr(zeros), _ptr(g_idx), int(group_size), _ptr(s_inv), _ptr(Y),
+                                  _dtype_code(Y.dtype), _ptr(workspace), ws_bytes,
+                                  _stream_handle(stream, dev))
+    _check(st, "w4a16_gemm_perm" if perm is not None else "w4a16_gemm")
     return Y
 
 

@@ -80,6 +80,7 @@ struct DecodeParams {
     const __half* zeros;      // [G,N] or null
     const int32_t* g_idx;     // [K] or null
     const float* s_inv;       // [K] or null
+    const int32_t* perm;      // [K] or null: X' column k is channel perm[k] (resident X' only)
     const void* X;            // [M,K] activations (read directly when X' is resident)
     void* Y;                  // [M,N]
     unsigned long long* slots;   // split-K partials: [P][8 tiles][NT][4][32] {fp32 bits, flag}
@@ -667,16 +668,48 @@ W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* x
         float sv[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) sv[i] = 1.0f;
-        if (p.s_inv && valid) {
-            const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c);
-            const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c + 1);
-            sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
-            sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
-        }
         uint4 v[8];
+        if (p.perm) {
+            // act-order weights packed with contiguous groups: gather channel perm[k] into
+            // column k (an entry outside [0, K) is reported and reads channel 0)
+            int src[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (valid) {
+                const int4 p0 = __ldg(reinterpret_cast<const int4*>(p.perm) + 2 * c);
+                const int4 p1 = __ldg(reinterpret_cast<const int4*>(p.perm) + 2 * c + 1);
+                src[0] = p0.x; src[1] = p0.y; src[2] = p0.z; src[3] = p0.w;
+                src[4] = p1.x; src[5] = p1.y; src[6] = p1.z; src[7] = p1.w;
 #pragma unroll
-        for (int m = 0; m < 8; ++m)
-            v[m] = (valid && m < p.M) ? x4[(size_t)m * cpt + c] : make_uint4(0u, 0u, 0u, 0u);
+                for (int i = 0; i < 8; ++i)
+                    if (src[i] < 0 || src[i] >= p.K) {
+                        atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
+                        src[i] = 0;
+                    }
+                if (p.s_inv) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) sv[i] = __ldg(p.s_inv + src[i]);
+                }
+            }
+            const unsigned short* xh = reinterpret_cast<const unsigned short*>(X);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                uint32_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                if (valid && m < p.M) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) h[i] = xh[(size_t)m * p.K + src[i]];
+                }
+                v[m] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+            }
+        } else {
+            if (p.s_inv && valid) {
+                const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c);
+                const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.s_inv) + 2 * c + 1);
+                sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+                sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+                v[m] = (valid && m < p.M) ? x4[(size_t)m * cpt + c] : make_uint4(0u, 0u, 0u, 0u);
+        }
         const int blk = c >> 3, ch = c & 7;
 #pragma unroll
         for (int m = 0; m < 8; ++m) {

@@ -18,6 +18,7 @@ struct QuantParams {
     const void* W;          // [N,K] fp16 or bf16
     const float* s;         // [K] or null
     const int32_t* g_idx;   // [K] or null
+    const int32_t* perm;    // [K] or null: column k of the packed matrix is channel perm[k]
     uint32_t* qweight;      // [N*K/8] device layout
     __half* scales;         // [G,N]
     __half* zeros;          // [G,N] or null (symmetric)
@@ -37,11 +38,20 @@ W4_DEV float load_w(const void* W, size_t idx) {
     else return __half2float(reinterpret_cast<const __half*>(W)[idx]);
 }
 
-// W'[n,k] = fp32(W) * s[k]: exactly one fp32 rounding (no contraction).
+// W'[n,k] = fp32(W) * s[k]: exactly one fp32 rounding (no contraction).  With perm,
+// column k is channel perm[k] (an entry outside [0, K) is reported and reads channel 0).
 template <bool BF16W>
 W4_DEV float scaled_w(const QuantParams& p, int n, int k) {
-    float w = load_w<BF16W>(p.W, (size_t)n * p.K + k);
-    return p.s ? __fmul_rn(w, __ldg(p.s + k)) : w;
+    int src = k;
+    if (p.perm) {
+        src = __ldg(p.perm + k);
+        if (src < 0 || src >= p.K) {
+            atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
+            src = 0;
+        }
+    }
+    float w = load_w<BF16W>(p.W, (size_t)n * p.K + src);
+    return p.s ? __fmul_rn(w, __ldg(p.s + src)) : w;
 }
 
 W4_DEV int group_of(const QuantParams& p, int k) {

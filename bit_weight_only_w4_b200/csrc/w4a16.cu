@@ -11,6 +11,7 @@
 #include "w4_decode.cuh"
 #include "w4_prefill.cuh"
 #include "w4_quant.cuh"
+#include "w4_actorder.cuh"
 
 namespace {
 
@@ -161,6 +162,14 @@ bool make_meta_map(CUtensorMap* map, const void* base, int64_t G, int64_t N, int
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// X' and its sums stay resident in shared memory (one token tile, M*K small).
+bool decode_x_resident(int64_t M, int64_t K) {
+    auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
+    if (M > 8) return false;
+    const int64_t sstride = std::max<int64_t>(2, (M + 1) / 2 * 2);
+    return up(M * K * 2, 128) + up((K / 32 + K / 64 + K / 128) * sstride * 4, 128) <= 80 * 1024;
+}
+
 template <int NT, bool BF16, int MODE>
 w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
                         cudaStream_t stream) {
@@ -181,7 +190,8 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     const int sstride_res = std::max(2, (int)((p.M + 1) / 2 * 2));
     const int res_x = up(p.M * p.K * 2, 128);
     const int res_s = up((p.K / 32 + p.K / 64 + p.K / 128) * sstride_res * 4, 128);
-    p.xres = (NT == 1 && !GIDX && res_x + res_s <= 80 * 1024) ? 1 : 0;
+    p.xres = (NT == 1 && !GIDX && decode_x_resident(p.M, p.K)) ? 1 : 0;
+    if (p.perm && !p.xres) return W4_ERR_UNSUPPORTED;   // the column gather is part of the resident X'
     p.sstride = p.xres ? sstride_res : C::mpad;
     // stage layout: codes | activation box (M rows) | X' | activation sums | s_inv |
     // scale rows | zero-point rows | g_idx   (no activation parts when X' is resident)
@@ -313,29 +323,18 @@ w4_status launch_prefill(const CUtensorMap& map, const w4p::PrefillParams& p, in
 
 }  // namespace
 
-extern "C" {
-
-const char* w4_status_string(w4_status s) {
-    switch (s) {
-        case W4_OK: return "W4_OK";
-        case W4_ERR_INVALID_ARG: return "W4_ERR_INVALID_ARG";
-        case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED";
-        case W4_ERR_CUDA: return "W4_ERR_CUDA";
-        case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT";
-        case W4_ERR_DEVICE_ARG: return "W4_ERR_DEVICE_ARG";
-    }
-    return "W4_ERR_UNKNOWN";
-}
-
-w4_status w4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, const float* s,
-                           int32_t group_size, int32_t symmetric, const int32_t* g_idx,
-                           uint32_t* qweight, void* scales, void* zeros, w4_stream_t stream) {
+// AWQ scaling + group RTN + packing; with perm (g_idx then NULL) column k of the packed
+// matrix is channel perm[k] and groups are contiguous runs of group_size columns.
+static w4_status quantize_pack_impl(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, const float* s,
+                             int32_t group_size, int32_t symmetric, const int32_t* g_idx,
+                             const int32_t* perm, uint32_t* qweight, void* scales, void* zeros,
+                             w4_stream_t stream) {
     if (!W || !qweight || !scales) return W4_ERR_INVALID_ARG;
     if (w_dtype != W4_F16 && w_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
     if (symmetric != 0 && symmetric != 1) return W4_ERR_INVALID_ARG;
     if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return W4_ERR_INVALID_ARG;
     if (!aligned(W, 2) || !aligned(qweight, 4) || !aligned(scales, 2) || !aligned(zeros, 2) ||
-        !aligned(s, 4) || !aligned(g_idx, 4))
+        !aligned(s, 4) || !aligned(g_idx, 4) || !aligned(perm, 4))
         return W4_ERR_INVALID_ARG;
     w4_status st = check_layer_shape(N, K, group_size);
     if (st != W4_OK) return st;
@@ -346,6 +345,7 @@ w4_status w4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K
     p.W = W;
     p.s = s;
     p.g_idx = g_idx;
+    p.perm = perm;
     p.qweight = qweight;
     p.scales = reinterpret_cast<__half*>(scales);
     p.zeros = reinterpret_cast<__half*>(zeros);
@@ -370,6 +370,46 @@ w4_status w4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K
     return launch_status();
 }
 
+extern "C" {
+
+const char* w4_status_string(w4_status s) {
+    switch (s) {
+        case W4_OK: return "W4_OK";
+        case W4_ERR_INVALID_ARG: return "W4_ERR_INVALID_ARG";
+        case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED";
+        case W4_ERR_CUDA: return "W4_ERR_CUDA";
+        case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT";
+        case W4_ERR_DEVICE_ARG: return "W4_ERR_DEVICE_ARG";
+    }
+    return "W4_ERR_UNKNOWN";
+}
+
+w4_status w4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, const float* s,
+                           int32_t group_size, int32_t symmetric, const int32_t* g_idx,
+                           uint32_t* qweight, void* scales, void* zeros, w4_stream_t stream) {
+    return quantize_pack_impl(W, w_dtype, N, K, s, group_size, symmetric, g_idx, nullptr, qweight, scales,
+                              zeros, stream);
+}
+
+w4_status w4_quantize_pack_perm(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, const float* s,
+                                int32_t group_size, int32_t symmetric, const int32_t* perm,
+                                uint32_t* qweight, void* scales, void* zeros, w4_stream_t stream) {
+    if (!perm) return W4_ERR_INVALID_ARG;
+    return quantize_pack_impl(W, w_dtype, N, K, s, group_size, symmetric, nullptr, perm, qweight, scales,
+                              zeros, stream);
+}
+
+w4_status w4_actorder_perm(const int32_t* g_idx, int64_t K, int32_t group_size, int32_t* perm,
+                           w4_stream_t stream) {
+    if (!g_idx || !perm || !aligned(g_idx, 4) || !aligned(perm, 16)) return W4_ERR_INVALID_ARG;
+    if (K <= 0 || K > INT_MAX || group_size <= 0 || K % group_size != 0) return W4_ERR_INVALID_ARG;
+    const int64_t G = K / group_size;
+    if (G * (int64_t)sizeof(int) > 48 * 1024) return W4_ERR_UNSUPPORTED;
+    w4a::actorder_perm_kernel<<<1, 32, (size_t)G * sizeof(int), as_stream(stream)>>>(g_idx, (int)K, group_size,
+                                                                                     (int)G, perm);
+    return launch_status();
+}
+
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size) {
     if (M < 0 || check_layer_shape(N, K, group_size) != W4_OK) return 0;
     if (M == 0) return 0;
@@ -381,11 +421,26 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size
     return kCounterBytes + slot_region_bytes(sms) + (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
 }
 
+static w4_status gemm_impl(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                           const uint32_t* qweight, const void* scales, const void* zeros,
+                           const int32_t* g_idx, const int32_t* perm, int32_t group_size,
+                           const float* s_inv, void* Y, w4_dtype out_dtype, void* workspace,
+                           size_t workspace_bytes, w4_stream_t stream);
+
 w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
                      const uint32_t* qweight, const void* scales, const void* zeros,
                      const int32_t* g_idx, int32_t group_size, const float* s_inv, void* Y,
                      w4_dtype out_dtype, void* workspace, size_t workspace_bytes,
                      w4_stream_t stream) {
+    return gemm_impl(X, act_dtype, M, N, K, qweight, scales, zeros, g_idx, nullptr, group_size, s_inv, Y,
+                     out_dtype, workspace, workspace_bytes, stream);
+}
+
+static w4_status gemm_impl(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                           const uint32_t* qweight, const void* scales, const void* zeros,
+                           const int32_t* g_idx, const int32_t* perm, int32_t group_size,
+                           const float* s_inv, void* Y, w4_dtype out_dtype, void* workspace,
+                           size_t workspace_bytes, w4_stream_t stream) {
     if (M < 0) return W4_ERR_INVALID_ARG;
     if (act_dtype != W4_F16 && act_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
     if (out_dtype != W4_F16 && out_dtype != W4_BF16 && out_dtype != W4_F32) return W4_ERR_INVALID_ARG;
@@ -403,6 +458,7 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
     const size_t need = w4a16_workspace_bytes(M, N, K, group_size);
     if (need == 0) return W4_ERR_CUDA;
     const bool prefill = M > kDecodeMaxM;
+    if (perm && (prefill || !decode_x_resident(M, K))) return W4_ERR_UNSUPPORTED;
     const bool needs_ws = !prefill || s_inv != nullptr;
     if (needs_ws && (!workspace || workspace_bytes < need)) return W4_ERR_INVALID_ARG;
     const int dev = current_device();
@@ -417,6 +473,7 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
         p.zeros = reinterpret_cast<const __half*>(zeros);
         p.g_idx = g_idx;
         p.s_inv = s_inv;
+        p.perm = perm;
         p.Y = Y;
         p.M = (int)M;
         p.N = (int)N;
@@ -462,6 +519,51 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
     if (bf16) return launch_prefill<true, false>(map, p, dev, strm);
     return gidx ? launch_prefill<false, true>(map, p, dev, strm)
                 : launch_prefill<false, false>(map, p, dev, strm);
+}
+
+size_t w4a16_workspace_bytes_perm(int64_t M, int64_t N, int64_t K, int32_t group_size) {
+    if (M < 0 || check_layer_shape(N, K, group_size) != W4_OK) return 0;
+    if (M == 0) return 0;
+    const int dev = current_device();
+    const int sms = dev >= 0 ? sm_count(dev) : 0;
+    if (sms <= 0) return 0;
+    // the gathered activations sit where the prefill path keeps its scaled activations:
+    // behind the zero region and the decode slot region, which the GEMM itself uses
+    return kCounterBytes + slot_region_bytes(sms) + (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
+}
+
+w4_status w4a16_gemm_perm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                          const uint32_t* qweight, const void* scales, const void* zeros,
+                          const int32_t* perm, int32_t group_size, const float* s_inv, void* Y,
+                          w4_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                          w4_stream_t stream) {
+    if (M < 0) return W4_ERR_INVALID_ARG;
+    if (act_dtype != W4_F16 && act_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
+    w4_status st = check_layer_shape(N, K, group_size);
+    if (st != W4_OK) return st;
+    if (M == 0) return W4_OK;
+    if (M > INT_MAX / 2 || (size_t)M * (size_t)K > (size_t)INT_MAX * 8) return W4_ERR_UNSUPPORTED;
+    if (!X || !perm || !workspace) return W4_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(perm, 16) || !aligned(s_inv, 16) || !aligned(workspace, 256))
+        return W4_ERR_INVALID_ARG;
+    const size_t need = w4a16_workspace_bytes_perm(M, N, K, group_size);
+    if (need == 0) return W4_ERR_CUDA;
+    if (workspace_bytes < need) return W4_ERR_INVALID_ARG;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    if (M <= kDecodeMaxM && decode_x_resident(M, K))   // the decode kernel gathers while preparing X'
+        return gemm_impl(X, act_dtype, M, N, K, qweight, scales, zeros, nullptr, perm, group_size, s_inv, Y,
+                         out_dtype, workspace, workspace_bytes, stream);
+    cudaStream_t strm = as_stream(stream);
+    void* xp = reinterpret_cast<unsigned char*>(workspace) + kCounterBytes + slot_region_bytes(sm_count(dev));
+    const size_t chunks = (size_t)M * (size_t)K / 8;
+    const unsigned blocks = (unsigned)std::min<size_t>((chunks + 255) / 256, (size_t)65535 * 8);
+    if (act_dtype == W4_BF16) w4a::gather_acts_kernel<true><<<blocks, 256, 0, strm>>>(X, perm, s_inv, xp, (int)M, (int)K);
+    else w4a::gather_acts_kernel<false><<<blocks, 256, 0, strm>>>(X, perm, s_inv, xp, (int)M, (int)K);
+    if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+    // the contiguous-group GEMM on the gathered, already scaled activations
+    return gemm_impl(xp, act_dtype, M, N, K, qweight, scales, zeros, nullptr, nullptr, group_size, nullptr, Y,
+                     out_dtype, workspace, workspace_bytes, stream);
 }
 
 w4_status w4_unpack_canonical(const uint32_t* qweight, int64_t N, int64_t K,

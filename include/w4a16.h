@@ -145,6 +145,65 @@ w4_status w4a16_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, in
                      w4_stream_t stream);
 
 /*
+ * Act-order weights with contiguous groups.  An act-order vector g_idx scatters each
+ * group's channels along K ("The Ultimate Guide to Quantized LLMs: GPTQ" and
+ * "Understanding Quantized Model Compression": one scale and zero point per group of
+ * input channels).  When every group holds exactly group_size channels, ordering the
+ * channels by group makes each group a contiguous run again, and the product is the same
+ * sum taken in that order:
+ *   perm[k'] = the k'-th channel in (g_idx[k], k) order   (a stable sort by group)
+ *   Y[m,n]   = sum_k' X'[m,perm[k']] * What[n,perm[k']],  group(perm[k']) = k' / group_size.
+ * w4_quantize_pack_perm packs column k' = channel perm[k'] (codes, scales and zero points
+ * identical to w4_quantize_pack with g_idx, the codes in k' order); w4a16_gemm_perm gathers
+ * the activation columns through perm (with s_inv of the original channel) and runs the
+ * contiguous-group kernels, so act-order weights stream at the speed of ordinary ones.
+ */
+
+/*
+ * w4_actorder_perm -- perm = the channels sorted by g_idx, ties in channel order.
+ *   g_idx      device int32 [K], every entry in [0, K/group_size)
+ *   perm       device int32 [K] output, 16-byte aligned
+ * One warp walks K in order (offline, once per layer).  Every group must hold exactly
+ * group_size channels: otherwise, or for an entry outside [0, K/group_size), perm is
+ * incomplete and w4_check_device_error() reports W4_ERR_DEVICE_ARG.  More than 12288 groups
+ * return W4_ERR_UNSUPPORTED.
+ */
+w4_status w4_actorder_perm(const int32_t* g_idx, int64_t K, int32_t group_size, int32_t* perm,
+                           w4_stream_t stream);
+
+/*
+ * w4_quantize_pack_perm -- w4_quantize_pack of the column-permuted matrix: column k of the
+ * packed result is channel perm[k] of W (and of s); groups are k / group_size.  Arguments
+ * as w4_quantize_pack, with perm (device int32 [K], entries in [0, K)) in place of g_idx.
+ * An entry outside [0, K) reads channel 0 and is reported as W4_ERR_DEVICE_ARG by
+ * w4_check_device_error().
+ */
+w4_status w4_quantize_pack_perm(const void* W, w4_dtype w_dtype, int64_t N, int64_t K,
+                                const float* s, int32_t group_size, int32_t symmetric,
+                                const int32_t* perm, uint32_t* qweight, void* scales,
+                                void* zeros, w4_stream_t stream);
+
+/*
+ * w4a16_gemm_perm -- Y = X' What^T for weights packed by w4_quantize_pack_perm:
+ *   Xp[m,k'] = X[m,perm[k']] * s_inv[perm[k']]  rounded to act_dtype (s_inv NULL: no scaling),
+ * written into the workspace by one gather kernel, then w4a16_gemm(Xp, ..., g_idx = NULL,
+ * s_inv = NULL).  Arguments as w4a16_gemm with perm in place of g_idx; fp16 and bf16
+ * activations.  workspace: at least w4a16_workspace_bytes_perm(M,N,K,group_size) bytes,
+ * 256-byte aligned, zero-filled before its first use (as for w4a16_gemm).  An entry of perm
+ * outside [0, K) reads channel 0 and is reported as W4_ERR_DEVICE_ARG by
+ * w4_check_device_error().
+ */
+w4_status w4a16_gemm_perm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                          const uint32_t* qweight, const void* scales, const void* zeros,
+                          const int32_t* perm, int32_t group_size, const float* s_inv,
+                          void* Y, w4_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                          w4_stream_t stream);
+
+/* Bytes of workspace w4a16_gemm_perm needs (w4a16_workspace_bytes plus M*K*2 for the
+ * gathered activations; 0 on invalid sizes). */
+size_t w4a16_workspace_bytes_perm(int64_t M, int64_t N, int64_t K, int32_t group_size);
+
+/*
  * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 32 (M <= 64 where the scratch fits)
  * without a caller-supplied workspace.  The pages have no counterpart to this call; it
  * exists for callers that cannot allocate device memory where they run the GEMM, such as

@@ -97,3 +97,26 @@ def test_binding_refuses_cpu_tensors():
     W = torch.zeros(16, 64, dtype=torch.float16)
     with pytest.raises(ValueError):
         w4.w4_quantize_pack(W, group_size=32)
+
+
+def test_actorder_entry_points_reject_bad_arguments(L):
+    v = ctypes.c_void_p
+    # w4_actorder_perm: pointers, K % group_size
+    assert L.w4_actorder_perm(None, 128, 32, v(256), None) == w4.W4_ERR_INVALID_ARG
+    assert L.w4_actorder_perm(v(256), 128, 32, None, None) == w4.W4_ERR_INVALID_ARG
+    assert L.w4_actorder_perm(v(256), 100, 32, v(256), None) == w4.W4_ERR_INVALID_ARG
+    assert L.w4_actorder_perm(v(256), 128, 0, v(256), None) == w4.W4_ERR_INVALID_ARG
+    # w4_quantize_pack_perm: perm is required
+    assert L.w4_quantize_pack_perm(v(16), 0, 16, 64, None, 32, 1, None, v(16), v(16), None, None) == \
+        w4.W4_ERR_INVALID_ARG
+    # w4a16_gemm_perm: perm and workspace are required, shapes as w4a16_gemm
+    g = L.w4a16_gemm_perm
+    assert g(v(16), 0, 1, 128, 128, v(16), v(16), None, None, 128, None, v(16), 0, v(256), 1 << 30,
+             None) == w4.W4_ERR_INVALID_ARG
+    assert g(v(16), 0, 1, 128, 128, v(16), v(16), None, v(16), 128, None, v(16), 0, None, 1 << 30,
+             None) == w4.W4_ERR_INVALID_ARG
+    assert g(v(16), 0, 1, 8, 128, v(16), v(16), None, v(16), 128, None, v(16), 0, v(256), 1 << 30,
+             None) == w4.W4_ERR_UNSUPPORTED
+    assert g(v(16), 0, 0, 128, 128, None, None, None, None, 128, None, None, 0, None, 0, None) == w4.W4_OK
+    assert L.w4a16_workspace_bytes_perm(1, 8, 128, 128) == 0
+    assert L.w4a16_workspace_bytes_perm(0, 128, 128, 128) == 0
