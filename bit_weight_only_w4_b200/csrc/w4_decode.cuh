@@ -653,7 +653,7 @@ W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw,
 // 64-channel block; sums are [segment][sstride].  Consecutive lanes take consecutive
 // 8-channel chunks, so the sums are warp shuffles; a lane takes its chunk for every token
 // (M <= 8 here), loading the chunk's s_inv once and all M activation chunks together.
-template <bool BF16>
+template <bool BF16, bool PERM>
 W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* xr, float* sr, int w,
                           int nw, int lane) {
     const int cpt = p.K / 8;                       // chunks per token
@@ -669,7 +669,7 @@ W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* x
 #pragma unroll
         for (int i = 0; i < 8; ++i) sv[i] = 1.0f;
         uint4 v[8];
-        if (p.perm) {
+        if constexpr (PERM) {
             // act-order weights packed with contiguous groups: gather channel perm[k] into
             // column k (an entry outside [0, K) is reported and reads channel 0)
             int src[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -916,7 +916,7 @@ struct Ring {
     }
 };
 
-template <int NT, bool BF16, int MODE>
+template <int NT, bool BF16, int MODE, bool PERM>
 __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_sc,
                   const __grid_constant__ CUtensorMap tmap_zr, const DecodeParams p) {
@@ -1071,7 +1071,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
     if (p.xres) {
         // ------------------------------------------------------------ resident X'
         pdl_wait();   // X may come from the preceding kernel
-        prep_resident<BF16>(p, p.X, smem + p.off_res, reinterpret_cast<float*>(smem + p.off_res_s),
+        prep_resident<BF16, PERM>(p, p.X, smem + p.off_res, reinterpret_cast<float*>(smem + p.off_res_s),
                             warp - 1, C::warps - 1, lane);
         named_bar_sync(3, C::threads - 32);
     }

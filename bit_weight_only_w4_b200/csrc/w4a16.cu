@@ -170,12 +170,12 @@ bool decode_x_resident(int64_t M, int64_t K) {
     return up(M * K * 2, 128) + up((K / 32 + K / 64 + K / 128) * sstride * 4, 128) <= 80 * 1024;
 }
 
-template <int NT, bool BF16, int MODE>
+template <int NT, bool BF16, int MODE, bool PERM>
 w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
                         cudaStream_t stream) {
     using C = w4d::Cfg<NT>;
     constexpr bool GIDX = MODE == w4d::kModeGidx;
-    auto kernel = w4d::decode_kernel<NT, BF16, MODE>;
+    auto kernel = w4d::decode_kernel<NT, BF16, MODE, PERM>;
     static std::once_flag flags[kMaxDevices];
     constexpr int kMaxSmem = 227 * 1024;
     bool attr_ok = true;
@@ -191,7 +191,8 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     const int res_x = up(p.M * p.K * 2, 128);
     const int res_s = up((p.K / 32 + p.K / 64 + p.K / 128) * sstride_res * 4, 128);
     p.xres = (NT == 1 && !GIDX && decode_x_resident(p.M, p.K)) ? 1 : 0;
-    if (p.perm && !p.xres) return W4_ERR_UNSUPPORTED;   // the column gather is part of the resident X'
+    if (PERM != (p.perm != nullptr) || (PERM && !p.xres))   // the gather is part of the resident X'
+        return W4_ERR_UNSUPPORTED;
     p.sstride = p.xres ? sstride_res : C::mpad;
     // stage layout: codes | activation box (M rows) | X' | activation sums | s_inv |
     // scale rows | zero-point rows | g_idx   (no activation parts when X' is resident)
@@ -262,27 +263,30 @@ int decode_mode(int64_t K, int32_t g, bool gidx) {
     return w4d::kModeAtom;
 }
 
-template <int NT, bool BF16>
+template <int NT, bool BF16, bool PERM>
 w4_status dispatch_mode(int mode, w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
                         cudaStream_t s) {
-    if constexpr (!BF16) {
-        if (mode == w4d::kModeGidx) return launch_decode<NT, false, w4d::kModeGidx>(p, X, ws, dev, s);
+    if constexpr (!BF16 && !PERM) {
+        if (mode == w4d::kModeGidx) return launch_decode<NT, false, w4d::kModeGidx, false>(p, X, ws, dev, s);
     } else {
         if (mode == w4d::kModeGidx) return W4_ERR_UNSUPPORTED;
     }
-    if (mode == w4d::kModeHalf) return launch_decode<NT, BF16, w4d::kModeHalf>(p, X, ws, dev, s);
-    if (mode == w4d::kModeG32) return launch_decode<NT, BF16, w4d::kModeG32>(p, X, ws, dev, s);
-    return launch_decode<NT, BF16, w4d::kModeAtom>(p, X, ws, dev, s);
+    if (mode == w4d::kModeHalf) return launch_decode<NT, BF16, w4d::kModeHalf, PERM>(p, X, ws, dev, s);
+    if (mode == w4d::kModeG32) return launch_decode<NT, BF16, w4d::kModeG32, PERM>(p, X, ws, dev, s);
+    return launch_decode<NT, BF16, w4d::kModeAtom, PERM>(p, X, ws, dev, s);
 }
 
 template <bool BF16>
 w4_status dispatch_decode(int mode, w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
                           cudaStream_t s) {
+    // act-order columns gathered while the resident X' is prepared: one token tile only
+    if (p.perm) return decode_tiles_for(p.M) == 1 ? dispatch_mode<1, BF16, true>(mode, p, X, ws, dev, s)
+                                                  : W4_ERR_UNSUPPORTED;
     switch (decode_tiles_for(p.M)) {
-        case 1: return dispatch_mode<1, BF16>(mode, p, X, ws, dev, s);
-        case 2: return dispatch_mode<2, BF16>(mode, p, X, ws, dev, s);
-        case 4: return dispatch_mode<4, BF16>(mode, p, X, ws, dev, s);
-        default: return dispatch_mode<8, BF16>(mode, p, X, ws, dev, s);
+        case 1: return dispatch_mode<1, BF16, false>(mode, p, X, ws, dev, s);
+        case 2: return dispatch_mode<2, BF16, false>(mode, p, X, ws, dev, s);
+        case 4: return dispatch_mode<4, BF16, false>(mode, p, X, ws, dev, s);
+        default: return dispatch_mode<8, BF16, false>(mode, p, X, ws, dev, s);
     }
 }
 
