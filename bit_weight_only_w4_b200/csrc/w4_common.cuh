@@ -221,28 +221,12 @@ struct ZeroConsts {
 // fp16: an fp16 with exponent field 25 (bits 0x6400) has unit spacing on [1024, 2048),
 // so OR-ing a nibble q into its low mantissa bits gives exactly 1024 + q; a nibble in
 // bits 4..7 gives 1024 + 16 q.  Subtracting (1024 + z), resp. scaling by 1/16 and
-// subtracting (64 + z), yields the exact integer q - z.
-W4_DEV ZeroConsts zero_consts_f16(float z0, float z1) {
-    ZeroConsts zc;
-    zc.lo0 = h2_as_u32(__float2half2_rn(1024.0f + z0));
-    zc.lo1 = h2_as_u32(__float2half2_rn(1024.0f + z1));
-    zc.hi0 = h2_as_u32(__float2half2_rn(-(64.0f + z0)));
-    zc.hi1 = h2_as_u32(__float2half2_rn(-(64.0f + z1)));
-    return zc;
-}
+// subtracting (64 + z), yields the exact integer q - z.  bf16: exponent 134 (bits 0x4300)
+// has unit spacing on [128, 256).
 
-// bf16: exponent 134 (bits 0x4300) has unit spacing on [128, 256).
-W4_DEV ZeroConsts zero_consts_bf16(float z0, float z1) {
-    ZeroConsts zc;
-    zc.lo0 = b2_as_u32(__float2bfloat162_rn(128.0f + z0));
-    zc.lo1 = b2_as_u32(__float2bfloat162_rn(128.0f + z1));
-    zc.hi0 = zc.lo0;
-    zc.hi1 = zc.lo1;
-    return zc;
-}
-
-// The same constants straight from the fp16 zero points (integers 0..15) of rows r0 / r1,
-// with fp16 arithmetic and byte permutes only (no type conversions):
+// The constants (bias + z) for the unpack below, straight from the fp16 zero points
+// (integers 0..15) of rows r0 / r1, with fp16 arithmetic and byte permutes only (no type
+// conversions):
 //   s = (1024 + z0, 1024 + z1)   exact in fp16, and its low mantissa nibbles are z0, z1;
 //   fp16: lo0 = (1024 + z0) x2, hi1 = (960 - (1024 + z1)) x2 = -(64 + z1) x2;
 //   bf16: lo0 = 0x4300 | z0 (x2), lo1 = 0x4300 | z1 (x2)   (128 + z in bf16).

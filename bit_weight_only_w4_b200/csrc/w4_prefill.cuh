@@ -173,11 +173,6 @@ W4_DEV void stmatrix_x4(uint32_t saddr, const uint32_t (&r)[4]) {
                  : "memory");
 }
 
-// byte offset of element (row, k) in a 128B-swizzled K-major tile (k < 64, 2-byte elems)
-W4_DEV uint32_t sw128_off(int row, int k) {
-    return (uint32_t)(row * 128 + ((((k >> 3) ^ (row & 7)) & 7) << 4) + ((k & 7) << 1));
-}
-
 W4_DEV void store_out(const PrefillParams& p, int m, int n, float v) {
     const size_t idx = (size_t)m * p.N + n;
     if (p.out_dtype == 2) reinterpret_cast<float*>(p.Y)[idx] = v;
