@@ -365,6 +365,22 @@ def time_actorder(w4, torch, M=1, g=128, copies=16, launches=64):
     return out
 
 
+def time_awq_search(w4, torch, M=128, n_grid=20):
+    """AWQ's scale search on one 4096 x 4096 layer with M seeded calibration rows: time of
+    the whole search, the chosen exponent and how much it lowers the output error."""
+    wl = workloads.workload(1)
+    li = workloads.make_layer(wl, 0, M=M)
+    W = dev_bits(li.W.view(np.uint16), torch.float16)
+    X = dev_bits(li.X, torch.float16)
+    w4.w4_awq_search(W, X, 128, False, n_grid)
+    torch.cuda.synchronize()
+    t = time.perf_counter()
+    best, a, losses, _ = w4.w4_awq_search(W, X, 128, False, n_grid)
+    ms = (time.perf_counter() - t) * 1e3
+    return {"layer": f"{li.K}x{li.N}, {M} calibration rows, {n_grid} candidates", "ms": round(ms, 2),
+            "alpha": a, "loss_rtn_over_best": round(float(losses[0] / losses[best]), 3)}
+
+
 def time_quantize(w4, torch, projs, iters=3):
     l = max(projs, key=lambda x: x["bytes"])
     li = l["li"]
@@ -476,6 +492,7 @@ def our_arm(args, world, rank, local):
         pf["frac_of_spec_2250"] = pf["tflops"] / 2250.0
         extras["prefill_m4096"] = pf
         extras["quantize_pack"] = time_quantize(w4, torch, projs)
+        extras["awq_search"] = time_awq_search(w4, torch)
         # last: its larger workspace may replace the cached one the graphs above captured
         extras["actorder_decode"] = time_actorder(w4, torch)
     cpu = None

@@ -74,6 +74,10 @@ def lib():
         L.w4a16_gemm_perm.restype = st
         L.w4a16_workspace_bytes_perm.argtypes = [i64, i64, i64, i32]
         L.w4a16_workspace_bytes_perm.restype = sz
+        L.w4_awq_search.argtypes = [vp, st, i64, i64, vp, st, i64, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+        L.w4_awq_search.restype = st
+        L.w4_awq_search_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32]
+        L.w4_awq_search_workspace_bytes.restype = sz
         _lib = L
     return _lib
 
@@ -163,6 +167,32 @@ def w4_actorder_perm(g_idx, group_size, perm=None, stream=None):
         st = lib().w4_actorder_perm(_ptr(g_idx), K, int(group_size), _ptr(perm), _stream_handle(stream, dev))
     _check(st, "w4_actorder_perm")
     return perm
+
+
+def w4_awq_search(W, X, group_size=128, symmetric=False, n_grid=20, stream=None):
+    """AWQ's scale search on the calibration rows X [M,K] for W [N,K] (both CUDA, fp16 or
+    bf16): candidates s = m^a / geomean(m^a), m the mean |X| per channel, a = j / n_grid.
+    Returns (best j, its exponent a, host float64 losses [n_grid], s_best float32 [K] on
+    the device).  Synchronous."""
+    torch = _torch()
+    N, K = W.shape
+    M = X.shape[0]
+    dev = _need_cuda(W, X)
+    s_best = torch.empty(K, dtype=torch.float32, device=dev)
+    losses = (ctypes.c_double * int(n_grid))()
+    best = ctypes.c_int32(-1)
+    with _DeviceGuard(dev):
+        need = lib().w4_awq_search_workspace_bytes(M, N, K, int(group_size), int(bool(symmetric)), int(n_grid))
+        if need == 0:
+            raise ValueError("w4_awq_search: unsupported sizes")
+        ws = workspace_for(dev, need)
+        st = lib().w4_awq_search(_ptr(W), _dtype_code(W.dtype), N, K, _ptr(X), _dtype_code(X.dtype), M,
+                                 int(group_size), int(bool(symmetric)), int(n_grid), _ptr(s_best),
+                                 ctypes.addressof(losses), ctypes.addressof(best), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream_handle(stream, dev))
+    _check(st, "w4_awq_search")
+    import numpy as np
+    return best.value, best.value / n_grid, np.array(losses[:], dtype=np.float64), s_best
 
 
 def w4_quantize_pack(W, s=None, group_size=128, symmetric=False, g_idx=None,

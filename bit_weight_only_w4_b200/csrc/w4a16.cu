@@ -12,6 +12,7 @@
 #include "w4_prefill.cuh"
 #include "w4_quant.cuh"
 #include "w4_actorder.cuh"
+#include "w4_awq.cuh"
 
 namespace {
 
@@ -329,6 +330,36 @@ w4_status launch_prefill(const CUtensorMap& map, const w4p::PrefillParams& p, in
 
 // AWQ scaling + group RTN + packing; with perm (g_idx then NULL) column k of the packed
 // matrix is channel perm[k] and groups are contiguous runs of group_size columns.
+// Workspace of w4_awq_search: per-channel statistics, the candidate scales, the packed
+// candidate, the reference and quantised products, loss partials, the losses, and the
+// GEMM's own workspace last (its zero-filled part stays zero between calls).
+struct AwqLayout {
+    size_t logm, mu, s, s_inv, qw, sc, zr, yref, yq, part, loss, gemm, total;
+    int nblk;
+};
+static AwqLayout awq_layout(int64_t M, int64_t N, int64_t K, int32_t group_size, int32_t symmetric,
+                            int32_t n_grid, size_t gemm_bytes) {
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    const size_t G = (size_t)(K / group_size);
+    const size_t n = (size_t)M * (size_t)N;
+    AwqLayout L;
+    L.nblk = (int)std::min<size_t>(1024, (n + 4095) / 4096);
+    L.logm = 0;
+    L.mu = L.logm + up((size_t)K * 8);
+    L.s = L.mu + 256;
+    L.s_inv = L.s + up((size_t)K * 4);
+    L.qw = L.s_inv + up((size_t)K * 4);
+    L.sc = L.qw + up((size_t)N * K / 2);
+    L.zr = L.sc + up(G * N * 2);
+    L.yref = L.zr + (symmetric ? 0 : up(G * N * 2));
+    L.yq = L.yref + up(n * 4);
+    L.part = L.yq + up(n * 4);
+    L.loss = L.part + up((size_t)L.nblk * 8);
+    L.gemm = L.loss + up((size_t)n_grid * 8);
+    L.total = L.gemm + up(gemm_bytes);
+    return L;
+}
+
 static w4_status quantize_pack_impl(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, const float* s,
                              int32_t group_size, int32_t symmetric, const int32_t* g_idx,
                              const int32_t* perm, uint32_t* qweight, void* scales, void* zeros,
@@ -568,6 +599,85 @@ w4_status w4a16_gemm_perm(const void* X, w4_dtype act_dtype, int64_t M, int64_t 
     // the contiguous-group GEMM on the gathered, already scaled activations
     return gemm_impl(xp, act_dtype, M, N, K, qweight, scales, zeros, nullptr, nullptr, group_size, nullptr, Y,
                      out_dtype, workspace, workspace_bytes, stream);
+}
+
+size_t w4_awq_search_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size,
+                                     int32_t symmetric, int32_t n_grid) {
+    if (M <= 0 || M > (1 << 20) || n_grid <= 0 || n_grid > 1024) return 0;
+    if (check_layer_shape(N, K, group_size) != W4_OK) return 0;
+    const size_t gemm = w4a16_workspace_bytes(M, N, K, group_size);
+    if (gemm == 0) return 0;
+    return awq_layout(M, N, K, group_size, symmetric, n_grid, gemm).total;
+}
+
+w4_status w4_awq_search(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, const void* X,
+                        w4_dtype x_dtype, int64_t M, int32_t group_size, int32_t symmetric,
+                        int32_t n_grid, float* s_best, double* losses, int32_t* best,
+                        void* workspace, size_t workspace_bytes, w4_stream_t stream) {
+    if (!W || !X || !s_best || !losses || !best || !workspace) return W4_ERR_INVALID_ARG;
+    if ((w_dtype != W4_F16 && w_dtype != W4_BF16) || (x_dtype != W4_F16 && x_dtype != W4_BF16))
+        return W4_ERR_INVALID_ARG;
+    if (symmetric != 0 && symmetric != 1) return W4_ERR_INVALID_ARG;
+    if (M <= 0 || M > (1 << 20) || n_grid <= 0 || n_grid > 1024) return W4_ERR_INVALID_ARG;
+    w4_status st = check_layer_shape(N, K, group_size);
+    if (st != W4_OK) return st;
+    if (K / group_size > kQuantMaxGroups) return W4_ERR_UNSUPPORTED;
+    if (!aligned(W, 16) || !aligned(X, 16) || !aligned(s_best, 4) || !aligned(workspace, 256))
+        return W4_ERR_INVALID_ARG;
+    const size_t gemm_bytes = w4a16_workspace_bytes(M, N, K, group_size);
+    if (gemm_bytes == 0) return W4_ERR_CUDA;
+    const AwqLayout L = awq_layout(M, N, K, group_size, symmetric, n_grid, gemm_bytes);
+    if (workspace_bytes < L.total) return W4_ERR_INVALID_ARG;
+    cudaStream_t strm = as_stream(stream);
+    unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+    double* logm = reinterpret_cast<double*>(ws + L.logm);
+    double* mu = reinterpret_cast<double*>(ws + L.mu);
+    float* s = reinterpret_cast<float*>(ws + L.s);
+    float* s_inv = reinterpret_cast<float*>(ws + L.s_inv);
+    uint32_t* qw = reinterpret_cast<uint32_t*>(ws + L.qw);
+    void* sc = ws + L.sc;
+    void* zr = symmetric ? nullptr : (void*)(ws + L.zr);
+    float* yref = reinterpret_cast<float*>(ws + L.yref);
+    float* yq = reinterpret_cast<float*>(ws + L.yq);
+    double* part = reinterpret_cast<double*>(ws + L.part);
+    double* loss = reinterpret_cast<double*>(ws + L.loss);
+    const bool xb = x_dtype == W4_BF16, wb = w_dtype == W4_BF16;
+    const unsigned kb = (unsigned)((K + 255) / 256);
+    // activation statistics and the unquantised reference product, once
+    if (xb) w4s::col_logmean_kernel<true><<<kb, 256, 0, strm>>>(X, (int)M, (int)K, logm);
+    else w4s::col_logmean_kernel<false><<<kb, 256, 0, strm>>>(X, (int)M, (int)K, logm);
+    w4s::mean_kernel<<<1, 32, 0, strm>>>(logm, (int)K, mu);
+    const dim3 rb(w4s::kT, w4s::kT), rg((unsigned)((N + w4s::kT - 1) / w4s::kT), (unsigned)((M + w4s::kT - 1) / w4s::kT));
+    if (xb && wb) w4s::ref_gemm_kernel<true, true><<<rg, rb, 0, strm>>>(X, W, (int)M, (int)N, (int)K, yref);
+    else if (xb) w4s::ref_gemm_kernel<true, false><<<rg, rb, 0, strm>>>(X, W, (int)M, (int)N, (int)K, yref);
+    else if (wb) w4s::ref_gemm_kernel<false, true><<<rg, rb, 0, strm>>>(X, W, (int)M, (int)N, (int)K, yref);
+    else w4s::ref_gemm_kernel<false, false><<<rg, rb, 0, strm>>>(X, W, (int)M, (int)N, (int)K, yref);
+    if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+    const size_t n = (size_t)M * (size_t)N;
+    const size_t chunk = (n + L.nblk - 1) / L.nblk;
+    for (int j = 0; j < n_grid; ++j) {
+        const double a = (double)j / (double)n_grid;
+        w4s::awq_scale_kernel<<<kb, 256, 0, strm>>>(logm, mu, a, (int)K, s, s_inv);
+        if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+        st = quantize_pack_impl(W, w_dtype, N, K, s, group_size, symmetric, nullptr, nullptr, qw, sc, zr, stream);
+        if (st != W4_OK) return st;
+        st = gemm_impl(X, x_dtype, M, N, K, qw, sc, zr, nullptr, nullptr, group_size, s_inv, yq, W4_F32,
+                       ws + L.gemm, workspace_bytes - L.gemm, stream);
+        if (st != W4_OK) return st;
+        w4s::sqdiff_partial_kernel<<<(unsigned)L.nblk, w4s::kLossThreads, 0, strm>>>(yref, yq, n, chunk, part);
+        w4s::sum_kernel<<<1, 32, 0, strm>>>(part, L.nblk, loss + j);
+        if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+    }
+    if (cudaMemcpyAsync(losses, loss, (size_t)n_grid * sizeof(double), cudaMemcpyDeviceToHost, strm) != cudaSuccess ||
+        cudaStreamSynchronize(strm) != cudaSuccess)
+        return W4_ERR_CUDA;
+    int b = 0;
+    for (int j = 1; j < n_grid; ++j)
+        if (losses[j] < losses[b]) b = j;   // the first of equal losses
+    *best = b;
+    w4s::awq_scale_kernel<<<kb, 256, 0, strm>>>(logm, mu, (double)b / (double)n_grid, (int)K, s_best, s_inv);
+    if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(strm) != cudaSuccess) return W4_ERR_CUDA;
+    return W4_OK;
 }
 
 w4_status w4_unpack_canonical(const uint32_t* qweight, int64_t N, int64_t K,

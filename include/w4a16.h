@@ -204,6 +204,38 @@ w4_status w4a16_gemm_perm(const void* X, w4_dtype act_dtype, int64_t M, int64_t 
 size_t w4a16_workspace_bytes_perm(int64_t M, int64_t N, int64_t K, int32_t group_size);
 
 /*
+ * w4_awq_search -- AWQ's per-channel scale search on a calibration batch ("Quantization
+ * Paradigms for Edge Inference: AWQ, GPTQ, and FP8 Matrix Cores", sec. 3: s minimises
+ * L(s) = || W X - Q(W diag(s)) diag(s)^-1 X ||_2, found from activation magnitudes).
+ * Candidates: with m[k] = mean_i |X[i,k]| and a_j = j / n_grid (j = 0 .. n_grid-1),
+ *   s_j[k] = fp32(exp(a_j (log m[k] - mean_k log m)))     (m^a_j over its geometric mean;
+ *                                                          s_0 = 1, plain RTN),
+ *   L_j    = sum_{i,n} (Yref[i,n] - Yq_j[i,n])^2          (fp64 sum of fp32 terms),
+ * with Yref = X W^T in fp32 and Yq_j = w4a16_gemm(X, w4_quantize_pack(W, s_j), s_inv =
+ * 1/s_j) in fp32.  Returns the first j of the smallest L_j.
+ *
+ *   W          device [N,K] row-major fp16/bf16 (w_dtype); X device [M,K] calibration rows
+ *              (x_dtype); 1 <= M <= 2^20; group_size, symmetric as for w4_quantize_pack
+ *   n_grid     1..1024 candidates
+ *   s_best     device fp32 [K] output: the chosen s (pass it to w4_quantize_pack, and its
+ *              reciprocal as the GEMM's s_inv)
+ *   losses     HOST fp64 [n_grid] output: L_j
+ *   best       HOST int32 output: the chosen j
+ *   workspace  device scratch of w4_awq_search_workspace_bytes(...) bytes, 256-byte
+ *              aligned, zero-filled before its first use (it holds a w4a16_gemm workspace)
+ * Offline and synchronous: the call waits for the stream before it returns.  Device-side
+ * errors of the kernels it runs are reported by w4_check_device_error().
+ */
+w4_status w4_awq_search(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, const void* X,
+                        w4_dtype x_dtype, int64_t M, int32_t group_size, int32_t symmetric,
+                        int32_t n_grid, float* s_best, double* losses, int32_t* best,
+                        void* workspace, size_t workspace_bytes, w4_stream_t stream);
+
+/* Bytes of workspace w4_awq_search needs (0 on invalid sizes). */
+size_t w4_awq_search_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size,
+                                     int32_t symmetric, int32_t n_grid);
+
+/*
  * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 32 (M <= 64 where the scratch fits)
  * without a caller-supplied workspace.  The pages have no counterpart to this call; it
  * exists for callers that cannot allocate device memory where they run the GEMM, such as

@@ -223,3 +223,37 @@ def reference_y(X_bits, s_inv, q, scales, zeros, group_size, g_idx=None, x_is_bf
     Xp = awq_scale_acts(X_bits, s_inv, x_is_bf16)
     What = dequant(q, scales, zeros, group_size, g_idx)
     return gemm_f32(Xp, What, rows)
+
+
+# ---- AWQ scale search ----------------------------------------------------------------
+def awq_search(W_bits, X_bits, group_size, symmetric=False, n_grid=20, w_is_bf16=False, x_is_bf16=False):
+    """AWQ's per-channel scale search ("Quantization Paradigms for Edge Inference: AWQ, GPTQ,
+    and FP8 Matrix Cores", sec. 3, eq. 2: s minimises || W X - Q(W diag(s)) diag(s)^-1 X ||_2,
+    s found from activation magnitudes), over the candidates
+        s_j = fp32(exp(a_j (log m - mean(log m)))),  m[k] = mean_i |X[i,k]|,  a_j = j / n_grid,
+    in plain steps: m and its logarithms in fp64; per candidate the oracle's quantiser on
+    W diag(s_j), X' = X s_j^-1 rounded to the activation type (as the GEMM does), the fp32
+    product X' What^T, and the squared error against the fp32 product X W^T summed in fp64.
+    Returns (first index of the smallest loss, losses fp64 [n_grid], s of that index)."""
+    X_bits = bits16(X_bits)
+    W_bits = bits16(W_bits)
+    M, K = X_bits.shape
+    Xf = bf16_to_f32(X_bits) if x_is_bf16 else f16_to_f32(X_bits)
+    Wf = bf16_to_f32(W_bits) if w_is_bf16 else f16_to_f32(W_bits)
+    m = np.abs(Xf.astype(np.float64)).sum(axis=0) / M
+    logm = np.log(np.maximum(m, 1e-30))
+    mu = logm.mean()
+    Yref = gemm_f32(Xf, Wf).astype(np.float64)
+    losses = np.empty(n_grid, np.float64)
+    cand = []
+    for j in range(n_grid):
+        s = np.exp((j / n_grid) * (logm - mu)).astype(np.float32)
+        s_inv = (np.float32(1) / s).astype(np.float32)
+        q, sc, zr = quantize_weights(W_bits, s, group_size, symmetric, is_bf16=w_is_bf16)
+        Xp = awq_scale_acts(X_bits, s_inv, x_is_bf16)
+        Xp = bf16_to_f32(f32_to_bf16(Xp)) if x_is_bf16 else f16_to_f32(f32_to_f16(Xp))
+        Yq = gemm_f32(Xp, dequant(q, sc, zr, group_size)).astype(np.float64)
+        losses[j] = ((Yref - Yq) ** 2).sum()
+        cand.append(s)
+    best = int(np.argmin(losses))
+    return best, losses, cand[best]
