@@ -185,7 +185,9 @@ def w4_awq_search(W, X, group_size=128, symmetric=False, n_grid=20, stream=None)
         need = lib().w4_awq_search_workspace_bytes(M, N, K, int(group_size), int(bool(symmetric)), int(n_grid))
         if need == 0:
             raise ValueError("w4_awq_search: unsupported sizes")
-        ws = workspace_for(dev, need)
+        # a buffer of its own: the search writes over the front of its workspace, where the
+        # cached GEMM workspace keeps the zero-filled split-K slots
+        ws = torch.zeros(need, dtype=torch.uint8, device=dev)
         st = lib().w4_awq_search(_ptr(W), _dtype_code(W.dtype), N, K, _ptr(X), _dtype_code(X.dtype), M,
                                  int(group_size), int(bool(symmetric)), int(n_grid), _ptr(s_best),
                                  ctypes.addressof(losses), ctypes.addressof(best), _ptr(ws),

@@ -61,3 +61,21 @@ def test_search_equal_magnitudes_gives_unit_scales():
     assert best == 0
     assert np.all(s == np.float32(1))
     assert np.all(losses == losses[0])
+
+
+def test_gemm_after_search_is_unaffected():
+    """The search uses a workspace of its own: a decode GEMM through the binding's cached
+    workspace right after it still matches the oracle."""
+    skip_without_gpu()
+    import torch
+    from tests.gpu_util import check_y, dev, to_f64
+    rng = np.random.default_rng(21)
+    X, W = layer(rng, 16, 256, 512)
+    run(X, W, 128, False, 3)
+    q, sc, zr = oracle.quantize_weights(W, None, 128, False)
+    Xd = dev_bits(X[:3], torch.float16)
+    Y = w4.w4a16_gemm(Xd, dev(oracle.pack_device(q).view(np.int32)), dev_bits(sc, torch.float16),
+                      dev_bits(zr, torch.float16), 128)
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    check_y(to_f64(Y), oracle.reference_y(X[:3], None, q, sc, zr, 128), "fp16")
