@@ -399,32 +399,43 @@ def time_quantize(w4, torch, projs, iters=3):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def cpu_oracle_sample(target_s=12.0, rows_per_layer=256):
-    """Time the oracle's online path (X*s_inv, dequantise, fp32 product) for M=1 on a
-    seeded sample of output rows of every decode layer, each layer's product repeated until
-    about target_s / 4 seconds of CPU work; returns (GB/s of effective weight bytes
-    processed, seconds, description)."""
+def oracle_sample(rows_per_layer=256):
+    """The seeded sample the oracle is timed on: M=1 inputs and rows_per_layer seeded output
+    rows of every decode layer, quantised by the oracle (weights regenerated only for those
+    rows).  Prepared once; not timed."""
     import oracle
     wl = workloads.workload(DECODE_CFG)
     rng = np.random.default_rng(0)
-    total_bytes, total_s, n_rows, reps = 0, 0.0, 0, []
+    sample = []
     for i, L in enumerate(wl.layers):
         li = workloads.make_layer(wl, i, M=1, with_weights=False)
-        # a fresh seeded sample of rows (weights regenerated only for those rows)
         ns = np.sort(rng.choice(L.N, size=rows_per_layer, replace=False))
         Wr = workloads.gen_weights(L.N, L.K, 0, wl.config_id, i)[ns]
         q, sc, zr = oracle.quantize_weights(Wr.view(np.uint16), li.s, 128)
+        by = workloads.effective_weight_bytes(rows_per_layer, L.K, 128, False, False)
+        sample.append((li, q, sc, zr, by))
+    return sample
+
+
+def cpu_oracle_sample(target_s=12.0, sample=None, rows_per_layer=256):
+    """Time the oracle's online path (X*s_inv, dequantise, fp32 product) on the prepared
+    sample, each layer's product repeated until about target_s / 4 seconds of CPU work;
+    returns (GB/s of effective weight bytes processed, seconds, description)."""
+    import oracle
+    sample = sample or oracle_sample(rows_per_layer)
+    total_bytes, total_s, reps = 0, 0.0, []
+    for li, q, sc, zr, by in sample:
         layer_s, r = 0.0, 0
-        while r == 0 or layer_s < target_s / len(wl.layers):
+        while r == 0 or layer_s < target_s / len(sample):
             t0 = time.perf_counter()
             oracle.reference_y(li.X, li.s_inv, q, sc, zr, 128)
             layer_s += time.perf_counter() - t0
             r += 1
         total_s += layer_s
-        total_bytes += r * workloads.effective_weight_bytes(rows_per_layer, L.K, 128, False, False)
-        n_rows += rows_per_layer
+        total_bytes += r * by
         reps.append(r)
-    desc = (f"M=1, {rows_per_layer} seeded output rows of each of the 4 layers ({n_rows} rows), "
+    rows = sample[0][1].shape[0]
+    desc = (f"M=1, {rows} seeded output rows of each of the 4 layers ({rows * len(sample)} rows), "
             f"each layer's product repeated {reps} times ({total_bytes / 1e6:.0f} MB of effective "
             f"weights in {total_s:.1f} s), single thread")
     return total_bytes / total_s / 1e9, total_s, desc
@@ -435,14 +446,15 @@ def reference_arm(args, world, rank):
         return
     import oracle
     oracle.lib()
+    sample = oracle_sample()
     vals = []
     desc = ""
     # each step a bounded sample, so that the whole run takes about two minutes
     per_step = max(0.5, min(12.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_oracle_sample(target_s=per_step)
+        cpu_oracle_sample(target_s=per_step, sample=sample)
     for _ in range(args.steps):
-        v, s, desc = cpu_oracle_sample(target_s=per_step)
+        v, s, desc = cpu_oracle_sample(target_s=per_step, sample=sample)
         vals.append(v)
     value = statistics.median(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
