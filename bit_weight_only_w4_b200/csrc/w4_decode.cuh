@@ -15,25 +15,28 @@
 //   unit      = 2 column blocks (128 input channels) of one band; all units of the layer
 //               are split into equal contiguous ranges, one per CTA (stream-K), so every
 //               SM streams the same number of bytes whatever N and K are;
-//   stage     = up to 2 units of one band: the codes (one bulk copy), the activations (one
-//               3-D TMA box of 4 column blocks x 8*NT token rows, 128B swizzle, rows >= M
-//               zero-filled), the s_inv slice and the group rows of scales and zero points;
-//   CTA       = 1 producer warp (its lanes issue the copies of a stage in parallel), XW
-//               activation warps and 16 MMA warps in two groups that take alternate
-//               stages; one CTA per SM, its ring filling the SM's shared memory, so every
-//               SM holds exactly one CTA of a GEMM even when the next GEMM's CTAs start
-//               early under programmatic dependent launch;
-//   activation= per stage, the activation warps write X' = X * s_inv (when given) to a
-//   warps       buffer of their own, the activation sums S and the fold constants of every
-//               staged (group, row);
+//   stage     = up to 4 units of one band with one token tile (2 with more): the codes
+//               (one bulk copy) and the group rows of scales and zero points (2-D boxes);
+//               staged activations add a 3-D TMA box of column blocks x 8*NT token rows
+//               (128B swizzle, rows >= M zero-filled) and the s_inv slice;
+//   CTA       = 1 producer warp (lane 0 issues a stage's copies), XW activation warps and
+//               16 MMA warps in two groups that take alternate stages (8 in one group at
+//               8 token tiles); one CTA per SM, its ring filling the SM's shared memory,
+//               so every SM holds exactly one CTA of a GEMM even when the next GEMM's CTAs
+//               start early under programmatic dependent launch;
+//   activations= with one token tile and a small M*K, X' = X * s_inv and its sums over 32,
+//               64 and 128 channels are prepared once per CTA and stay resident (with
+//               act-order weights packed in permuted order, gathered through perm);
+//               otherwise the activation warps prepare each stage's X' and sums;
 //   zero point= the MMA multiplies the biased codes o + m*q (o + m*q is what the AND/OR
 //               unpack yields; no subtraction per weight) and the per-group fold removes
 //               the bias and the zero point with the activation sums S = sum_k X'[m,k] of
 //               the group: sum_k (q-z) X' = (c - (o + m*z) S) / m, in fp32;
 //   fix-up    = a band split between CTAs is completed by the CTA holding its last unit;
-//               the others process their share first and publish fp32 partials as
-//               {value, flag} words, so the finishing CTA only reads them (deterministic
-//               order, no atomics).
+//               a CTA processes its contributor part first (publishing fp32 partials as
+//               {value, flag} words), its whole bands next and the completing part last,
+//               after which all MMA threads sum the contributors' shares in CTA order
+//               (deterministic, no atomics).
 #pragma once
 #include "w4_common.cuh"
 
@@ -567,11 +570,10 @@ W4_DEV void consume_gidx(const StageView& v, const DecodeParams& p, const Lane& 
 }
 
 // ---------------------------------------------------------------- activation warps
-// Per stage: X' = X * s_inv rounded to the activation type (into the X' buffer, when s_inv
-// is given; otherwise the MMA warps read the tensor box itself), the sums of X' over 32,
-// 64 and 128 consecutive channels per token, and the fold constants {sc', bz} of every
-// staged (group row, band row).  The stage's channels form 8-channel chunks (column block
-// c/8, 16-byte chunk c%8); each warp pass covers 32 consecutive chunks of one token.
+// Per stage: X' = X * s_inv rounded to the activation type (a plain copy without s_inv)
+// into the stage's X' buffer, which the MMA warps read, and the sums of X' over 32, 64 and
+// 128 consecutive channels per token.  The stage's channels form 8-channel chunks (column
+// block c/8, 16-byte chunk c%8); each warp pass covers 32 consecutive chunks of one token.
 template <int NT, bool BF16, bool GIDX>
 W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw, int lane) {
     using C = Cfg<NT>;
