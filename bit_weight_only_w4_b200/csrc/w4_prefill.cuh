@@ -7,21 +7,22 @@
 // tensor cores and the next tiles are staged while the current ones are multiplied
 // ("Kernel Execution: Marlin vs. ExLlamaV2 INT4 GEMM Micro-Architecture", items 1-3).
 //
-// One CTA computes a 128 (output rows) x 128 (tokens) tile of Y^T = What * X'^T:
+// Persistent CTAs (one per SM) walk tiles of 256 output rows x 128 tokens of
+// Y^T = What * X'^T (CTA t takes tiles t, t + gridDim.x, ...), 16 warps in four warpgroups:
 //   warp 0      TMA: activation tile (2-D tensor map, 128B swizzle) + packed weight tiles
 //               (1-D bulk copies) + zero-point rows into a 5-slot load ring;
-//   warp 1      allocates tensor memory and issues tcgen05.mma (one thread): A = the
-//               dequantised weights (128 x 64 per stage, K-major, 128B swizzle, shared
-//               memory), B = the activations, D = fp32 in tensor memory;
-//   warps 2-5   unpack the packed tile into exact integers q - z (fp16/bf16) in the
-//               swizzled A layout, into a 2-slot ring of its own (the load ring runs
+//   warp 1      allocates tensor memory and issues tcgen05.mma (one elected lane): A = the
+//               dequantised weights of one 128-row half (K-major, 128B swizzle, shared
+//               memory), B = the activations, D = fp32 in tensor memory; two 128 x 128 x 16
+//               MMAs per 16-deep step, one per half;
+//   warps 2-7   unpack the packed tiles into exact integers q - z (fp16/bf16) in the
+//               swizzled A layout, into a 2-slot ring of their own (the load ring runs
 //               further ahead than the dequantised tiles need to);
-//   warps 6-9   epilogue: after each quantisation group the MMA warp hands over that
+//   warps 8-15  epilogue: after each quantisation group the MMA warp hands over that
 //               group's fp32 partial tile (two tensor-memory buffers, ping-pong); each
-//               thread owns one output row, multiplies the partial by the row's group
-//               scale and adds it to register accumulators; at the end it stores Y.
-// With act-order g_idx the scale is folded into fp16 weights instead and the whole K
-// accumulates in one tensor-memory buffer.
+//               thread owns one output row of one half, multiplies the partial by the
+//               row's group scale and adds it to register accumulators; at the tile's end
+//               it stores Y through a staging buffer.
 #pragma once
 #include "w4_common.cuh"
 
