@@ -23,6 +23,8 @@
 //               thread owns one output row of one half, multiplies the partial by the
 //               row's group scale and adds it to register accumulators; at the tile's end
 //               it stores Y through a staging buffer.
+// With act-order g_idx the scale is folded into fp16 weights instead and the whole K
+// accumulates in one tensor-memory buffer.
 #pragma once
 #include "w4_common.cuh"
 
