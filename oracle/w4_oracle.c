@@ -24,7 +24,7 @@
  *          Micro-Architecture", item 3: two 4-bit weights share one byte and are
  *          recovered with shift and AND.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   - W is [N,K] row-major (out x in); Y = X' * What^T is [M,N].
  *   - group of channel k: k / group_size, or g_idx[k] when a g_idx array is given.
  *   - asymmetric: sc = fp16(max((max-min)/15, 2^-14)), z = clamp(rint(-min/sc),0,15);
