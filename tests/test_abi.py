@@ -120,3 +120,36 @@ def test_actorder_entry_points_reject_bad_arguments(L):
     assert g(v(16), 0, 0, 128, 128, None, None, None, None, 128, None, None, 0, None, 0, None) == w4.W4_OK
     assert L.w4a16_workspace_bytes_perm(1, 8, 128, 128) == 0
     assert L.w4a16_workspace_bytes_perm(0, 128, 128, 128) == 0
+
+
+def test_awq_search_rejects_bad_arguments(L):
+    """Every case below is refused by the host checks, before any CUDA call."""
+    v = ctypes.c_void_p
+    ok = dict(W=v(256), wd=0, N=128, K=256, X=v(256), xd=0, M=8, g=128, sym=0, n_grid=4, s=v(256),
+              losses=v(256), best=v(256), ws=v(256), wsb=1 << 30)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.w4_awq_search(a["W"], a["wd"], a["N"], a["K"], a["X"], a["xd"], a["M"], a["g"], a["sym"],
+                               a["n_grid"], a["s"], a["losses"], a["best"], a["ws"], a["wsb"], None)
+
+    for bad in ("W", "X", "s", "losses", "best", "ws"):
+        assert call(**{bad: None}) == w4.W4_ERR_INVALID_ARG, bad
+    assert call(wd=2) == w4.W4_ERR_INVALID_ARG           # fp32 weights
+    assert call(xd=7) == w4.W4_ERR_INVALID_ARG
+    assert call(sym=2) == w4.W4_ERR_INVALID_ARG
+    for M in (0, -1, (1 << 20) + 1):
+        assert call(M=M) == w4.W4_ERR_INVALID_ARG, M
+    for n_grid in (0, 1025):
+        assert call(n_grid=n_grid) == w4.W4_ERR_INVALID_ARG, n_grid
+    assert call(K=200) == w4.W4_ERR_INVALID_ARG          # K % group_size
+    assert call(N=8) == w4.W4_ERR_UNSUPPORTED            # N % 16
+    assert call(W=v(258)) == w4.W4_ERR_INVALID_ARG       # 16-byte alignment
+    assert call(X=v(264)) == w4.W4_ERR_INVALID_ARG
+    assert call(s=v(258)) == w4.W4_ERR_INVALID_ARG
+    assert call(ws=v(272)) == w4.W4_ERR_INVALID_ARG      # 256-byte alignment
+    ws = L.w4_awq_search_workspace_bytes
+    assert ws(0, 128, 256, 128, 0, 4) == 0
+    assert ws(8, 128, 256, 128, 0, 0) == 0
+    assert ws(8, 128, 256, 128, 0, 1025) == 0
+    assert ws(8, 8, 256, 128, 0, 4) == 0
