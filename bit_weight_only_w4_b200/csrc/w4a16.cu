@@ -20,6 +20,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kDecodeMaxM = 64;
 constexpr int kQuantMaxGroups = 1536;
 constexpr int64_t kMaxBands = 8192;                       // N <= 1,048,576 (fix-up counters)
+constexpr int64_t kAwqMaxRows = 1 << 19;                  // calibration rows (the reference product's grid.y)
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -62,7 +63,7 @@ bool ensure_smem(Kernel k, int bytes, std::once_flag (&flags)[kMaxDevices], int 
         ok = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
              cudaSuccess;
     });
-    // a failed first attempt is retried on the next call by the launch itself failing
+    // a failure is reported to the first call only; later launches then fail on their own
     return ok;
 }
 
@@ -188,10 +189,11 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     // X' resident (one token tile, small M*K): X' and its sums are prepared once per CTA;
     // the ring then carries only codes and group metadata.
     auto up = [](int v, int a) { return (v + a - 1) / a * a; };
-    const int sstride_res = std::max(2, (int)((p.M + 1) / 2 * 2));
-    const int res_x = up(p.M * p.K * 2, 128);
-    const int res_s = up((p.K / 32 + p.K / 64 + p.K / 128) * sstride_res * 4, 128);
     p.xres = (NT == 1 && !GIDX && decode_x_resident(p.M, p.K)) ? 1 : 0;
+    // sizes of the resident X' and sums (decode_x_resident bounds them to 80 KB together)
+    const int sstride_res = std::max(2, (int)((p.M + 1) / 2 * 2));
+    const int res_x = p.xres ? up(p.M * p.K * 2, 128) : 0;
+    const int res_s = p.xres ? up((p.K / 32 + p.K / 64 + p.K / 128) * sstride_res * 4, 128) : 0;
     if (PERM != (p.perm != nullptr) || (PERM && !p.xres))   // the gather is part of the resident X'
         return W4_ERR_UNSUPPORTED;
     p.sstride = p.xres ? sstride_res : C::mpad;
@@ -503,7 +505,7 @@ static w4_status gemm_impl(const void* X, w4_dtype act_dtype, int64_t M, int64_t
     if (!prefill) {
         w4d::DecodeParams p;
         std::memset(&p, 0, sizeof(p));
-            p.qw = qweight;
+        p.qw = qweight;
         p.scales = reinterpret_cast<const __half*>(scales);
         p.zeros = reinterpret_cast<const __half*>(zeros);
         p.g_idx = g_idx;
@@ -603,7 +605,7 @@ w4_status w4a16_gemm_perm(const void* X, w4_dtype act_dtype, int64_t M, int64_t 
 
 size_t w4_awq_search_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size,
                                      int32_t symmetric, int32_t n_grid) {
-    if (M <= 0 || M > (1 << 20) || n_grid <= 0 || n_grid > 1024) return 0;
+    if (M <= 0 || M > kAwqMaxRows || n_grid <= 0 || n_grid > 1024) return 0;
     if (check_layer_shape(N, K, group_size) != W4_OK) return 0;
     const size_t gemm = w4a16_workspace_bytes(M, N, K, group_size);
     if (gemm == 0) return 0;
@@ -618,7 +620,7 @@ w4_status w4_awq_search(const void* W, w4_dtype w_dtype, int64_t N, int64_t K, c
     if ((w_dtype != W4_F16 && w_dtype != W4_BF16) || (x_dtype != W4_F16 && x_dtype != W4_BF16))
         return W4_ERR_INVALID_ARG;
     if (symmetric != 0 && symmetric != 1) return W4_ERR_INVALID_ARG;
-    if (M <= 0 || M > (1 << 20) || n_grid <= 0 || n_grid > 1024) return W4_ERR_INVALID_ARG;
+    if (M <= 0 || M > kAwqMaxRows || n_grid <= 0 || n_grid > 1024) return W4_ERR_INVALID_ARG;
     w4_status st = check_layer_shape(N, K, group_size);
     if (st != W4_OK) return st;
     if (K / group_size > kQuantMaxGroups) return W4_ERR_UNSUPPORTED;

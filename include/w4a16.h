@@ -215,7 +215,7 @@ size_t w4a16_workspace_bytes_perm(int64_t M, int64_t N, int64_t K, int32_t group
  * 1/s_j) in fp32.  Returns the first j of the smallest L_j.
  *
  *   W          device [N,K] row-major fp16/bf16 (w_dtype); X device [M,K] calibration rows
- *              (x_dtype); 1 <= M <= 2^20; group_size, symmetric as for w4_quantize_pack
+ *              (x_dtype); 1 <= M <= 2^19; group_size, symmetric as for w4_quantize_pack
  *   n_grid     1..1024 candidates
  *   s_best     device fp32 [K] output: the chosen s (pass it to w4_quantize_pack, and its
  *              reciprocal as the GEMM's s_inv)

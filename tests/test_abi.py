@@ -138,7 +138,7 @@ def test_awq_search_rejects_bad_arguments(L):
     assert call(wd=2) == w4.W4_ERR_INVALID_ARG           # fp32 weights
     assert call(xd=7) == w4.W4_ERR_INVALID_ARG
     assert call(sym=2) == w4.W4_ERR_INVALID_ARG
-    for M in (0, -1, (1 << 20) + 1):
+    for M in (0, -1, (1 << 19) + 1):
         assert call(M=M) == w4.W4_ERR_INVALID_ARG, M
     for n_grid in (0, 1025):
         assert call(n_grid=n_grid) == w4.W4_ERR_INVALID_ARG, n_grid
