@@ -130,6 +130,41 @@ def _need_cuda(*tensors):
     return dev
 
 
+def _expect(t, name, dtypes, shape=None, numel=None):
+    """Refuse a tensor of the wrong dtype or size before its pointer reaches the library,
+    which sees only the pointer and would read past a short buffer."""
+    if t is None:
+        return
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must be {' or '.join(str(d) for d in dtypes)}, not {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} must hold {numel} elements, not {t.numel()}")
+
+
+def _matrix(t, name):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be a matrix, not of shape {tuple(t.shape)}")
+    return t.shape
+
+
+def _groups(K, group_size):
+    if group_size <= 0 or K % group_size != 0:
+        raise ValueError(f"group_size {group_size} must divide K = {K}")
+    return K // group_size
+
+
+def _f16s():
+    torch = _torch()
+    return (torch.float16, torch.bfloat16)
+
+
+def _words():
+    torch = _torch()
+    return (torch.int32, torch.uint32)
+
+
 class _DeviceGuard:
     def __init__(self, device):
         self.device = device
@@ -157,10 +192,12 @@ def w4_actorder_perm(g_idx, group_size, perm=None, stream=None):
     act-order weights with contiguous groups (every group must hold group_size channels;
     otherwise w4_check_device_error() reports W4_ERR_DEVICE_ARG)."""
     torch = _torch()
+    if g_idx.dim() != 1:
+        raise ValueError("g_idx must be a vector")
     K = g_idx.shape[0]
+    _expect(g_idx, "g_idx", (torch.int32,))
+    _expect(perm, "perm", (torch.int32,), numel=K)
     dev = _need_cuda(g_idx, perm)
-    if g_idx.dtype != torch.int32:
-        raise TypeError("g_idx must be int32")
     if perm is None:
         perm = torch.empty(K, dtype=torch.int32, device=dev)
     with _DeviceGuard(dev):
@@ -175,8 +212,12 @@ def w4_awq_search(W, X, group_size=128, symmetric=False, n_grid=20, stream=None)
     Returns (best j, its exponent a, host float64 losses [n_grid], s_best float32 [K] on
     the device).  Synchronous."""
     torch = _torch()
-    N, K = W.shape
-    M = X.shape[0]
+    N, K = _matrix(W, "W")
+    M, KX = _matrix(X, "X")
+    if KX != K:
+        raise ValueError(f"X has {KX} channels, W has {K}")
+    _expect(W, "W", _f16s())
+    _expect(X, "X", _f16s())
     dev = _need_cuda(W, X)
     s_best = torch.empty(K, dtype=torch.float32, device=dev)
     losses = (ctypes.c_double * int(n_grid))()
@@ -205,10 +246,17 @@ def w4_quantize_pack(W, s=None, group_size=128, symmetric=False, g_idx=None,
     channel perm[k] and groups are contiguous.  Returns (qweight uint32-as-int32 [N*K/8]
     device layout, scales fp16 [G,N], zeros fp16 [G,N] or None when symmetric)."""
     torch = _torch()
-    N, K = W.shape
-    G = K // group_size
+    N, K = _matrix(W, "W")
+    G = _groups(K, group_size)
     if perm is not None and g_idx is not None:
         raise ValueError("pass g_idx or perm, not both")
+    _expect(W, "W", _f16s())
+    _expect(s, "s", (torch.float32,), numel=K)
+    _expect(g_idx, "g_idx", (torch.int32,), numel=K)
+    _expect(perm, "perm", (torch.int32,), numel=K)
+    _expect(qweight, "qweight", _words(), numel=N * K // 8)
+    _expect(scales, "scales", (torch.float16,), shape=(G, N))
+    _expect(zeros, "zeros", (torch.float16,), shape=(G, N))
     dev = _need_cuda(W, s, g_idx, qweight, scales, zeros, perm)
     if qweight is None:
         qweight = torch.empty(N * K // 8, dtype=torch.int32, device=dev)
@@ -216,12 +264,6 @@ def w4_quantize_pack(W, s=None, group_size=128, symmetric=False, g_idx=None,
         scales = torch.empty(G, N, dtype=torch.float16, device=dev)
     if zeros is None and not symmetric:
         zeros = torch.empty(G, N, dtype=torch.float16, device=dev)
-    if s is not None and s.dtype != torch.float32:
-        raise TypeError("s must be float32")
-    if g_idx is not None and g_idx.dtype != torch.int32:
-        raise TypeError("g_idx must be int32")
-    if perm is not None and perm.dtype != torch.int32:
-        raise TypeError("perm must be int32")
     with _DeviceGuard(dev):
         if perm is not None:
             st = lib().w4_quantize_pack_perm(_ptr(W), _dtype_code(W.dtype), N, K, _ptr(s), int(group_size),
@@ -252,6 +294,22 @@ def workspace_for(device, nbytes):
         return buf
 
 
+def _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y):
+    """Shapes and dtypes of a GEMM call; returns (M, K, N), N taken from the scales."""
+    torch = _torch()
+    M, K = _matrix(X, "X")
+    G = _groups(K, group_size)
+    N = _matrix(scales, "scales")[1]
+    _expect(X, "X", _f16s())
+    _expect(qweight, "qweight", _words(), numel=N * K // 8)
+    _expect(scales, "scales", (torch.float16,), shape=(G, N))
+    _expect(zeros, "zeros", (torch.float16,), shape=(G, N))
+    _expect(g_idx, "g_idx", (torch.int32,), numel=K)
+    _expect(s_inv, "s_inv", (torch.float32,), numel=K)
+    _expect(Y, "Y", _f16s() + (torch.float32,), shape=(M, N))
+    return M, K, N
+
+
 def w4a16_gemm(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None,
                out_dtype=None, Y=None, workspace=None, stream=None, perm=None):
     """Y[M,N] = (X * s_inv)[M,K] @ dequant(qweight, scales, zeros, g_idx)^T on the GPU.
@@ -259,10 +317,10 @@ def w4a16_gemm(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None
     With perm, the weights were packed with that permutation (w4_quantize_pack(perm=...))
     and the activation columns are gathered through it (w4a16_gemm_perm)."""
     torch = _torch()
-    M, K = X.shape
-    N = scales.shape[1]
+    M, K, N = _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y)
     if perm is not None and g_idx is not None:
         raise ValueError("pass g_idx or perm, not both")
+    _expect(perm, "perm", (torch.int32,), numel=K)
     dev = _need_cuda(X, qweight, scales, zeros, g_idx, s_inv, Y, workspace, perm)
     out_dtype = out_dtype or X.dtype
     if Y is None:
@@ -295,8 +353,7 @@ def w4a16_gemm_noalloc(X, qweight, scales, zeros, group_size=128, g_idx=None, s_
     the point of the call: the library's fixed per-device scratch is used instead.  Only
     Y is allocated here, and only when not passed in."""
     torch = _torch()
-    M, K = X.shape
-    N = scales.shape[1]
+    M, K, N = _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y)
     dev = _need_cuda(X, qweight, scales, zeros, g_idx, s_inv, Y)
     out_dtype = out_dtype or X.dtype
     if Y is None:
@@ -312,6 +369,8 @@ def w4a16_gemm_noalloc(X, qweight, scales, zeros, group_size=128, g_idx=None, s_
 
 def w4_unpack_canonical(qweight, N, K, out=None, stream=None):
     torch = _torch()
+    _expect(qweight, "qweight", _words(), numel=N * K // 8)
+    _expect(out, "out", _words(), numel=N * K // 8)
     dev = _need_cuda(qweight, out)
     if out is None:
         out = torch.empty(N, K // 8, dtype=torch.int32, device=dev)

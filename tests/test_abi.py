@@ -153,3 +153,77 @@ def test_awq_search_rejects_bad_arguments(L):
     assert ws(8, 128, 256, 128, 0, 0) == 0
     assert ws(8, 128, 256, 128, 0, 1025) == 0
     assert ws(8, 8, 256, 128, 0, 4) == 0
+
+
+def test_binding_refuses_wrong_dtypes_and_sizes():
+    """The binding checks every tensor's dtype and size before its pointer reaches the
+    library (which could not tell a short buffer from a long one).  CPU tensors suffice:
+    the checks run before the device check."""
+    import torch
+    M, N, K, g = 2, 32, 256, 64
+    G = K // g
+    X = torch.zeros(M, K, dtype=torch.float16)
+    qw = torch.zeros(N * K // 8, dtype=torch.int32)
+    sc = torch.zeros(G, N, dtype=torch.float16)
+    si = torch.zeros(K, dtype=torch.float32)
+    gi = torch.zeros(K, dtype=torch.int32)
+
+    def gemm(**kw):
+        a = dict(X=X, qweight=qw, scales=sc, zeros=sc, group_size=g)
+        a.update(kw)
+        return w4.w4a16_gemm(**a)
+
+    bad = [
+        (TypeError, "qweight", dict(qweight=qw.to(torch.int64))),
+        (ValueError, "qweight", dict(qweight=qw[:-1])),
+        (ValueError, "scales", dict(scales=sc[:-1], zeros=None)),
+        (ValueError, "zeros", dict(zeros=sc[:, :-1])),
+        (TypeError, "scales", dict(scales=sc.to(torch.bfloat16), zeros=None)),
+        (TypeError, "s_inv", dict(s_inv=si.half())),
+        (ValueError, "s_inv", dict(s_inv=si[:-1])),
+        (TypeError, "g_idx", dict(g_idx=gi.long())),
+        (ValueError, "g_idx", dict(g_idx=gi[:-1])),
+        (ValueError, "perm", dict(perm=gi[:-1])),
+        (ValueError, "Y", dict(Y=torch.zeros(M, N + 1, dtype=torch.float16))),
+        (TypeError, "Y", dict(Y=torch.zeros(M, N, dtype=torch.float64))),
+        (TypeError, "X", dict(X=X.float())),
+        (ValueError, "X", dict(X=X.reshape(-1))),
+        (ValueError, "group_size", dict(group_size=96)),
+        (ValueError, "group_size", dict(group_size=0)),
+    ]
+    for exc, what, kw in bad:
+        with pytest.raises(exc, match=what):
+            gemm(**kw)
+        if "perm" not in kw:
+            a = dict(X=X, qweight=qw, scales=sc, zeros=sc, group_size=g)
+            a.update(kw)
+            with pytest.raises(exc, match=what):
+                w4.w4a16_gemm_noalloc(**a)
+    with pytest.raises(ValueError, match="CUDA"):    # well-formed: stops at the device check
+        gemm(s_inv=si, Y=torch.zeros(M, N, dtype=torch.float16))
+
+    W = torch.zeros(N, K, dtype=torch.float16)
+    for exc, what, kw in [
+        (ValueError, "W", dict(W=W.reshape(-1))),
+        (TypeError, "W", dict(W=W.float())),
+        (ValueError, "s", dict(s=si[:-1])),
+        (ValueError, "perm", dict(perm=gi[:-1])),
+        (ValueError, "qweight", dict(qweight=qw[:-1])),
+        (ValueError, "scales", dict(scales=sc[:, :-1])),
+        (ValueError, "group_size", dict(group_size=100)),
+    ]:
+        a = dict(W=W, group_size=g)
+        a.update(kw)
+        with pytest.raises(exc, match=what):
+            w4.w4_quantize_pack(**a)
+
+    with pytest.raises(ValueError, match="channels"):
+        w4.w4_awq_search(W, torch.zeros(M, K + 64, dtype=torch.float16), g)
+    with pytest.raises(TypeError, match="X"):
+        w4.w4_awq_search(W, torch.zeros(M, K, dtype=torch.float32), g)
+    with pytest.raises(ValueError, match="vector"):
+        w4.w4_actorder_perm(gi.reshape(2, -1), g)
+    with pytest.raises(ValueError, match="perm"):
+        w4.w4_actorder_perm(gi, g, perm=gi[:-1])
+    with pytest.raises(ValueError, match="out"):
+        w4.w4_unpack_canonical(qw, N, K, out=qw[:-1])
