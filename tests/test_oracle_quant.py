@@ -4,7 +4,9 @@ Pins (none retypes the oracle's formulas):
   * AWQ identity ("Quantization Paradigms for Edge Inference: AWQ, GPTQ, and FP8 Matrix
     Cores", sec. 3, eq. 1): with power-of-two s the transformed product is bit-identical.
   * On-grid closed form: weights built as (q - z) * sc with sc a power of two and every
-    group spanning codes 0 and 15 must come back as exactly those q, z, sc.
+    group spanning codes 0 and 15 must come back as exactly those q, z, sc (fp16 and
+    bf16 weights).
+  * bf16 operands of the transform are read as bf16 (the format's top-half definition).
   * Brute force of round-to-nearest-even over all 16 codes.
   * Range properties of the scale / zero point; reconstruction error <= sc/2.
   * A hand-worked group (tests/golden/quant_hand_example.txt).
@@ -99,6 +101,48 @@ def test_on_grid_weights_recovered_exactly(symmetric, g, act_order):
     # dequantisation of the on-grid case reproduces the weights exactly
     What = oracle.dequant(q, scales, zeros, g, g_idx)
     assert np.array_equal(What, W.view(np.float16).astype(np.float32))
+
+
+def bf16_exact(W32):
+    """bf16 bit patterns of fp32 values that bf16 holds exactly: the upper 16 bits."""
+    W32 = np.ascontiguousarray(W32, np.float32)
+    assert np.all((W32.view(np.uint32) & 0xFFFF) == 0)
+    return (W32.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def bf16_decode(b):
+    """bf16 bit patterns -> fp32 by the format's definition (the bits are fp32's top half)."""
+    return (np.asarray(b, np.uint32) << 16).view(np.float32)
+
+
+@pytest.mark.parametrize("symmetric", [False, True])
+def test_on_grid_bf16_weights_recovered_exactly(symmetric):
+    """bf16 weights: (q - z) * 2^e needs at most 4 significant bits, so the on-grid weights
+    are exact in bf16 too and must come back as exactly q, z, sc."""
+    rng = np.random.default_rng(71 + symmetric)
+    N, K, g = 16, 256, 64
+    W16, q_true, sc_true, z_true = _on_grid(N, K, g, symmetric, rng)
+    Wb = bf16_exact(W16.view(np.float16).astype(np.float32))
+    q, scales, zeros = oracle.quantize_weights(Wb, None, g, symmetric, is_bf16=True)
+    assert np.array_equal(q, q_true)
+    assert np.array_equal(oracle.f16_to_f32(scales), sc_true)
+    if not symmetric:
+        assert np.array_equal(oracle.f16_to_f32(zeros), z_true.astype(np.float32))
+
+
+def test_awq_transform_reads_bf16_operands_as_bf16():
+    """The transform of bf16 operands decodes them as bf16: without s it returns the decoded
+    values, and with power-of-two s it scales them exactly (no rounding can occur)."""
+    rng = np.random.default_rng(72)
+    M, N, K = 3, 8, 64
+    Xb = bf16_exact(oracle.bf16_to_f32(oracle.f32_to_bf16(rng.standard_normal((M, K)).astype(np.float32))))
+    Wb = bf16_exact(oracle.bf16_to_f32(oracle.f32_to_bf16((rng.standard_normal((N, K)) * 0.02).astype(np.float32))))
+    s = (2.0 ** rng.integers(-3, 4, size=K)).astype(np.float32)
+    s_inv = (np.float32(1) / s).astype(np.float32)
+    assert np.array_equal(oracle.awq_scale_acts(Xb, None, True), bf16_decode(Xb))
+    assert np.array_equal(oracle.awq_scale_weights(Wb, None, True), bf16_decode(Wb))
+    assert np.array_equal(oracle.awq_scale_acts(Xb, s_inv, True), bf16_decode(Xb) * s_inv)
+    assert np.array_equal(oracle.awq_scale_weights(Wb, s, True), bf16_decode(Wb) * s)
 
 
 @pytest.mark.parametrize("symmetric", [False, True])
