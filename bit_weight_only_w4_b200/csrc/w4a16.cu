@@ -89,17 +89,6 @@ size_t decode_workspace_bytes(int64_t M, int sms) {
     return kCounterBytes + decode_slot_bytes(decode_tiles_for(M), sms);
 }
 
-int smem_per_sm(int dev) {
-    static int cache[kMaxDevices];
-    static std::once_flag flags[kMaxDevices];
-    std::call_once(flags[dev], [&] {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-        cache[dev] = v;
-    });
-    return cache[dev];
-}
-
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
