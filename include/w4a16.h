@@ -185,9 +185,11 @@ w4_status w4_quantize_pack_perm(const void* W, w4_dtype w_dtype, int64_t N, int6
 
 /*
  * w4a16_gemm_perm -- Y = X' What^T for weights packed by w4_quantize_pack_perm:
- *   Xp[m,k'] = X[m,perm[k']] * s_inv[perm[k']]  rounded to act_dtype (s_inv NULL: no scaling),
- * written into the workspace by one gather kernel, then w4a16_gemm(Xp, ..., g_idx = NULL,
- * s_inv = NULL).  Arguments as w4a16_gemm with perm in place of g_idx; fp16 and bf16
+ *   Xp[m,k'] = X[m,perm[k']] * s_inv[perm[k']]  rounded to act_dtype (s_inv NULL: no scaling).
+ * When the decode kernel keeps X' resident in shared memory (M <= 8 and M*K small), it
+ * gathers the columns itself while preparing X', in the one launch.  Otherwise one gather
+ * kernel writes Xp into the workspace and w4a16_gemm(Xp, ..., g_idx = NULL, s_inv = NULL)
+ * follows.  Arguments as w4a16_gemm with perm in place of g_idx; fp16 and bf16
  * activations.  workspace: at least w4a16_workspace_bytes_perm(M,N,K,group_size) bytes,
  * 256-byte aligned, zero-filled before its first use (as for w4a16_gemm).  An entry of perm
  * outside [0, K) reads channel 0 and is reported as W4_ERR_DEVICE_ARG by
