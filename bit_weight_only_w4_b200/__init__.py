@@ -100,7 +100,8 @@ def _dtype_code(dt):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # c_void_p arguments take a plain int (or None for NULL)
+    return None if t is None else t.data_ptr()
 
 
 def _stream_handle(stream, device):
@@ -172,10 +173,13 @@ class _DeviceGuard:
     def __enter__(self):
         torch = _torch()
         self.prev = torch.cuda.current_device()
-        torch.cuda.set_device(self.device)
+        self.switch = self.prev != self.device.index
+        if self.switch:
+            torch.cuda.set_device(self.device)
 
     def __exit__(self, *exc):
-        _torch().cuda.set_device(self.prev)
+        if self.switch:
+            _torch().cuda.set_device(self.prev)
 
 
 # ---------------------------------------------------------------- C ABI, same names
@@ -294,8 +298,42 @@ def workspace_for(device, nbytes):
         return buf
 
 
-def _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y):
-    """Shapes and dtypes of a GEMM call; returns (M, K, N), N taken from the scales."""
+_DTYPES = None
+
+
+def _dtypes():
+    """(float16, bfloat16, float32, int32, uint32), looked up once."""
+    global _DTYPES
+    if _DTYPES is None:
+        torch = _torch()
+        _DTYPES = (torch.float16, torch.bfloat16, torch.float32, torch.int32, torch.uint32)
+    return _DTYPES
+
+
+def _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y, perm=None):
+    """Shapes and dtypes of a GEMM call; returns (M, K, N), N taken from the scales.  A
+    well-formed call passes one combined test (the decode path is called per token and
+    per layer); any failure goes through the per-tensor checks, which name the culprit."""
+    f16, bf16, f32, i32, u32 = _dtypes()
+    xs, ss = X.shape, scales.shape
+    if len(xs) == 2 and len(ss) == 2 and group_size > 0 and xs[1] % group_size == 0:
+        M, K = xs
+        N = ss[1]
+        if ((X.dtype is f16 or X.dtype is bf16)
+                and (qweight.dtype is i32 or qweight.dtype is u32) and qweight.numel() == N * K // 8
+                and scales.dtype is f16 and ss[0] == K // group_size
+                and (zeros is None or (zeros.dtype is f16 and zeros.shape == ss))
+                and (g_idx is None or (g_idx.dtype is i32 and g_idx.numel() == K))
+                and (s_inv is None or (s_inv.dtype is f32 and s_inv.numel() == K))
+                and (perm is None or (perm.dtype is i32 and perm.numel() == K))
+                and (Y is None or ((Y.dtype is f16 or Y.dtype is bf16 or Y.dtype is f32)
+                                   and Y.shape == (M, N)))):
+            return M, K, N
+    _gemm_args_checked(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y, perm)
+    raise ValueError("inconsistent GEMM arguments")
+
+
+def _gemm_args_checked(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y, perm=None):
     torch = _torch()
     M, K = _matrix(X, "X")
     G = _groups(K, group_size)
@@ -307,7 +345,7 @@ def _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y):
     _expect(g_idx, "g_idx", (torch.int32,), numel=K)
     _expect(s_inv, "s_inv", (torch.float32,), numel=K)
     _expect(Y, "Y", _f16s() + (torch.float32,), shape=(M, N))
-    return M, K, N
+    _expect(perm, "perm", (torch.int32,), numel=K)
 
 
 def w4a16_gemm(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None,
@@ -317,10 +355,9 @@ def w4a16_gemm(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None
     With perm, the weights were packed with that permutation (w4_quantize_pack(perm=...))
     and the activation columns are gathered through it (w4a16_gemm_perm)."""
     torch = _torch()
-    M, K, N = _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y)
+    M, K, N = _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y, perm)
     if perm is not None and g_idx is not None:
         raise ValueError("pass g_idx or perm, not both")
-    _expect(perm, "perm", (torch.int32,), numel=K)
     dev = _need_cuda(X, qweight, scales, zeros, g_idx, s_inv, Y, workspace, perm)
     out_dtype = out_dtype or X.dtype
     if Y is None:
