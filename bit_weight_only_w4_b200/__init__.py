@@ -286,8 +286,9 @@ _ws_lock = threading.Lock()
 
 
 def workspace_for(device, nbytes):
-    """A zero-initialised scratch buffer of at least nbytes on `device`, shared by calls
-    on one stream (the kernels leave it zero-filled where that matters)."""
+    """A zero-initialised scratch buffer of at least nbytes on `device`, shared by every
+    call on that device that passes no workspace of its own (the kernels leave it
+    zero-filled where that matters).  Calls sharing it must be ordered on the GPU."""
     torch = _torch()
     key = torch.device(device).index
     with _ws_lock:
@@ -353,7 +354,12 @@ def w4a16_gemm(X, qweight, scales, zeros, group_size=128, g_idx=None, s_inv=None
     """Y[M,N] = (X * s_inv)[M,K] @ dequant(qweight, scales, zeros, g_idx)^T on the GPU.
 
     With perm, the weights were packed with that permutation (w4_quantize_pack(perm=...))
-    and the activation columns are gathered through it (w4a16_gemm_perm)."""
+    and the activation columns are gathered through it (w4a16_gemm_perm).
+
+    Without `workspace`, every call on a device shares one cached zero-filled buffer, which
+    is safe for calls ordered on one stream.  Calls that may run concurrently (unordered
+    streams) must each pass a workspace of their own: torch.zeros(w4a16_workspace_bytes(...),
+    dtype=torch.uint8, device=...)."""
     torch = _torch()
     M, K, N = _gemm_args(X, qweight, scales, zeros, group_size, g_idx, s_inv, Y, perm)
     if perm is not None and g_idx is not None:
