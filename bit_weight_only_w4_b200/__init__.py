@@ -1,8 +1,9 @@
 """B200 (sm_100a) W4A16: 4-bit weight-only quantised linear layers with 16-bit activations.
 
 Thin Python binding of the C ABI in include/w4a16.h.  The functions below carry the C
-names and only marshal arguments: PyTorch provides device memory, streams and output
-allocation; every step of the computation runs in the library's CUDA kernels
+names, check each tensor's dtype and size, and marshal arguments: PyTorch provides
+device memory, streams and output allocation; every step of the computation runs in
+the library's CUDA kernels
 (bit_weight_only_w4_b200/_lib/libw4a16.so, built in-tree by
 ``python -m bit_weight_only_w4_b200.build``).  There is no CPU fallback: if the library
 is missing or a call fails, an exception is raised.

@@ -249,3 +249,13 @@ def test_library_builds_without_warnings(L):
         strict = ("decode_kernelILi1E" in fn or "prefill_kernel" in fn or "quantize" in fn)
         limit = 0 if strict else 64
         assert st <= limit and ld <= limit, (fn, st, ld)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library the package raises; it never falls back to a CPU path."""
+    monkeypatch.setattr(w4, "LIB_PATH", str(tmp_path / "libw4a16.so"))
+    monkeypatch.setattr(w4, "_lib", None)
+    with pytest.raises(RuntimeError, match="not found"):
+        w4.lib()
+    with pytest.raises(RuntimeError, match="not found"):
+        w4.w4a16_workspace_bytes(1, 128, 128, 128)
