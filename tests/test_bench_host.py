@@ -52,3 +52,48 @@ def test_clock_sampler_without_nvidia_smi_reports_nothing():
     import bench
     cs = bench.ClockSampler(0)
     assert cs.stop() is None
+
+
+def test_our_arm_prints_every_contract_key(monkeypatch, capsys):
+    """bench.py's own line assembly, with the GPU measurements replaced by fixed numbers:
+    the JSON line carries every key of the benchmark contract, value is the whole job's
+    bytes over the timed milliseconds, and the roofline fraction is achieved / peak."""
+    sys.path.insert(0, ROOT)
+    import json
+    import types
+    import bench
+    from bit_weight_only_w4_b200 import workloads
+
+    wl = workloads.workload(bench.DECODE_CFG)
+    projs = [{"bytes": 1_000_000} for _ in wl.layers]
+    step_bytes = bench.N_LAYERS * 4_000_000
+    monkeypatch.setattr(bench, "prepare_weights", lambda w4, torch: (wl, projs, step_bytes))
+    monkeypatch.setattr(bench, "time_decode", lambda *a, **k: {
+        "total_ms": 100.0, "launches": 10 * bench.N_LAYERS * len(projs),
+        "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+        "per_layer": {"qkv": 10.0}})
+    monkeypatch.setattr(bench, "time_e2e", lambda *a, **k: (200.0, 32768, 98304))
+    monkeypatch.setattr(bench, "cpu_oracle_sample", lambda *a, **k: (0.04, 12.0, "stub"))
+    monkeypatch.setattr(bench, "load_peaks", lambda: ({"hbm_gbs": 6000.0, "bf16_tflops": 1600.0}, "measured"))
+    import bit_weight_only_w4_b200 as w4
+    monkeypatch.setattr(w4, "LIB_PATH", __file__)       # "built": no build attempted
+    args = types.SimpleNamespace(steps=10, warmup=3, quick=True, no_cpu=False, gpus=1)
+    bench.our_arm(args, 1, 0, 0)
+    line = json.loads(capsys.readouterr().out)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "roofline", "e2e", "gpu_launches", "clocks", "cpu_baseline"):
+        assert key in line, key
+    assert line["value"] == 10 * step_bytes / 0.1 / 1e9
+    assert line["ms_per_step"] == 10.0
+    r = line["roofline"]
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in r, key
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["frac"] - r["achieved"] / 6000.0) < 1e-12
+    e = line["e2e"]
+    assert e["h2d_bytes_per_step"] == 32768 and e["d2h_bytes_per_step"] == 98304
+    assert e["value"] == 10 * step_bytes / 0.2 / 1e9
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["gpu_launches"] == 10 * bench.N_LAYERS * 4
+    assert "workload" in line["config"]
