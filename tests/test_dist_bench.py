@@ -62,3 +62,9 @@ def test_reference_arm_prints_from_rank_zero_only(capsys, monkeypatch):
     bench.reference_arm(Args(), 2, 0)
     line = json.loads(capsys.readouterr().out)
     assert line["impl"] == "reference" and line["value"] == 1.0 and line["n_gpus"] == 2
+    for key in ("metric", "unit", "steps", "warmup", "higher_is_better", "scaling", "dtype",
+                "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == 1.0
+    assert line["e2e"] == {"value": 1.0, "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
