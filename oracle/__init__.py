@@ -52,6 +52,20 @@ def lib():
         L.oracle_dequant.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp]
         L.oracle_gemm_f32.argtypes = [vp, vp, i64, i64, i64, vp, i64, vp]
         L.oracle_gemm_f64.argtypes = [vp, vp, i64, i64, i64, vp, i64, vp]
+        L.oracle_e2m1_to_f32.argtypes = [ctypes.c_uint8]
+        L.oracle_e2m1_to_f32.restype = ctypes.c_float
+        L.oracle_f32_to_e2m1.argtypes = [ctypes.c_float]
+        L.oracle_f32_to_e2m1.restype = ctypes.c_uint8
+        L.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_to_f32.restype = ctypes.c_float
+        L.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+        L.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+        L.oracle_nvfp4_quantize.argtypes = [vp, ctypes.c_int, i64, i64, vp, vp, vp]
+        L.oracle_nvfp4_quantize.restype = ctypes.c_int
+        L.oracle_nvfp4_dequant.argtypes = [vp, vp, ctypes.c_float, i64, i64, vp]
+        L.oracle_mxfp4_quantize.argtypes = [vp, ctypes.c_int, i64, i64, vp, vp]
+        L.oracle_mxfp4_quantize.restype = ctypes.c_int
+        L.oracle_mxfp4_dequant.argtypes = [vp, vp, i64, i64, vp]
         _LIB = L
     return _LIB
 
@@ -257,3 +271,65 @@ def awq_search(W_bits, X_bits, group_size, symmetric=False, n_grid=20, w_is_bf16
         cand.append(s)
     best = int(np.argmin(losses))
     return best, losses, cand[best]
+
+
+# ---- block-scaled 4-bit floating point (NVFP4, MXFP4) --------------------------------
+def e2m1_to_f32(c):
+    return float(lib().oracle_e2m1_to_f32(int(c)))
+
+
+def f32_to_e2m1(x):
+    return int(lib().oracle_f32_to_e2m1(float(x)))
+
+
+def e4m3_to_f32(b):
+    return float(lib().oracle_e4m3_to_f32(int(b)))
+
+
+def f32_to_e4m3(x):
+    return int(lib().oracle_f32_to_e4m3(float(x)))
+
+
+def nvfp4_quantize(A_bits, is_bf16=False):
+    """NVFP4 of A [R,K] ("Production Quantization: AWQ, GPTQ, GGUF K-quants, FP8,
+    MXFP4/NVFP4", section "MXFP4 / NVFP4": a scale per block; block of 16, E4M3 block
+    scales and the tensor scale are readings, stated in w4_oracle.c).
+    Returns (codes uint8 [R,K], block scales uint8 [R,K/16], tensor scale fp32)."""
+    A_bits = bits16(A_bits)
+    R, K = A_bits.shape
+    codes = np.empty((R, K), np.uint8)
+    bs = np.empty((R, K // 16), np.uint8)
+    gs = ctypes.c_float()
+    if lib().oracle_nvfp4_quantize(_p(A_bits), int(is_bf16), R, K, _p(codes), _p(bs), ctypes.byref(gs)) != 0:
+        raise ValueError("NVFP4 needs K % 16 == 0")
+    return codes, bs, np.float32(gs.value)
+
+
+def nvfp4_dequant(codes, bscale, gs):
+    codes = _c(codes, np.uint8)
+    bscale = _c(bscale, np.uint8)
+    R, K = codes.shape
+    out = np.empty((R, K), np.float64)
+    lib().oracle_nvfp4_dequant(_p(codes), _p(bscale), float(gs), R, K, _p(out))
+    return out
+
+
+def mxfp4_quantize(A_bits, is_bf16=False):
+    """MXFP4 of A [R,K] (same page and section; block of 32 and the E8M0 scale are
+    readings).  Returns (codes uint8 [R,K], scale bytes uint8 [R,K/32])."""
+    A_bits = bits16(A_bits)
+    R, K = A_bits.shape
+    codes = np.empty((R, K), np.uint8)
+    es = np.empty((R, K // 32), np.uint8)
+    if lib().oracle_mxfp4_quantize(_p(A_bits), int(is_bf16), R, K, _p(codes), _p(es)) != 0:
+        raise ValueError("MXFP4 needs K % 32 == 0")
+    return codes, es
+
+
+def mxfp4_dequant(codes, escale):
+    codes = _c(codes, np.uint8)
+    escale = _c(escale, np.uint8)
+    R, K = codes.shape
+    out = np.empty((R, K), np.float64)
+    lib().oracle_mxfp4_dequant(_p(codes), _p(escale), R, K, _p(out))
+    return out

@@ -23,6 +23,9 @@
  *   [PACK] same article, section "Kernel Execution: Marlin vs. ExLlamaV2 INT4 GEMM
  *          Micro-Architecture", item 3: two 4-bit weights share one byte and are
  *          recovered with shift and AND.
+ *   [FP4]  "Production Quantization: AWQ, GPTQ, GGUF K-quants, FP8, MXFP4/NVFP4",
+ *          section "MXFP4 / NVFP4" and glossary: block-scaled 4-bit floating point (the
+ *          last section of this file; its format readings are stated there).
  *
  * Readings where the pages are silent:
  *   - W is [N,K] row-major (out x in); Y = X' * What^T is [M,N].
@@ -360,4 +363,131 @@ void oracle_gemm_f64(const float* Xp, const float* What, int64_t M, int64_t N, i
             Y[i * N + n] = acc;
         }
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* Block-scaled 4-bit floating point (NVFP4, MXFP4).                   */
+/* ------------------------------------------------------------------ */
+/* "Production Quantization: AWQ, GPTQ, GGUF K-quants, FP8, MXFP4/NVFP4", section
+ * "MXFP4 / NVFP4" and its glossary: microscaling 4-bit floating point in which every
+ * block of weights carries its own scale factor, run by Blackwell's tensor cores.  The
+ * pages fix nothing further; the encodings below are the formats' published
+ * definitions, taken as readings:
+ *   element  E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; magnitudes
+ *            0, 0.5, 1, 1.5, 2, 3, 4, 6; no infinity or NaN.
+ *   NVFP4    blocks of 16 consecutive k, an E4M3 block scale (bias 7, no infinity,
+ *            largest finite 448) and one fp32 scale for the whole tensor:
+ *              gs = amax / (6 * 448)  (1 for an all-zero tensor),
+ *              sb = E4M3(blockmax / 6 / gs),   q = E2M1(w / (dec(sb) * gs)).
+ *   MXFP4    blocks of 32, a power-of-two scale 2^e stored as the byte e + 127 (E8M0),
+ *              e = floor(log2(blockmax)) - 2   (2 = the largest E2M1 exponent),
+ *              q = E2M1(w / 2^e).
+ * Every encoding rounds to the nearest representable value, ties to the even
+ * mantissa, and saturates finite values beyond the largest magnitude.  The search is
+ * exhaustive over the codes, which is the definition of round-to-nearest. */
+
+float oracle_e2m1_to_f32(uint8_t c) {
+    const int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    const float mag = e == 0 ? 0.5f * (float)m : ldexpf(1.0f + 0.5f * (float)m, e - 1);
+    return s ? -mag : mag;
+}
+
+uint8_t oracle_f32_to_e2m1(float x) {
+    const double a = fabs((double)x);
+    uint8_t best = 0;
+    double bd = INFINITY;
+    for (uint8_t c = 0; c < 8; ++c) {
+        const double d = fabs(a - (double)oracle_e2m1_to_f32(c));
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            bd = d;
+            best = c;
+        }
+    }
+    return (uint8_t)((signbit(x) ? 8 : 0) | best);
+}
+
+float oracle_e4m3_to_f32(uint8_t b) {
+    const int s = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    float mag;
+    if (e == 15 && m == 7) mag = NAN;
+    else if (e == 0) mag = ldexpf((float)m, -9);               /* (m/8) 2^-6 */
+    else mag = ldexpf((float)(8 + m), e - 10);                 /* (1 + m/8) 2^(e-7) */
+    return s ? -mag : mag;
+}
+
+uint8_t oracle_f32_to_e4m3(float x) {
+    const double a = fabs((double)x);
+    uint8_t best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < 127; ++c) {                           /* 127 = NaN */
+        const double d = fabs(a - (double)oracle_e4m3_to_f32((uint8_t)c));
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            bd = d;
+            best = (uint8_t)c;
+        }
+    }
+    return (uint8_t)((signbit(x) ? 0x80 : 0) | best);
+}
+
+/* NVFP4 of A [R,K] (fp16/bf16 bits), K % 16 == 0: codes [R,K] one E2M1 code per byte,
+   block scales [R,K/16] E4M3 bytes, *gs the tensor scale.  Returns 0, -1 on bad K. */
+int oracle_nvfp4_quantize(const uint16_t* A, int is_bf16, int64_t R, int64_t K,
+                          uint8_t* codes, uint8_t* bscale, float* gs) {
+    if (K % 16 != 0) return -1;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < R * K; ++i) amax = fmaxf(amax, fabsf(load16(A, i, is_bf16)));
+    const float g = amax > 0.0f ? amax / (6.0f * 448.0f) : 1.0f;
+    *gs = g;
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t b = 0; b < K / 16; ++b) {
+            float bmax = 0.0f;
+            for (int64_t k = 16 * b; k < 16 * b + 16; ++k) bmax = fmaxf(bmax, fabsf(load16(A, r * K + k, is_bf16)));
+            const uint8_t sb = oracle_f32_to_e4m3(bmax / 6.0f / g);
+            bscale[r * (K / 16) + b] = sb;
+            const float sd = oracle_e4m3_to_f32(sb) * g;
+            for (int64_t k = 16 * b; k < 16 * b + 16; ++k) {
+                const float w = load16(A, r * K + k, is_bf16);
+                codes[r * K + k] = sd > 0.0f ? oracle_f32_to_e2m1(w / sd) : 0;
+            }
+        }
+    return 0;
+}
+
+/* dequantised NVFP4 values: A^[r,k] = E2M1(code) * (E4M3(sb) * gs), in fp64 (exact:
+   the first factor has 2 significant bits, the block scale 4, gs is one fp32). */
+void oracle_nvfp4_dequant(const uint8_t* codes, const uint8_t* bscale, float gs, int64_t R, int64_t K,
+                          double* out) {
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = (double)oracle_e2m1_to_f32(codes[r * K + k]) *
+                             (double)oracle_e4m3_to_f32(bscale[r * (K / 16) + k / 16]) * (double)gs;
+}
+
+/* MXFP4 of A [R,K], K % 32 == 0: codes [R,K], scale bytes [R,K/32] (E8M0: 2^(byte-127)). */
+int oracle_mxfp4_quantize(const uint16_t* A, int is_bf16, int64_t R, int64_t K, uint8_t* codes,
+                          uint8_t* escale) {
+    if (K % 32 != 0) return -1;
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t b = 0; b < K / 32; ++b) {
+            float bmax = 0.0f;
+            for (int64_t k = 32 * b; k < 32 * b + 32; ++k) bmax = fmaxf(bmax, fabsf(load16(A, r * K + k, is_bf16)));
+            int e = -127;
+            if (bmax > 0.0f) {
+                int ex;
+                (void)frexpf(bmax, &ex);                       /* bmax = f 2^ex, f in [0.5, 1) */
+                e = ex - 1 - 2;
+                if (e < -127) e = -127;
+            }
+            escale[r * (K / 32) + b] = (uint8_t)(e + 127);
+            for (int64_t k = 32 * b; k < 32 * b + 32; ++k)
+                codes[r * K + k] = oracle_f32_to_e2m1(ldexpf(load16(A, r * K + k, is_bf16), -e));
+        }
+    return 0;
+}
+
+void oracle_mxfp4_dequant(const uint8_t* codes, const uint8_t* escale, int64_t R, int64_t K, double* out) {
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = ldexp((double)oracle_e2m1_to_f32(codes[r * K + k]),
+                                   (int)escale[r * (K / 32) + k / 32] - 127);
 }
