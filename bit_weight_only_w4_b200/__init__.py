@@ -79,8 +79,20 @@ def lib():
         L.w4_awq_search.restype = st
         L.w4_awq_search_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32]
         L.w4_awq_search_workspace_bytes.restype = sz
+        L.w4a16_gemm_chain.argtypes = [ctypes.POINTER(ChainLayer), i32, i64, st, st, vp, sz, vp]
+        L.w4a16_gemm_chain.restype = st
+        L.w4a16_chain_workspace_bytes.argtypes = [i64]
+        L.w4a16_chain_workspace_bytes.restype = sz
         _lib = L
     return _lib
+
+
+class ChainLayer(ctypes.Structure):
+    """w4_chain_layer of include/w4a16.h."""
+    _fields_ = [("X", ctypes.c_void_p), ("ldx", ctypes.c_int64), ("qweight", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p), ("s_inv", ctypes.c_void_p),
+                ("Y", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("group_size", ctypes.c_int32)]
 
 
 # ---------------------------------------------------------------- marshalling helpers
@@ -411,6 +423,61 @@ def w4a16_gemm_noalloc(X, qweight, scales, zeros, group_size=128, g_idx=None, s_
     return Y
 
 
+def w4a16_chain_workspace_bytes(M):
+    return int(lib().w4a16_chain_workspace_bytes(int(M)))
+
+
+def w4a16_gemm_chain(layers, workspace=None, stream=None):
+    """Run a list of small-batch GEMMs (M <= 8) in order, in one persistent launch per 32
+    layers.  Each layer is a dict with X, qweight, scales, zeros, group_size, s_inv and Y
+    (X [M,K] may be a view of an earlier layer's Y: rows may be further apart than K,
+    elements must be contiguous).  Layer l+1 reads its X only after every earlier output
+    is stored.  Outputs are written into the given Y tensors; returns the list of Ys."""
+    torch = _torch()
+    n = len(layers)
+    if n == 0:
+        return []
+    arr = (ChainLayer * n)()
+    M = None
+    act = None
+    out = None
+    devs = []
+    for i, d in enumerate(layers):
+        X, Y = d["X"], d["Y"]
+        qw, sc, zr, s_inv = d["qweight"], d["scales"], d.get("zeros"), d.get("s_inv")
+        g = int(d.get("group_size", 128))
+        if X.dim() != 2 or Y.dim() != 2 or X.stride(1) != 1 or not Y.is_contiguous():
+            raise ValueError(f"layer {i}: X must be a 2-D row-strided view, Y a contiguous matrix")
+        m, K = X.shape
+        N = Y.shape[1]
+        if M is None:
+            M, act, out = m, X.dtype, Y.dtype
+        if m != M or Y.shape[0] != M or X.dtype != act or Y.dtype != out:
+            raise ValueError(f"layer {i}: every layer has the same M, activation and output dtype")
+        _expect(qw, "qweight", _words(), numel=N * K // 8)
+        G = _groups(K, g)
+        _expect(sc, "scales", _f16s(), shape=(G, N))
+        _expect(zr, "zeros", _f16s(), shape=(G, N))
+        _expect(s_inv, "s_inv", (torch.float32,), numel=K)
+        if not X.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors (there is no CPU path)")
+        devs += [Y, qw, sc, zr, s_inv]
+        arr[i] = ChainLayer(_ptr(X), X.stride(0), _ptr(qw), _ptr(sc), _ptr(zr), _ptr(s_inv), _ptr(Y),
+                            N, K, g)
+    dev = _need_cuda(*devs, workspace)
+    if any(d["X"].device != dev for d in layers):
+        raise ValueError("tensors are on different devices")
+    with _DeviceGuard(dev):
+        need = w4a16_chain_workspace_bytes(M)
+        if workspace is None and need > 0:
+            workspace = workspace_for(dev, need)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib().w4a16_gemm_chain(arr, n, M, _dtype_code(act), _dtype_code(out), _ptr(workspace),
+                                    ws_bytes, _stream_handle(stream, dev))
+    _check(st, "w4a16_gemm_chain")
+    return [d["Y"] for d in layers]
+
+
 def w4_unpack_canonical(qweight, N, K, out=None, stream=None):
     torch = _torch()
     _expect(qweight, "qweight", _words(), numel=N * K // 8)
@@ -426,7 +493,18 @@ def w4_unpack_canonical(qweight, N, K, out=None, stream=None):
 
 
 def w4_check_device_error():
+    """Synchronise the current device and raise if a kernel reported an error.  After a
+    timeout the library zeroes its allocation-free scratch again, and this binding zeroes
+    its cached workspace of the current device (a kernel that gave up a wait may have left
+    split-K flags in either)."""
     st = lib().w4_check_device_error()
+    if st == W4_ERR_TIMEOUT:
+        torch = _torch()
+        with _ws_lock:
+            buf = _ws_cache.get(torch.cuda.current_device())
+            if buf is not None:
+                buf.zero_()
+                torch.cuda.synchronize()
     _check(st, "w4_check_device_error")
 
 

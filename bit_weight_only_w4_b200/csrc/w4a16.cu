@@ -12,6 +12,7 @@
 #include "w4_prefill.cuh"
 #include "w4_quant.cuh"
 #include "w4_actorder.cuh"
+#include "w4_chain.cuh"
 #include "w4_awq.cuh"
 
 namespace {
@@ -396,6 +397,12 @@ static w4_status quantize_pack_impl(const void* W, w4_dtype w_dtype, int64_t N, 
     return launch_status();
 }
 
+namespace {
+// Zero the allocation-free scratch of device `dev` again if it has been set up (defined
+// with the scratch, below).
+cudaError_t noalloc_rezero(int dev);
+}  // namespace
+
 extern "C" {
 
 const char* w4_status_string(w4_status s) {
@@ -692,6 +699,11 @@ w4_status w4_check_device_error(void) {
         const unsigned zero = 0;
         if (cudaMemcpyToSymbol(g_w4_error_word, &zero, sizeof(zero)) != cudaSuccess) return W4_ERR_CUDA;
     }
+    // A kernel that gave up a wait may have left split-K flags set in the scratch it used.
+    // The library's own allocation-free scratch is zeroed again here (every kernel has
+    // finished after the synchronisation above); a caller's workspace is the caller's to
+    // zero.
+    if ((word & W4_DEVERR_TIMEOUT) && noalloc_rezero(current_device()) != cudaSuccess) return W4_ERR_CUDA;
     if (word & W4_DEVERR_TIMEOUT) return W4_ERR_TIMEOUT;
     if (word & W4_DEVERR_GIDX) return W4_ERR_DEVICE_ARG;
     return W4_OK;
@@ -734,25 +746,35 @@ constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;   // 8 MiB
 __device__ __align__(256) unsigned char g_w4_noalloc_scratch[kNoAllocScratchBytes];
 
 struct NoAllocScratch {
-    std::once_flag once;
-    void* ptr = nullptr;
-    cudaError_t err = cudaSuccess;
+    std::mutex mu;
+    void* ptr = nullptr;   // set once the set-up has succeeded; a failed set-up is retried
 };
 NoAllocScratch g_noalloc[kMaxDevices];
 
-// Set-up on the first call per device (that device current): look up the array's device
-// address and zero it (every call expects the split-K flags it reads to start at zero and
-// leaves them at zero).
+// Set-up on the first successful call per device (that device current): look up the
+// array's device address and zero it (every call expects the split-K flags it reads to
+// start at zero and leaves them at zero).  A failed set-up leaves ptr null, so the next
+// call tries again.
 void* noalloc_scratch(int dev) {
     NoAllocScratch& s = g_noalloc[dev];
-    std::call_once(s.once, [&] {
-        void* p = nullptr;
-        s.err = cudaGetSymbolAddress(&p, g_w4_noalloc_scratch);
-        if (s.err == cudaSuccess) s.err = cudaMemset(p, 0, kNoAllocScratchBytes);
-        if (s.err == cudaSuccess) s.err = cudaDeviceSynchronize();
-        if (s.err == cudaSuccess) s.ptr = p;
-    });
-    return s.ptr;
+    std::lock_guard<std::mutex> lock(s.mu);
+    if (s.ptr) return s.ptr;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_w4_noalloc_scratch) != cudaSuccess) return nullptr;
+    if (cudaMemset(p, 0, kNoAllocScratchBytes) != cudaSuccess) return nullptr;
+    if (cudaDeviceSynchronize() != cudaSuccess) return nullptr;
+    s.ptr = p;
+    return p;
+}
+
+cudaError_t noalloc_rezero(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaSuccess;
+    NoAllocScratch& s = g_noalloc[dev];
+    std::lock_guard<std::mutex> lock(s.mu);
+    if (!s.ptr) return cudaSuccess;   // never set up: nothing was used
+    cudaError_t e = cudaMemset(s.ptr, 0, kNoAllocScratchBytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    return e;
 }
 
 }  // namespace
@@ -804,4 +826,184 @@ extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64
     const int mode = decode_mode(K, group_size, gidx);
     if (bf16) return dispatch_decode<true>(mode, p, X, ws, dev, strm);
     return dispatch_decode<false>(mode, p, X, ws, dev, strm);
+}
+
+// ---------------------------------------------------------------------------------------
+// w4a16_gemm_chain: a list of decode GEMMs (M <= 8, one token tile, X' resident) in
+// persistent launches of up to w4c::kMaxLayers layers each.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+size_t chain_workspace_bytes(int sms) { return kCounterBytes + decode_slot_bytes(1, sms); }
+
+// The layer-sequence kernel keeps every layer's X' and sums resident; up to 120 KB of them
+// still leave the weight ring at least three stages (checked again per launch).
+bool chain_x_resident(int64_t M, int64_t K) {
+    auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
+    if (M > 8) return false;
+    const int64_t sstride = std::max<int64_t>(2, (M + 1) / 2 * 2);
+    return up(M * K * 2, 128) + up((K / 32 + K / 64 + K / 128) * sstride * 4, 128) <= 120 * 1024;
+}
+
+template <bool BF16, int MODE>
+w4_status launch_chain(w4c::ChainParams& cp, int smem, int grid, int dev, cudaStream_t stream) {
+    static std::once_flag flags[kMaxDevices];
+    auto k = w4c::chain_kernel<BF16, MODE>;
+    bool attr_ok = true;
+    std::call_once(flags[dev], [&] {
+        attr_ok = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) ==
+                  cudaSuccess;
+    });
+    if (!attr_ok) return W4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(w4d::Cfg<1>::threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k, cp) != cudaSuccess) return W4_ERR_CUDA;
+    return launch_status();
+}
+
+// One launch over layers [l0, l0 + n) of the list (n <= kMaxLayers).
+w4_status chain_launch(const w4_chain_layer* layers, int l0, int n, int M, bool bf16, int out_dtype, int mode,
+                       unsigned char* ws, int dev, int sms, cudaStream_t stream) {
+    using C = w4d::Cfg<1>;
+    auto up = [](int v, int a) { return (v + a - 1) / a * a; };
+    constexpr int kMaxSmem = 227 * 1024;
+    // ring geometry shared by the launch's layers: codes | scale rows | zero-point rows |
+    // stage descriptor, sized for the largest per-stage group-row count
+    const int span = 64 * C::aps;
+    int ngs_max = 1, kmax = 64;
+    bool any_zeros = false;
+    for (int l = l0; l < l0 + n; ++l) {
+        const int g = layers[l].group_size;
+        const int G = (int)(layers[l].K / g);
+        const int ngs = g == 32 ? span / 32 : std::min(G, (span + 2 * g - 65) / g);
+        ngs_max = std::max(ngs_max, ngs);
+        kmax = std::max(kmax, (int)layers[l].K);
+        any_zeros = any_zeros || layers[l].zeros != nullptr;
+    }
+    const int sstride = std::max(2, (M + 1) / 2 * 2);
+    const int res_x = up(M * kmax * 2, 128);
+    const int res_s = up((kmax / 32 + kmax / 64 + kmax / 128) * sstride * 4, 128);
+    const int off_sc = C::aps * w4d::kTilesPerBand * 512;
+    const int off_zr = off_sc + ngs_max * 256;
+    const int off_desc = off_zr + (any_zeros ? ngs_max * 256 : 0);
+    const int stage_bytes = up(off_desc + 48, 1024);
+    const int fixed = res_x + res_s + C::xchg_bytes + 3 * w4d::kMaxStages * 8 + 16 + 1024;
+    const int stages = std::min(w4d::kMaxStages, (kMaxSmem - fixed) / stage_bytes);
+    if (stages < 3) return W4_ERR_UNSUPPORTED;
+    const int smem = stages * stage_bytes + fixed;
+
+    static w4c::ChainParams cp_storage[kMaxDevices];   // large: kept off the stack
+    static std::mutex cp_mu[kMaxDevices];
+    std::lock_guard<std::mutex> lock(cp_mu[dev]);
+    w4c::ChainParams& cp = cp_storage[dev];
+    std::memset(&cp, 0, sizeof(cp));
+    cp.n_layers = n;
+    cp.counter = reinterpret_cast<unsigned int*>(ws);   // word 0 of the zero region
+    for (int j = 0; j < n; ++j) {
+        const w4_chain_layer& Lc = layers[l0 + j];
+        w4d::DecodeParams& p = cp.L[j];
+        p.qw = Lc.qweight;
+        p.scales = reinterpret_cast<const __half*>(Lc.scales);
+        p.zeros = reinterpret_cast<const __half*>(Lc.zeros);
+        p.s_inv = Lc.s_inv;
+        p.X = Lc.X;
+        p.Y = Lc.Y;
+        p.slots = reinterpret_cast<unsigned long long*>(ws + kCounterBytes);
+        p.M = M;
+        p.N = (int)Lc.N;
+        p.K = (int)Lc.K;
+        p.ldx = (int)Lc.ldx;
+        p.group_size = Lc.group_size;
+        p.G = (int)(Lc.K / Lc.group_size);
+        p.out_dtype = out_dtype;
+        p.KA = (int)(Lc.K / 64);
+        p.KU = (p.KA + 1) / 2;
+        p.tiles = (int)(Lc.N / 16);
+        const int bands = (p.tiles + w4d::kTilesPerBand - 1) / w4d::kTilesPerBand;
+        p.units = bands * p.KU;
+        p.base = p.units / sms;
+        p.rem = p.units % sms;
+        const int g = p.group_size;
+        p.ngs = g == 32 ? span / 32 : std::min(p.G, (span + 2 * g - 65) / g);
+        p.stages = stages;
+        p.xres = 1;
+        p.sstride = sstride;
+        p.off_x = p.off_xs = p.off_sx = p.off_si = off_sc;
+        p.off_sc = off_sc;
+        p.off_zr = off_zr;
+        p.off_gi = off_desc;
+        p.off_desc = off_desc;
+        p.stage_bytes = stage_bytes;
+        p.off_res = stages * stage_bytes;
+        p.off_res_s = p.off_res + res_x;
+        p.off_xchg = p.off_res + res_x + res_s;
+        if (!make_meta_map(&cp.sc[j], p.scales, p.G, p.N, p.ngs)) return W4_ERR_CUDA;
+        if (p.zeros && !make_meta_map(&cp.zr[j], p.zeros, p.G, p.N, p.ngs)) return W4_ERR_CUDA;
+        if (!p.zeros) cp.zr[j] = cp.sc[j];
+    }
+    if (bf16) {
+        if (mode == w4d::kModeHalf) return launch_chain<true, w4d::kModeHalf>(cp, smem, sms, dev, stream);
+        if (mode == w4d::kModeG32) return launch_chain<true, w4d::kModeG32>(cp, smem, sms, dev, stream);
+        return launch_chain<true, w4d::kModeAtom>(cp, smem, sms, dev, stream);
+    }
+    if (mode == w4d::kModeHalf) return launch_chain<false, w4d::kModeHalf>(cp, smem, sms, dev, stream);
+    if (mode == w4d::kModeG32) return launch_chain<false, w4d::kModeG32>(cp, smem, sms, dev, stream);
+    return launch_chain<false, w4d::kModeAtom>(cp, smem, sms, dev, stream);
+}
+
+}  // namespace
+
+extern "C" size_t w4a16_chain_workspace_bytes(int64_t M) {
+    if (M < 1 || M > 8) return 0;
+    const int dev = current_device();
+    const int sms = dev >= 0 ? sm_count(dev) : 0;
+    return sms > 0 ? chain_workspace_bytes(sms) : 0;
+}
+
+extern "C" w4_status w4a16_gemm_chain(const w4_chain_layer* layers, int32_t n_layers, int64_t M,
+                                      w4_dtype act_dtype, w4_dtype out_dtype, void* workspace,
+                                      size_t workspace_bytes, w4_stream_t stream) {
+    if (!layers || n_layers < 0 || M < 0) return W4_ERR_INVALID_ARG;
+    if (act_dtype != W4_F16 && act_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
+    if (out_dtype != W4_F16 && out_dtype != W4_BF16 && out_dtype != W4_F32) return W4_ERR_INVALID_ARG;
+    if (n_layers == 0 || M == 0) return W4_OK;
+    if (M > 8) return W4_ERR_UNSUPPORTED;
+    int mode = -1;
+    for (int l = 0; l < n_layers; ++l) {
+        const w4_chain_layer& L = layers[l];
+        w4_status st = check_layer_shape(L.N, L.K, L.group_size);
+        if (st != W4_OK) return st;
+        if (!L.X || !L.qweight || !L.scales || !L.Y) return W4_ERR_INVALID_ARG;
+        if (!aligned(L.X, 16) || !aligned(L.qweight, 16) || !aligned(L.scales, 16) || !aligned(L.zeros, 16) ||
+            !aligned(L.s_inv, 16) || !aligned(L.Y, 16))
+            return W4_ERR_INVALID_ARG;
+        if (L.ldx < L.K || L.ldx % 8 != 0 || L.ldx > INT_MAX / 16) return W4_ERR_INVALID_ARG;
+        if (!chain_x_resident(M, L.K)) return W4_ERR_UNSUPPORTED;
+        const int m = decode_mode(L.K, L.group_size, false);
+        if (mode >= 0 && m != mode) return W4_ERR_UNSUPPORTED;   // one group mode per list
+        mode = m;
+    }
+    if (!aligned(workspace, 256)) return W4_ERR_INVALID_ARG;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    const int sms = sm_count(dev);
+    if (sms <= 0) return W4_ERR_CUDA;
+    if (!workspace || workspace_bytes < chain_workspace_bytes(sms)) return W4_ERR_INVALID_ARG;
+    unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
+    cudaStream_t strm = as_stream(stream);
+    for (int l0 = 0; l0 < n_layers; l0 += w4c::kMaxLayers) {
+        const int n = std::min(w4c::kMaxLayers, n_layers - l0);
+        w4_status st = chain_launch(layers, l0, n, (int)M, act_dtype == W4_BF16, (int)out_dtype, mode, ws, dev,
+                                    sms, strm);
+        if (st != W4_OK) return st;
+    }
+    return W4_OK;
 }

@@ -238,6 +238,60 @@ size_t w4_awq_search_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t gr
                                      int32_t symmetric, int32_t n_grid);
 
 /*
+ * w4a16_gemm_chain -- a list of small-batch GEMMs in order, in one persistent launch per
+ * 32 layers: Y_l = (X_l * s_inv_l) @ dequant(W_l)^T for l = 0, 1, ..., each exactly as
+ * w4a16_gemm computes it for the same M.  A decode step reads every weight once per
+ * token and is bound by memory bandwidth (edgesiliconlab.com article on AWQ vs GPTQ,
+ * "The Mathematics of Memory Bandwidth Saturation"); in one launch the packed weights
+ * of layer l+1 are already streaming while the GPU finishes layer l, which separate
+ * launches cannot do.
+ *
+ * Layer l+1 starts reading X_{l+1} only after every output of layers 0..l is stored, so
+ * X_{l+1} may point into the output of any earlier layer of the list (a slice of a row:
+ * X + offset with row stride ldx).  Each X_l row holds K_l values of act_dtype; Y_l is
+ * written in out_dtype, so a layer that feeds a later one wants out_dtype == act_dtype.
+ *
+ *   layers     HOST array of n_layers descriptors (read during the call only):
+ *                X       device [M, K] activations, rows ldx elements apart
+ *                        (ldx >= K, ldx % 8 == 0), 16-byte aligned
+ *                qweight, scales, zeros, group_size, N, K: as for w4a16_gemm (no g_idx)
+ *                s_inv   device fp32 [K] or NULL
+ *                Y       device [M, N] output (row-major, rows N apart)
+ *   M          1..8; every layer's M*K*2 bytes of X' plus its channel sums must fit the
+ *              resident budget (120 KB, leaving the weight ring at least three stages),
+ *              else W4_ERR_UNSUPPORTED (K = 11008 allows M <= 4, K = 4096 every M <= 8)
+ *   every layer must use the same group handling: group sizes all multiples of 128 with
+ *              K % 128 == 0, or all 32, or all other multiples of 64
+ *   workspace  device, >= w4a16_chain_workspace_bytes(M) bytes, 256-byte aligned,
+ *              ZERO-FILLED BEFORE ITS FIRST USE; each launch leaves it zero again (a
+ *              w4a16_gemm workspace of at least this size may be shared with it on one
+ *              stream); after W4_ERR_TIMEOUT zero it again
+ * All CTAs of a launch (one per SM) must be resident together, which holds when no
+ * other work occupies the GPU's SMs; the waits between layers are bounded and report
+ * W4_ERR_TIMEOUT through w4_check_device_error() if that is ever violated.
+ * Asynchronous on `stream`.  n_layers == 0 or M == 0 is a no-op.
+ */
+typedef struct {
+    const void* X;
+    int64_t ldx;
+    const uint32_t* qweight;
+    const void* scales;
+    const void* zeros;
+    const float* s_inv;
+    void* Y;
+    int64_t N;
+    int64_t K;
+    int32_t group_size;
+} w4_chain_layer;
+
+w4_status w4a16_gemm_chain(const w4_chain_layer* layers, int32_t n_layers, int64_t M,
+                           w4_dtype act_dtype, w4_dtype out_dtype, void* workspace,
+                           size_t workspace_bytes, w4_stream_t stream);
+
+/* Bytes of workspace w4a16_gemm_chain needs on the current device (0 unless 1 <= M <= 8). */
+size_t w4a16_chain_workspace_bytes(int64_t M);
+
+/*
  * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 32 (M <= 64 where the scratch fits)
  * without a caller-supplied workspace.  The pages have no counterpart to this call; it
  * exists for callers that cannot allocate device memory where they run the GEMM, such as
@@ -251,9 +305,13 @@ size_t w4_awq_search_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t gr
  * 148-SM B200; any M > 64) return W4_ERR_UNSUPPORTED; use w4a16_gemm for them.  The
  * first call on a device sets up that device (looks up the array's address, zeroes the
  * array and synchronises the device); make that first call before any stream
- * capture.  Every call on a device shares the one array: calls that may overlap on the
- * GPU (different streams without ordering) race and give wrong results.  The call
- * allocates nothing and frees nothing.
+ * capture.  If the set-up fails the call returns W4_ERR_CUDA and the next call tries it
+ * again.  Every call on a device shares the one array: calls that may overlap on the
+ * GPU (different streams without ordering) race and give wrong results.  A call whose
+ * kernel gave up a bounded wait can leave split-K flags set in the array; when
+ * w4_check_device_error() reports W4_ERR_TIMEOUT it zeroes the array of the current
+ * device again, so later calls start clean.  The call allocates nothing and frees
+ * nothing.
  */
 w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
                              const uint32_t* qweight, const void* scales, const void* zeros,
@@ -271,7 +329,10 @@ w4_status w4_unpack_canonical(const uint32_t* qweight, int64_t N, int64_t K,
 
 /* Synchronises the current device, then reports and clears the device-side error word:
  * W4_ERR_TIMEOUT if a kernel gave up a bounded wait, W4_ERR_DEVICE_ARG if a kernel met
- * an out-of-range g_idx entry, W4_ERR_CUDA if the device reports a CUDA error, W4_OK. */
+ * an out-of-range g_idx entry, W4_ERR_CUDA if the device reports a CUDA error, W4_OK.
+ * On W4_ERR_TIMEOUT it also zeroes the current device's w4a16_gemm_noalloc scratch again
+ * (a timed-out kernel may have left split-K flags in it); workspaces passed to
+ * w4a16_gemm belong to the caller, who zeroes them again. */
 w4_status w4_check_device_error(void);
 
 /* Bound, in nanoseconds, of every wait inside the library's kernels (default 2e9).

@@ -211,13 +211,13 @@ def test_single_layer_config():
 
 
 @pytest.mark.parametrize("M", [1, 8, 32, 64])
-@pytest.mark.parametrize("layer", [0, 2, 3])
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
 def test_llama70b_layers(layer, M):
     skip_without_gpu()
     sampled_case(3, layer, M)
 
 
-@pytest.mark.parametrize("M", [512, 4096])
+@pytest.mark.parametrize("M", [512, 2048, 4096, 8192])
 @pytest.mark.parametrize("layer", [0, 1])
 def test_llama8b_prefill_layers(layer, M):
     skip_without_gpu()
@@ -235,7 +235,14 @@ def test_gptq_act_order_config(M, g):
 def test_chained_layers_in_a_graph(M):
     """Each GEMM reads the previous GEMM's output; launched back to back from a CUDA
     graph, so a kernel that overlaps its predecessor (programmatic dependent launch)
-    must still see the finished activations and leave the shared workspace intact."""
+    must still see the finished activations and leave the shared workspace intact.
+
+    Held to the stated bound (relative L2 1e-3, max-abs 2e-2).  The oracle chain rounds
+    every output to fp16 as the GPU stores it, so the two chains differ only where the
+    GPU's fp32 summation order (about 1e-5 relative here) moves a value across an fp16
+    rounding boundary: a 1-ulp difference (at most 2^-10 relative) on a small fraction of
+    the elements.  Such differences pass through the following layers at about their own
+    relative size, so after six layers the relative L2 stays near 1e-4."""
     skip_without_gpu()
     import torch
     K = N = 1024
@@ -278,4 +285,4 @@ def test_chained_layers_in_a_graph(M):
         graph.replay()
         torch.cuda.synchronize()
         w4.w4_check_device_error()
-        check_y(to_f64(bufs[-1]), ref, "fp16", tol_rel=5e-3)
+        check_y(to_f64(bufs[-1]), ref, "fp16")

@@ -3,9 +3,10 @@
 Some callers cannot allocate device memory where they run the GEMM (plug-ins of
 inference runtimes that forbid allocation after set-up, C callers without a caching
 allocator); this entry point uses the library's fixed per-device scratch instead of a
-caller workspace.  Here it is called through the C ABI and its output is compared with
-the workspace entry point's, twice in a row, since every call reuses the same scratch.
-This file is collected last so a failure here cannot hide the other tests.
+caller workspace.  Here it is called through the C ABI, twice in a row (every call reuses
+the same scratch), and each result is compared element by element with the CPU oracle's
+fp32 product and with the workspace entry point's output.  This file is collected last so
+a failure here cannot hide the other tests.
 """
 import ctypes
 
@@ -30,35 +31,83 @@ def _noalloc_c(X, qw, sc, zr, g, s_inv, Y):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (7, 1536, 2048), (16, 12288, 4096)])
-def test_noalloc_matches_workspace_entry_point_twice(M, N, K):
-    skip_without_gpu()
+def _layer(M, N, K, g=128):
     import torch
-    g = 128
     rng = np.random.default_rng(M * 101 + N + K)
     X, W, s, s_inv = random_layer(rng, M, N, K)
     q, scales, zeros = oracle.quantize_weights(W, s, g)
-    Xd = dev_bits(X, torch.float16)
-    qw = dev(oracle.pack_device(q).view(np.int32))
-    sc = dev_bits(scales, torch.float16)
-    zr = dev_bits(zeros, torch.float16)
-    si = dev(s_inv)
-    Y_ws = to_f64(w4.w4a16_gemm(Xd, qw, sc, zr, g, s_inv=si))
+    d = {"Xd": dev_bits(X, torch.float16), "qw": dev(oracle.pack_device(q).view(np.int32)),
+         "sc": dev_bits(scales, torch.float16), "zr": dev_bits(zeros, torch.float16),
+         "si": dev(s_inv)}
+    Y_ref = oracle.reference_y(X, s_inv, q, scales, zeros, g)
+    return d, Y_ref
+
+
+def _run_noalloc(d, M, N, g=128):
+    import torch
+    Y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    assert _noalloc_c(d["Xd"], d["qw"], d["sc"], d["zr"], g, d["si"], Y) == w4.W4_OK
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    return to_f64(Y)
+
+
+# M = 17..32 (four token tiles) is the largest case the 8 MiB scratch holds on 148 SMs.
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (7, 1536, 2048), (16, 12288, 4096),
+                                   (17, 4096, 4096), (32, 11008, 4096)])
+def test_noalloc_matches_oracle_twice(M, N, K):
+    skip_without_gpu()
+    g = 128
+    d, Y_ref = _layer(M, N, K, g)
+    Y_ws = to_f64(w4.w4a16_gemm(d["Xd"], d["qw"], d["sc"], d["zr"], g, s_inv=d["si"]))
     for _ in range(2):
-        Y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
-        assert _noalloc_c(Xd, qw, sc, zr, g, si, Y) == w4.W4_OK
-        torch.cuda.synchronize()
-        w4.w4_check_device_error()
-        check_y(to_f64(Y), Y_ws, "fp16")
+        Y = _run_noalloc(d, M, N, g)
+        check_y(Y, Y_ref, "fp16")          # parity with the oracle
+        check_y(Y, Y_ws, "fp16")           # and with the workspace entry point
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
+    """M = 33 needs eight token tiles of split-K slots (about 9.7 MB on 148 SMs): more
+    than the fixed scratch, so the scratch-size check (not the M <= 64 limit) refuses it."""
     skip_without_gpu()
     import torch
     K, N, g = 1024, 256, 128
-    X = torch.zeros(65, K, dtype=torch.float16, device="cuda")
+    M = 33
+    X = torch.zeros(M, K, dtype=torch.float16, device="cuda")
     qw = torch.zeros(N * K // 8, dtype=torch.int32, device="cuda")
     sc = torch.ones(K // g, N, dtype=torch.float16, device="cuda")
-    Y = torch.empty(65, N, dtype=torch.float16, device="cuda")
+    Y = torch.empty(M, N, dtype=torch.float16, device="cuda")
     s_inv = torch.ones(K, dtype=torch.float32, device="cuda")
     assert _noalloc_c(X, qw, sc, sc, g, s_inv, Y) == w4.W4_ERR_UNSUPPORTED
+    # the same sizes through the workspace entry point are fine
+    w4.w4a16_gemm(X, qw, sc, sc, g, s_inv=s_inv, Y=Y)
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+
+
+def test_noalloc_recovers_after_a_timed_out_call():
+    """With the wait bound at its 1 us minimum, a completing CTA gives up waiting for the
+    split-K shares of its band (a bounded wait; nothing faults) and leaves flags set in the
+    shared scratch.  w4_check_device_error reports the timeout and zeroes the scratch
+    again, so the next calls, with the normal bound, match the oracle."""
+    skip_without_gpu()
+    import torch
+    M, N, K, g = 16, 12288, 4096, 128
+    d, Y_ref = _layer(M, N, K, g)
+    w4.w4_check_device_error()                     # start clean
+    timeouts = 0
+    try:
+        w4.w4_set_wait_limit_ns(1000)
+        for _ in range(5):
+            Y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+            assert _noalloc_c(d["Xd"], d["qw"], d["sc"], d["zr"], g, d["si"], Y) == w4.W4_OK
+            try:
+                w4.w4_check_device_error()
+            except w4.W4Error as e:
+                assert e.status == w4.W4_ERR_TIMEOUT
+                timeouts += 1
+    finally:
+        w4.w4_set_wait_limit_ns(2_000_000_000)
+    assert timeouts > 0, "the 1 us bound never expired"
+    for _ in range(2):
+        check_y(_run_noalloc(d, M, N, g), Y_ref, "fp16")
