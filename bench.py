@@ -181,6 +181,7 @@ def prepare_weights(w4, torch, n_layers=N_LAYERS):
         s = torch.from_numpy(li.s).cuda()
         qw, sc, zr = w4.w4_quantize_pack(W, s, li.group_size)
         projs.append({"li": li, "W": W, "s": s, "s_inv": torch.from_numpy(li.s_inv).cuda(),
+                      "s_inv_chain": torch.from_numpy(workloads.chain_s_inv(li.s_inv)).cuda(),
                       "bytes": workloads.effective_weight_bytes(li.N, li.K, li.group_size,
                                                                 False, False)})
         projs[-1]["copies"] = [(qw, sc, zr)] + [(qw.clone(), sc.clone(), zr.clone())
@@ -197,6 +198,54 @@ def make_acts(wl, projs, M, torch):
         xs.append(dev_bits(li.X, torch.float16))
     ys = [torch.empty(M, pr["li"].N, dtype=torch.float16, device="cuda") for pr in projs]
     return xs, ys
+
+
+def chain_layers(w4, torch, projs, M, n_blocks=N_LAYERS):
+    """The decode step as a chain: every block's four projections, each reading an earlier
+    output as workloads.CHAIN_SOURCE defines (block b > 0 reads block b-1's down output),
+    with the stand-in gains folded into s_inv.  Returns (layer dicts, block-0 input, last
+    output)."""
+    wl = workloads.workload(DECODE_CFG)
+    x0 = dev_bits(workloads.make_layer(wl, 0, M=M, with_weights=False).X, torch.float16)
+    layers, prev = [], None
+    for b in range(n_blocks):
+        ys = [torch.empty(M, pr["li"].N, dtype=torch.float16, device="cuda") for pr in projs]
+        for j, pr in enumerate(projs):
+            src, c0 = workloads.CHAIN_SOURCE[j]
+            K = pr["li"].K
+            if src < 0:
+                X = x0 if prev is None else prev
+            else:
+                X = ys[src][:, c0:c0 + K]
+            qw, sc, zr = pr["copies"][b]
+            layers.append({"X": X, "qweight": qw, "scales": sc, "zeros": zr, "group_size": 128,
+                           "s_inv": pr["s_inv_chain"], "Y": ys[j]})
+        prev = ys[3]
+    return layers, x0, prev
+
+
+def run_chain_per_launch(w4, layers):
+    """The same chain as one w4a16_gemm call per projection (programmatic dependent launch
+    between consecutive kernels)."""
+    for d in layers:
+        w4.w4a16_gemm(d["X"], d["qweight"], d["scales"], d["zeros"], 128, s_inv=d["s_inv"], Y=d["Y"])
+
+
+def time_steps(torch, fn, steps, warmup, world=1, clocks=None, w4=None):
+    """Warm-up calls of fn, then `steps` calls captured in one CUDA graph and timed on the
+    device.  Returns (total ms, clock summary)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if w4 is not None:
+        w4.w4_check_device_error()
+    g = capture(torch, lambda: [fn() for _ in range(steps)])
+    torch.cuda.synchronize()
+    ms, clk = time_graph(torch, g, world, clocks)
+    if w4 is not None:
+        w4.w4_check_device_error()
+    del g
+    return ms, clk
 
 
 def run_decode_steps(w4, projs, xs, ys, steps):
@@ -441,21 +490,107 @@ def cpu_oracle_sample(target_s=12.0, sample=None, rows_per_layer=256):
     return total_bytes / total_s / 1e9, total_s, desc
 
 
+def cpu_info():
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count() or 1
+    return model, os.cpu_count() or 1, usable
+
+
+def threaded_sample(threads, rows_per_thread=64):
+    """Per thread, rows_per_thread distinct seeded output rows of every decode layer,
+    quantised by the oracle (prepared once; not timed)."""
+    sample = oracle_sample(rows_per_layer=rows_per_thread * threads)
+    parts = []
+    for t in range(threads):
+        r0, r1 = t * rows_per_thread, (t + 1) * rows_per_thread
+        parts.append([(li, np.ascontiguousarray(q[r0:r1]), np.ascontiguousarray(sc[:, r0:r1]),
+                       np.ascontiguousarray(zr[:, r0:r1]),
+                       workloads.effective_weight_bytes(rows_per_thread, li.K, 128, False, False))
+                      for li, q, sc, zr, _ in sample])
+    return parts
+
+
+def cpu_oracle_threads(parts, target_s=8.0):
+    """The oracle's online path with the output-row (N) loop split over len(parts)
+    threads, each running the oracle on its own rows until target_s has passed (the
+    oracle's C calls release the GIL).  Returns (GB/s of effective weight bytes, seconds)."""
+    import threading
+    import oracle
+    threads = len(parts)
+    done = [0] * threads
+    t_end = [0.0]
+
+    def work(t):
+        b = 0
+        while time.perf_counter() < t_end[0]:
+            for li, q, sc, zr, by in parts[t]:
+                oracle.reference_y(li.X, li.s_inv, q, sc, zr, 128)
+                b += by
+        done[t] = b
+
+    ths = [threading.Thread(target=work, args=(t,)) for t in range(threads)]
+    start = time.perf_counter()
+    t_end[0] = start + target_s
+    for th in ths:
+        th.start()
+    for th in ths:
+        th.join()
+    el = time.perf_counter() - start
+    return sum(done) / el / 1e9, el
+
+
+def threaded_desc(parts, seconds):
+    rows = sum(q.shape[0] for _, q, _, _, _ in parts[0]) // len(parts[0]) * len(parts)
+    return (f"M=1 online path (X*s_inv, dequantise, fp32 product) of the 4 decode layers, "
+            f"output rows split over {len(parts)} threads, {rows} seeded rows per layer, "
+            f"{seconds:.1f} s")
+
+
+def cpu_baseline():
+    """The oracle timed on this host: one thread (the oracle as it stands), and the same
+    path with the output rows split over every usable core."""
+    model, nproc, usable = cpu_info()
+    v1, sec1, desc1 = cpu_oracle_sample(target_s=8.0)
+    threads = max(1, min(usable, 128))
+    parts = threaded_sample(threads)
+    vt, sect = cpu_oracle_threads(parts)
+    return {"value": vt, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": threaded_desc(parts, sect),
+            "single_thread": {"value": v1, "cores": 1, "sample": desc1, "seconds": round(sec1, 2)},
+            "cpu_model": model, "nproc": nproc, "usable_cores": usable}
+
+
 def reference_arm(args, world, rank):
+    """The CPU oracle as the reference arm: its online path on the decode workload, output
+    rows split over every usable core, each step a bounded sample."""
     if rank != 0:
         return
     import oracle
     oracle.lib()
-    sample = oracle_sample()
+    model, nproc, usable = cpu_info()
+    threads = max(1, min(usable, 128))
+    parts = threaded_sample(threads)
     vals = []
     desc = ""
     # each step a bounded sample, so that the whole run takes about two minutes
     per_step = max(0.5, min(12.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_oracle_sample(target_s=per_step, sample=sample)
+        cpu_oracle_threads(parts, target_s=per_step)
     for _ in range(args.steps):
-        v, s, desc = cpu_oracle_sample(target_s=per_step, sample=sample)
+        v, sec = cpu_oracle_threads(parts, target_s=per_step)
         vals.append(v)
+        desc = threaded_desc(parts, sec)
     value = statistics.median(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -463,11 +598,153 @@ def reference_arm(args, world, rank):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": workload_desc(workloads.workload(DECODE_CFG), 1),
                        "sample": desc},
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": desc, "cpu_model": model, "nproc": nproc},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
+
+
+def time_chain(M, steps, warmup, w4, torch, world, projs, clocks=None):
+    """The chained decode step at M tokens through w4a16_gemm_chain (one persistent launch
+    per 32 projections), replayed from a CUDA graph.  Returns (total ms, clocks, launches)."""
+    layers, _, _ = chain_layers(w4, torch, projs, M)
+    ms, clk = time_steps(torch, lambda: w4.w4a16_gemm_chain(layers), steps, warmup, world, clocks, w4)
+    return ms, clk, steps * math.ceil(len(layers) / 32)
+
+
+def time_chain_per_launch(M, steps, warmup, w4, torch, world, projs):
+    layers, _, _ = chain_layers(w4, torch, projs, M)
+    ms, _ = time_steps(torch, lambda: run_chain_per_launch(w4, layers), steps, warmup, world, None, w4)
+    return ms
+
+
+def time_chain_e2e(M, steps, warmup, w4, torch, world, projs):
+    """The chained step through the public call with host buffers: each step copies the
+    block-0 input host->device (pinned), runs the chain and reads the last block's output
+    back device->host, all inside the timed region (eager calls)."""
+    layers, x0, last = chain_layers(w4, torch, projs, M)
+    hx = x0.cpu().pin_memory()
+    hy = torch.empty_like(last, device="cpu").pin_memory()
+
+    def step():
+        x0.copy_(hx, non_blocking=True)
+        w4.w4a16_gemm_chain(layers)
+        hy.copy_(last, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    return ms, hx.numel() * hx.element_size(), hy.numel() * hy.element_size()
+
+
+def rotated_copies(w4, torch, W, s, g, nbytes, symmetric=False, min_copies=2):
+    """Quantise W once and clone the packed weights so that the copies together exceed
+    four times L2 (each timed launch then reads its weights from HBM)."""
+    qw, sc, zr = w4.w4_quantize_pack(W, s, g, symmetric)
+    n = max(min_copies, math.ceil(4 * L2_BYTES / nbytes))
+    return [(qw, sc, zr)] + [(qw.clone(), sc.clone(), None if zr is None else zr.clone())
+                             for _ in range(n - 1)]
+
+
+def time_layer(w4, torch, copies, X, g, s_inv, N, launches=None, perm=None, g_idx=None):
+    """Average time of one w4a16_gemm launch over rotated weight copies (CUDA graph)."""
+    M = X.shape[0]
+    Y = torch.empty(M, N, dtype=torch.float16 if X.dtype == torch.float16 else torch.float32,
+                    device="cuda")
+    n = launches or max(len(copies), 32)
+
+    def run(i):
+        qw, sc, zr = copies[i % len(copies)]
+        w4.w4a16_gemm(X, qw, sc, zr, g, g_idx=g_idx, s_inv=s_inv, Y=Y, perm=perm)
+    for i in range(len(copies)):
+        run(i)
+    torch.cuda.synchronize()
+    graph = capture(torch, lambda: [run(i) for i in range(n)])
+    graph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    graph.replay()
+    b.record()
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    return a.elapsed_time(b) * 1e3 / n
+
+
+def time_config_layers(w4, torch, config_id, Ms, device_weights=False):
+    """Per-launch GB/s of every layer of a decode workload at each M (fresh weights,
+    rotated copies larger than L2)."""
+    wl = workloads.workload(config_id)
+    out = {}
+    for i, L in enumerate(wl.layers):
+        if device_weights:
+            # seeded on the device: these layers hold up to 470 M weights, whose host
+            # generation would dominate the run; the values only need the same distribution
+            gen = torch.Generator(device="cuda").manual_seed(1000 * config_id + i)
+            W = (torch.randn(L.N, L.K, generator=gen, device="cuda") * workloads.W_STD).half()
+            s_np, s_inv_np = workloads.awq_scales(L.K, 0, config_id, i)
+        else:
+            li = workloads.make_layer(wl, i, M=1)
+            W = dev_bits(li.W.view(np.uint16), torch.float16)
+            s_np, s_inv_np = li.s, li.s_inv
+        s = torch.from_numpy(s_np).cuda()
+        s_inv = torch.from_numpy(s_inv_np).cuda()
+        by = workloads.effective_weight_bytes(L.N, L.K, 128, False, False)
+        copies = rotated_copies(w4, torch, W, s, 128, by)
+        del W
+        row = {}
+        for M in Ms:
+            X = dev_bits(workloads.gen_acts(M, L.K, 0, config_id, i), torch.float16)
+            us = time_layer(w4, torch, copies, X, 128, s_inv, L.N)
+            row[str(M)] = {"us": round(us, 3), "gbs": round(by / us / 1e3, 1)}
+        out[f"{L.name} {L.K}x{L.N}"] = row
+        del copies
+        torch.cuda.empty_cache()
+    return out
+
+
+def time_prefill_sweep(w4, torch, peaks, Ms=(512, 2048, 4096, 8192)):
+    out = {}
+    for M in Ms:
+        pf = time_prefill(w4, torch, M=M, iters=3 if M >= 4096 else 5)
+        pf["frac_of_measured_bf16_burst"] = pf["tflops"] / peaks["bf16_tflops"]
+        out[str(M)] = pf
+    return out
+
+
+def time_gptq_sweep(w4, torch, Ms=(1, 16, 1024), gs=(32, 64, 128, 4096)):
+    """The act-order workload (4096 -> 11008, symmetric, g_idx) through the permuted path
+    (w4a16_gemm_perm) at every M and group size: GB/s at M <= 16, TFLOPS at M = 1024."""
+    wl = workloads.workload(ACTORDER_CFG)
+    out = {}
+    for g in gs:
+        li = workloads.make_layer(wl, 0, M=1, group_size=g)
+        W = dev_bits(li.W.view(np.uint16), torch.float16)
+        g_idx = torch.from_numpy(li.g_idx).cuda()
+        pm = w4.w4_actorder_perm(g_idx, g)
+        qw, sc, _ = w4.w4_quantize_pack(W, None, g, True, perm=pm)
+        by = workloads.effective_weight_bytes(li.N, li.K, g, True, True)
+        copies = [(qw, sc, None)] + [(qw.clone(), sc.clone(), None) for _ in range(15)]
+        row = {}
+        for M in Ms:
+            X = dev_bits(workloads.gen_acts(M, li.K, 0, ACTORDER_CFG, 0), torch.float16)
+            us = time_layer(w4, torch, copies, X, g, None, li.N, launches=32 if M > 64 else 64, perm=pm)
+            r = {"us": round(us, 3), "gbs": round(by / us / 1e3, 1)}
+            if M > 64:
+                r["tflops"] = round(workloads.gemm_flops(M, li.N, li.K) / us / 1e6, 1)
+            row[str(M)] = r
+        out[f"g{g}"] = row
+    return out
 
 
 def our_arm(args, world, rank, local):
@@ -479,64 +756,87 @@ def our_arm(args, world, rank, local):
     peaks, peak_src = load_peaks()
     M = 1
     wl, projs, step_bytes = prepare_weights(w4, torch)
+    launches_per_step = N_LAYERS * len(projs)
     clocks = ClockSampler(local)
-    dec = time_decode(M, args.steps, args.warmup, w4, torch, world, wl, projs, step_bytes,
-                      clocks, per_layer=True)
-    t_ms = max_over_ranks(dec["total_ms"], world)
+    # the headline: the chained decode step, one persistent launch per 32 projections
+    t_ms_local, clk, launches = time_chain(M, args.steps, args.warmup, w4, torch, world, projs, clocks)
+    t_ms = max_over_ranks(t_ms_local, world)
     value = world * args.steps * step_bytes / (t_ms * 1e-3) / 1e9
-    # dominant kernel = the decode GEMM (every launch of the timed region is one):
+    # dominant kernel = the layer-sequence kernel (every launch of the timed region is one):
     # achieved = algorithmic bytes per launch / average launch duration on its stream
-    achieved = args.steps * step_bytes / (dec["total_ms"] * 1e-3) / 1e9
-    e2e_ms, h2d, d2h = time_e2e(M, args.steps, args.warmup, w4, torch, world, wl, projs)
+    achieved = args.steps * step_bytes / (t_ms_local * 1e-3) / 1e9
+    e2e_ms, h2d, d2h = time_chain_e2e(M, args.steps, args.warmup, w4, torch, world, projs)
     e2e_val = world * args.steps * step_bytes / (e2e_ms * 1e-3) / 1e9
-
-    extras = {"tokens_per_s_linear_layers": round(1e3 * args.steps / t_ms, 1)}
+    # the same chain as separate launches, and the projections one by one (independent inputs)
+    pl_ms = time_chain_per_launch(M, args.steps, args.warmup, w4, torch, world, projs)
+    dec = time_decode(M, max(3, args.steps // 4), args.warmup, w4, torch, world, wl, projs, step_bytes,
+                      per_layer=True)
+    step_gb = step_bytes / 1e9
+    extras = {
+        "tokens_per_s_linear_layers": round(1e3 * args.steps / t_ms, 1),
+        "roofline_tokens_per_s": round(workloads.roofline_tokens_per_s(peaks["hbm_gbs"], step_gb), 1),
+        "step_per_launch": {"gbs": round(args.steps * step_bytes / (pl_ms * 1e-3) / 1e9, 1),
+                            "ms_per_step": pl_ms / args.steps,
+                            "note": "same chain, one w4a16_gemm launch per projection"},
+        "step_independent_inputs_per_launch": {
+            "gbs": round(max(3, args.steps // 4) * step_bytes / (dec["total_ms"] * 1e-3) / 1e9, 1),
+            "note": "128 w4a16_gemm launches on fixed inputs (no dependencies)"},
+    }
     if not args.quick:
         sweep = {"1": round(value / world, 1)}
+        how = {"1": "chain"}
+        st = max(3, args.steps // 4)
         for m in (2, 4, 8, 16):
-            st = max(3, args.steps // 4)
-            d = time_decode(m, st, args.warmup, w4, torch, world, wl, projs, step_bytes)
-            sweep[str(m)] = round(st * step_bytes / (max_over_ranks(d["total_ms"], world) * 1e-3)
-                                  / 1e9, 1)
+            # the chain holds every layer's activations in shared memory: up to M = 4 at
+            # K = 11008; beyond, the step's 128 GEMMs run as separate launches
+            if m <= 4:
+                ms, _, _ = time_chain(m, st, args.warmup, w4, torch, world, projs)
+                how[str(m)] = "chain"
+            else:
+                ms = time_decode(m, st, args.warmup, w4, torch, world, wl, projs, step_bytes)["total_ms"]
+                how[str(m)] = "per-launch, independent inputs"
+            sweep[str(m)] = round(st * step_bytes / (max_over_ranks(ms, world) * 1e-3) / 1e9, 1)
         extras["decode_sweep_gbs_per_gpu"] = sweep
-        pf = time_prefill(w4, torch)
-        pf["frac_of_measured_bf16_burst"] = pf["tflops"] / peaks["bf16_tflops"]
-        pf["frac_of_spec_2250"] = pf["tflops"] / 2250.0
-        extras["prefill_m4096"] = pf
+        extras["decode_sweep_path"] = how
+        extras["single_layer_4096"] = time_config_layers(w4, torch, 1, (1,))
+        extras["llama70b_layers"] = time_config_layers(w4, torch, 3, (1, 8, 32, 64), device_weights=True)
+        extras["prefill"] = time_prefill_sweep(w4, torch, peaks)
+        extras["prefill_m4096"] = extras["prefill"]["4096"]
+        extras["gptq_actorder_perm"] = time_gptq_sweep(w4, torch)
         extras["quantize_pack"] = time_quantize(w4, torch, projs)
         extras["awq_search"] = time_awq_search(w4, torch)
         # last: its larger workspace may replace the cached one the graphs above captured
         extras["actorder_decode"] = time_actorder(w4, torch)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        v, sec, desc = cpu_oracle_sample()
-        cpu = {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
-               "seconds": round(sec, 2)}
-    # DRAM traffic per launch of the decode kernel, as a ratio to its algorithmic bytes from
-    # one ncu capture of the gate_up launch (48.583 MB read + 0.001 MB written for 47.88 MB
-    # algorithmic: profiles/decode_gate_up_4096x22016_m1.md); the average launch of the step
-    # is scaled by its algorithmic bytes.  Set to None whenever the decode kernel changes.
-    DECODE_TRAFFIC_RATIO = 1.015
-    launches_per_step = N_LAYERS * len(projs)
-    traffic = (DECODE_TRAFFIC_RATIO * step_bytes / launches_per_step) if DECODE_TRAFFIC_RATIO else None
+        cpu = cpu_baseline()
+    # DRAM traffic per launch of the dominant kernel, as a ratio to its algorithmic bytes,
+    # from one ncu capture of that kernel; the step's average launch is scaled by its
+    # algorithmic bytes (traffic grows with the codes streamed).  None until the kernel
+    # as built here has been captured.
+    TRAFFIC_RATIO = None
+    traffic = (TRAFFIC_RATIO * step_bytes / (launches / args.steps)) if TRAFFIC_RATIO else None
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
         "config": {"workload": workload_desc(wl, M) + f"; step = 1 token through {N_LAYERS} "
-                   f"blocks x 4 projections ({N_LAYERS * 4} GEMMs)",
+                   f"blocks x 4 projections ({launches_per_step} GEMMs), each projection fed "
+                   "from the previous output (query slice -> o, gate half -> down; fixed gains "
+                   "in s_inv stand in for the normalisations)",
                    "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of packed weights "
                          "per step (one copy per block)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "peak_source": peak_src, "kernel": "w4a16 decode (stream-K, mma.sync)",
+                     "peak_source": peak_src,
+                     "kernel": "w4a16 layer sequence (persistent, stream-K, mma.sync)",
                      "per_layer": dec["per_layer"]},
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": dec["launches"],
-        "clocks": dec["clocks"],
+        "gpu_launches": launches,
+        "clocks": clk,
         "cpu_baseline": cpu,
     }
     line.update(extras)

@@ -102,6 +102,7 @@ struct DecodeParams {
     int off_xchg;             // byte offset of the MMA-warp exchange buffer
     // byte offsets inside one stage
     int off_x, off_xs, off_sx, off_si, off_sc, off_zr, off_gi, off_desc, stage_bytes;
+    int ldx;                  // row stride of X in elements (read by the layer-sequence kernel)
 };
 
 W4_DEV int unit_begin(const DecodeParams& p, int c) { return c * p.base + min(c, p.rem); }
@@ -655,10 +656,13 @@ W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw,
 // 64-channel block; sums are [segment][sstride].  Consecutive lanes take consecutive
 // 8-channel chunks, so the sums are warp shuffles; a lane takes its chunk for every token
 // (M <= 8 here), loading the chunk's s_inv once and all M activation chunks together.
-template <bool BF16, bool PERM>
+// COHERENT: X was written earlier in the same launch by other CTAs (the layer-sequence
+// kernel), so it is read through L2 (ld.global.cg), with rows p.ldx elements apart.
+template <bool BF16, bool PERM, bool COHERENT = false>
 W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* xr, float* sr, int w,
                           int nw, int lane) {
     const int cpt = p.K / 8;                       // chunks per token
+    const int rpt = COHERENT ? p.ldx / 8 : cpt;    // chunks between consecutive token rows
     const int ss = p.sstride;
     float* s32 = sr;
     float* s64 = s32 + (p.K / 32) * ss;
@@ -709,8 +713,12 @@ W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* x
                 sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
             }
 #pragma unroll
-            for (int m = 0; m < 8; ++m)
-                v[m] = (valid && m < p.M) ? x4[(size_t)m * cpt + c] : make_uint4(0u, 0u, 0u, 0u);
+            for (int m = 0; m < 8; ++m) {
+                if constexpr (COHERENT)
+                    v[m] = (valid && m < p.M) ? __ldcg(x4 + (size_t)m * rpt + c) : make_uint4(0u, 0u, 0u, 0u);
+                else
+                    v[m] = (valid && m < p.M) ? x4[(size_t)m * rpt + c] : make_uint4(0u, 0u, 0u, 0u);
+            }
         }
         const int blk = c >> 3, ch = c & 7;
 #pragma unroll

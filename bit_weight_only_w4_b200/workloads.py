@@ -189,6 +189,36 @@ def make_layer(wl: Workload, layer_index: int, M: int, group_size: Optional[int]
     return LayerInputs(layer.K, layer.N, M, wl.act_dtype, X, W, s, s_call, g, wl.symmetric, gi)
 
 
+# ---- the decode step as a chain of projections ---------------------------------------
+# One transformer block's projections in decode order, each fed from an earlier output.
+# The non-GEMM parts of a block (attention, residual, normalisation, the gated MLP's
+# activation) are not part of the W4A16 path; a fixed stand-in takes their place:
+#   qkv      reads the block's input (the previous block's down output; the seeded X for
+#            the first block);
+#   o        reads the first 4096 values of the qkv output (the query slice stands in for
+#            the attention output);
+#   gate_up  reads the o output;
+#   down     reads the first 11008 values of the gate_up output (the gate half stands in
+#            for silu(gate) * up).
+# CHAIN_SOURCE[j] = (index of the projection whose output is read, -1 for the block
+# input, first column of the slice).
+CHAIN_SOURCE = ((-1, 0), (0, 0), (1, 0), (2, 0))
+
+
+def chain_gain(K: int) -> float:
+    """A fixed per-layer gain standing in for the normalisation before each projection:
+    with W ~ N(0, 0.02^2) a projection of K inputs multiplies the activations' size by
+    about 0.02 sqrt(K), so its input is scaled by the inverse (folded into s_inv, as AWQ
+    folds s^-1 into the preceding normalisation) and values stay O(1) through the chain."""
+    return 1.0 / (W_STD * float(np.sqrt(K)))
+
+
+def chain_s_inv(s_inv: np.ndarray) -> np.ndarray:
+    """s_inv of a projection inside the decode chain: the layer's AWQ s^-1 times its gain."""
+    K = s_inv.shape[0]
+    return (s_inv.astype(np.float32) * np.float32(chain_gain(K))).astype(np.float32)
+
+
 # ---- byte and flop accounting of the measurement -------------------------------------
 def effective_weight_bytes(N: int, K: int, group_size: int, symmetric: bool,
                            has_gidx: bool) -> int:

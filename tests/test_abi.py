@@ -229,11 +229,41 @@ def test_binding_refuses_wrong_dtypes_and_sizes():
         w4.w4_unpack_canonical(qw, N, K, out=qw[:-1])
 
 
+def test_chain_rejects_bad_arguments(L):
+    """w4a16_gemm_chain checks its layer list before any CUDA call."""
+    Lc = w4.ChainLayer
+
+    def layer(**kw):
+        d = dict(X=256, ldx=256, qweight=256, scales=256, zeros=256, s_inv=None, Y=256, N=256,
+                 K=256, group_size=128)
+        d.update(kw)
+        return Lc(**d)
+
+    def call(layers, M=1, act=0, out=0):
+        arr = (Lc * len(layers))(*layers)
+        return L.w4a16_gemm_chain(arr, len(layers), M, act, out, ctypes.c_void_p(256), 1 << 30, None)
+
+    assert L.w4a16_gemm_chain(None, 1, 1, 0, 0, None, 0, None) == w4.W4_ERR_INVALID_ARG
+    assert call([layer()], M=9) == w4.W4_ERR_UNSUPPORTED          # one token tile only
+    assert call([layer()], act=2) == w4.W4_ERR_INVALID_ARG        # fp32 activations
+    assert call([layer(ldx=128)]) == w4.W4_ERR_INVALID_ARG        # rows shorter than K
+    assert call([layer(ldx=260)]) == w4.W4_ERR_INVALID_ARG        # rows not 16-byte apart
+    assert call([layer(X=0)]) == w4.W4_ERR_INVALID_ARG            # NULL activations
+    assert call([layer(X=258)]) == w4.W4_ERR_INVALID_ARG          # misaligned
+    assert call([layer(N=8)]) == w4.W4_ERR_UNSUPPORTED            # N % 16
+    assert call([layer(), layer(group_size=32)]) == w4.W4_ERR_UNSUPPORTED   # two group modes
+    assert call([layer(K=65536, ldx=65536)], M=8) == w4.W4_ERR_UNSUPPORTED  # X' not resident
+    assert call([], M=1) == w4.W4_OK                                 # nothing to do
+    assert L.w4a16_chain_workspace_bytes(0) == 0 and L.w4a16_chain_workspace_bytes(9) == 0
+
+
 def test_library_builds_without_warnings(L):
     """nvcc's log of the in-tree build holds no warning (an unused function, a narrowing
     conversion, a missing return...).  ptxas reports no spill in the one-token-tile decode
-    kernels (M <= 8), the prefill kernels and the quantiser, and at most 64 bytes a thread
-    in the multi-tile decode kernels, which run at a 96-register cap."""
+    kernels (M <= 8), the fp16 layer-sequence kernel with 128-multiple groups (the decode
+    step's), the prefill kernels and the quantiser, and at most 64 bytes a thread in the
+    multi-tile decode kernels and the other layer-sequence kernels, which run at a
+    96-register cap."""
     log = open(os.path.join(os.path.dirname(w4.LIB_PATH), "build.log")).read()
     assert "warning" not in log.lower()
     name, seen = None, {}
@@ -246,7 +276,8 @@ def test_library_builds_without_warnings(L):
             seen[name] = (int(m.group(1)), int(m.group(2)))
     assert seen
     for fn, (st, ld) in seen.items():
-        strict = ("decode_kernelILi1E" in fn or "prefill_kernel" in fn or "quantize" in fn)
+        strict = ("decode_kernelILi1E" in fn or "prefill_kernel" in fn or "quantize" in fn or
+                  "chain_kernelILb0ELi0E" in fn)
         limit = 0 if strict else 64
         assert st <= limit and ld <= limit, (fn, st, ld)
 

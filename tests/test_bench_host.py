@@ -68,12 +68,17 @@ def test_our_arm_prints_every_contract_key(monkeypatch, capsys):
     projs = [{"bytes": 1_000_000} for _ in wl.layers]
     step_bytes = bench.N_LAYERS * 4_000_000
     monkeypatch.setattr(bench, "prepare_weights", lambda w4, torch: (wl, projs, step_bytes))
+    clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    monkeypatch.setattr(bench, "time_chain", lambda *a, **k: (100.0, clk, 10 * 4))
+    monkeypatch.setattr(bench, "time_chain_e2e", lambda *a, **k: (200.0, 32768, 98304))
+    monkeypatch.setattr(bench, "time_chain_per_launch", lambda *a, **k: 150.0)
     monkeypatch.setattr(bench, "time_decode", lambda *a, **k: {
-        "total_ms": 100.0, "launches": 10 * bench.N_LAYERS * len(projs),
-        "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+        "total_ms": 40.0, "launches": 3 * bench.N_LAYERS * len(projs), "clocks": None,
         "per_layer": {"qkv": 10.0}})
-    monkeypatch.setattr(bench, "time_e2e", lambda *a, **k: (200.0, 32768, 98304))
     monkeypatch.setattr(bench, "cpu_oracle_sample", lambda *a, **k: (0.04, 12.0, "stub"))
+    monkeypatch.setattr(bench, "threaded_sample", lambda threads: [[None]] * threads)
+    monkeypatch.setattr(bench, "cpu_oracle_threads", lambda parts, target_s=8.0: (0.04 * len(parts), 8.0))
+    monkeypatch.setattr(bench, "threaded_desc", lambda parts, sec: "stub threads")
     monkeypatch.setattr(bench, "load_peaks", lambda: ({"hbm_gbs": 6000.0, "bf16_tflops": 1600.0}, "measured"))
     import bit_weight_only_w4_b200 as w4
     monkeypatch.setattr(w4, "LIB_PATH", __file__)       # "built": no build attempted
@@ -94,6 +99,9 @@ def test_our_arm_prints_every_contract_key(monkeypatch, capsys):
     e = line["e2e"]
     assert e["h2d_bytes_per_step"] == 32768 and e["d2h_bytes_per_step"] == 98304
     assert e["value"] == 10 * step_bytes / 0.2 / 1e9
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
-    assert line["gpu_launches"] == 10 * bench.N_LAYERS * 4
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == 0.04 * cb["cores"]
+    assert cb["single_thread"]["cores"] == 1 and "cpu_model" in cb and cb["nproc"] >= 1
+    assert line["gpu_launches"] == 10 * 4
+    assert line["step_per_launch"]["ms_per_step"] == 15.0
     assert "workload" in line["config"]

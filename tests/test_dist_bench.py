@@ -55,8 +55,9 @@ def test_reference_arm_prints_from_rank_zero_only(capsys, monkeypatch):
     class Args:
         gpus, steps, warmup = 2, 1, 3
     calls = []
-    monkeypatch.setattr(bench, "oracle_sample", lambda *a, **k: calls.append("sample") or [])
-    monkeypatch.setattr(bench, "cpu_oracle_sample", lambda **k: (1.0, 0.1, "stub sample"))
+    monkeypatch.setattr(bench, "threaded_sample", lambda *a, **k: calls.append("sample") or [[None]])
+    monkeypatch.setattr(bench, "cpu_oracle_threads", lambda parts, target_s=8.0: (1.0, 0.1))
+    monkeypatch.setattr(bench, "threaded_desc", lambda parts, sec: "stub sample")
     bench.reference_arm(Args(), 2, 1)
     assert capsys.readouterr().out == "" and calls == []
     bench.reference_arm(Args(), 2, 0)
