@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libw4a16.so")
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA, W4_ERR_TIMEOUT, W4_ERR_DEVICE_ARG = range(6)
 W4_F16, W4_BF16, W4_F32 = 0, 1, 2
+W4_FP4_NVFP4, W4_FP4_MXFP4 = 0, 1
+FP4_BLOCK = {W4_FP4_NVFP4: 16, W4_FP4_MXFP4: 32}
 
 _lib = None
 _lib_lock = threading.Lock()
@@ -79,6 +81,12 @@ def lib():
         L.w4_awq_search.restype = st
         L.w4_awq_search_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32]
         L.w4_awq_search_workspace_bytes.restype = sz
+        L.w4_fp4_quantize_pack.argtypes = [vp, st, i64, i64, st, vp, vp, vp, vp]
+        L.w4_fp4_quantize_pack.restype = st
+        L.w4a16_fp4_gemm.argtypes = [vp, st, i64, i64, i64, vp, vp, vp, st, vp, st, vp, sz, vp]
+        L.w4a16_fp4_gemm.restype = st
+        L.w4a16_fp4_workspace_bytes.argtypes = [i64, i64, i64, st]
+        L.w4a16_fp4_workspace_bytes.restype = sz
         L.w4a16_gemm_chain.argtypes = [ctypes.POINTER(ChainLayer), i32, i64, st, st, vp, sz, vp]
         L.w4a16_gemm_chain.restype = st
         L.w4a16_chain_workspace_bytes.argtypes = [i64]
@@ -420,6 +428,81 @@ def w4a16_gemm_noalloc(X, qweight, scales, zeros, group_size=128, g_idx=None, s_
                                       _ptr(s_inv), _ptr(Y), _dtype_code(Y.dtype),
                                       _stream_handle(stream, dev))
     _check(st, "w4a16_gemm_noalloc")
+    return Y
+
+
+def _fp4_format(fmt):
+    if fmt in ("nvfp4", W4_FP4_NVFP4):
+        return W4_FP4_NVFP4
+    if fmt in ("mxfp4", W4_FP4_MXFP4):
+        return W4_FP4_MXFP4
+    raise ValueError(f"unknown FP4 format {fmt!r} (nvfp4 or mxfp4)")
+
+
+def w4_fp4_quantize_pack(W, fmt="nvfp4", qweight=None, block_scales=None, tensor_scale=None,
+                         stream=None):
+    """Quantise W [N,K] (fp16/bf16) to NVFP4 or MXFP4.  Returns (qweight int32 [N*K/8]
+    in the device layout, block_scales uint8 [K/B, N], tensor_scale fp32 [1] or None)."""
+    torch = _torch()
+    f = _fp4_format(fmt)
+    B = FP4_BLOCK[f]
+    _matrix(W, "W")
+    _expect(W, "W", _f16s())
+    N, K = W.shape
+    if K % B != 0:
+        raise ValueError(f"K = {K} must be a multiple of the block ({B})")
+    _expect(qweight, "qweight", _words(), numel=N * K // 8)
+    _expect(block_scales, "block_scales", (torch.uint8,), shape=(K // B, N))
+    _expect(tensor_scale, "tensor_scale", (torch.float32,), numel=1)
+    dev = _need_cuda(W, qweight, block_scales, tensor_scale)
+    if qweight is None:
+        qweight = torch.empty(N * K // 8, dtype=torch.int32, device=dev)
+    if block_scales is None:
+        block_scales = torch.empty(K // B, N, dtype=torch.uint8, device=dev)
+    if f == W4_FP4_NVFP4 and tensor_scale is None:
+        tensor_scale = torch.empty(1, dtype=torch.float32, device=dev)
+    if f == W4_FP4_MXFP4:
+        tensor_scale = None
+    with _DeviceGuard(dev):
+        st = lib().w4_fp4_quantize_pack(_ptr(W), _dtype_code(W.dtype), N, K, f, _ptr(qweight),
+                                        _ptr(block_scales), _ptr(tensor_scale), _stream_handle(stream, dev))
+    _check(st, "w4_fp4_quantize_pack")
+    return qweight, block_scales, tensor_scale
+
+
+def w4a16_fp4_workspace_bytes(M, N, K, fmt="nvfp4"):
+    return int(lib().w4a16_fp4_workspace_bytes(int(M), int(N), int(K), _fp4_format(fmt)))
+
+
+def w4a16_fp4_gemm(X, qweight, block_scales, tensor_scale=None, fmt="nvfp4", out_dtype=None, Y=None,
+                   workspace=None, stream=None):
+    """Y = X @ What^T with NVFP4 / MXFP4 weights from w4_fp4_quantize_pack (fp16 X)."""
+    torch = _torch()
+    f = _fp4_format(fmt)
+    B = FP4_BLOCK[f]
+    _matrix(X, "X")
+    _expect(X, "X", _f16s())
+    M, K = X.shape
+    if K % B != 0:
+        raise ValueError(f"K = {K} must be a multiple of the block ({B})")
+    N = block_scales.shape[1]
+    _expect(qweight, "qweight", _words(), numel=N * K // 8)
+    _expect(block_scales, "block_scales", (torch.uint8,), shape=(K // B, N))
+    _expect(tensor_scale, "tensor_scale", (torch.float32,), numel=1)
+    _expect(Y, "Y", (torch.float16, torch.bfloat16, torch.float32), shape=(M, N))
+    dev = _need_cuda(X, qweight, block_scales, tensor_scale, Y, workspace)
+    out_dtype = out_dtype or (Y.dtype if Y is not None else X.dtype)
+    if Y is None:
+        Y = torch.empty(M, N, dtype=out_dtype, device=dev)
+    with _DeviceGuard(dev):
+        need = w4a16_fp4_workspace_bytes(M, N, K, f) if M > 0 else 0
+        if workspace is None and need > 0:
+            workspace = workspace_for(dev, need)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib().w4a16_fp4_gemm(_ptr(X), _dtype_code(X.dtype), M, N, K, _ptr(qweight), _ptr(block_scales),
+                                  _ptr(tensor_scale), f, _ptr(Y), _dtype_code(Y.dtype), _ptr(workspace),
+                                  ws_bytes, _stream_handle(stream, dev))
+    _check(st, "w4a16_fp4_gemm")
     return Y
 
 

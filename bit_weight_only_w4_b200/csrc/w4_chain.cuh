@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(w4d::Cfg<1>::threads, 1)
                         desc[0] = make_int4(a0, na, tb, g_first);
                         desc[1] = make_int4(kg[0], kg[1], kg[2], kg[3]);
                         desc[2] = make_int4(kg[4], kg[5], kg[6], kg[7]);
-                        const uint32_t bytes = na * tb * 512 + p.ngs * 256 * (p.zeros ? 2 : 1);
+                        const uint32_t bytes = na * tb * 512 + p.ngs * p.srow_bytes * (p.zeros ? 2 : 1);
                         mbar_arrive_expect_tx(&full[r.s], bytes);
                         bulk_g2s_hint(st, p.qw + 128 * ((size_t)kTilesPerBand * p.KA * band + (size_t)a0 * tb),
                                       na * tb * 512, &full[r.s], policy);

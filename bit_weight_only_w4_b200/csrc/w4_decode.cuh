@@ -39,6 +39,7 @@
 //               (deterministic, no atomics).
 #pragma once
 #include "w4_common.cuh"
+#include "w4_fp4.cuh"
 
 namespace w4d {
 
@@ -51,6 +52,8 @@ enum : int {
     kModeAtom = 1,   // group size a multiple of 64: folds at 64-channel boundaries
     kModeG32 = 2,    // group size 32: folds every 32 channels
     kModeGidx = 3,   // act-order g_idx: the scale is folded into each fp16 weight
+    kModeNvfp4 = 4,  // NVFP4 weights: E2M1 decoded to fp16, E4M3 block scale per 16 channels
+    kModeMxfp4 = 5,  // MXFP4 weights: E2M1 decoded to fp16, power-of-two scale per 32 channels
 };
 
 template <int NT>
@@ -103,6 +106,8 @@ struct DecodeParams {
     // byte offsets inside one stage
     int off_x, off_xs, off_sx, off_si, off_sc, off_zr, off_gi, off_desc, stage_bytes;
     int ldx;                  // row stride of X in elements (read by the layer-sequence kernel)
+    int srow_bytes;           // bytes of one staged scale row: 256 (fp16 x 128), 128 (FP4 bytes)
+    const float* tscale;      // NVFP4 tensor scale (device fp32), else null
 };
 
 W4_DEV int unit_begin(const DecodeParams& p, int c) { return c * p.base + min(c, p.rem); }
@@ -511,6 +516,82 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
                     zero_acc<NT, TPW>(c);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) S[nt] = make_float2(0.0f, 0.0f);
+                }
+            }
+        }
+    }
+}
+
+// FP4 weights: two E2M1 codes of one A-operand register become two exact fp16 values in
+// one hardware conversion (the byte holds the register's first column in its low
+// nibble); the MMA sums each scale block's products and the block's scale multiplies
+// that partial in fp32.  Nibbles i and i+4 of a device-layout word are the register's
+// two columns, so the bytes are (n0|n4), (n2|n6) from the word and (n1|n5), (n3|n7)
+// from the word shifted by 4.
+W4_DEV void unpack_fp4(uint32_t w, uint32_t (&a)[4]) {
+    const uint32_t zx = (w & 0x0F0Fu) | ((w >> 12) & 0xF0F0u);
+    const uint32_t zy = ((w >> 4) & 0x0F0Fu) | ((w >> 16) & 0xF0F0u);
+    a[0] = w4f::e2m1x2_to_h2(zx & 0xFFu);
+    a[1] = w4f::e2m1x2_to_h2(zy & 0xFFu);
+    a[2] = w4f::e2m1x2_to_h2((zx >> 8) & 0xFFu);
+    a[3] = w4f::e2m1x2_to_h2((zy >> 8) & 0xFFu);
+}
+
+// Scale of one staged block-scale byte: E4M3 (NVFP4) or 2^(byte - 127) (MXFP4; the
+// byte 0, 2^-127, reads as 0: such a block's weights are below 2^-124).
+template <int MODE>
+W4_DEV float fp4_block_scale(uint32_t byte) {
+    if constexpr (MODE == kModeNvfp4) return w4f::e4m3_to_f32(byte);
+    else return __int_as_float(byte << 23);
+}
+
+// gs: the NVFP4 tensor scale, folded into every block scale (1 for MXFP4).
+template <int NT, int TPW, int MODE>
+W4_DEV void consume_fp4(const StageView& v, const Lane& L, int t0, int ab, int ae, float gs,
+                        float (&acc)[TPW][NT][4]) {
+    constexpr int B = MODE == kModeNvfp4 ? 16 : 32;   // channels per scale block
+    const unsigned char* wl = v.codes + t0 * 512 + L.lane * 16;
+#pragma unroll 1
+    for (int a = ab; a < ae; ++a) {
+        uint4 w[TPW];
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt) w[tt] = ld_u128(wl + (a * v.tb + tt) * 512);
+        const unsigned char* xa = v.x + a * 128;
+        float c[TPW][NT][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t b0[NT], b1[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                b0[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + L.xlo[j]);
+                b1[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + L.xhi[j]);
+            }
+            const bool first = B == 16 || (j & 1) == 0;
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt) {
+                uint32_t af[4];
+                unpack_fp4(word_j<TPW>(w[tt], j), af);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (first) mma_16816_z<false>(c[tt][nt], af, b0[nt], b1[nt]);
+                    else mma_16816<false>(c[tt][nt], af, b0[nt], b1[nt]);
+                }
+            }
+            if (B == 16 || (j & 1)) {
+                // the block's staged scale row, rows r0 / r1 of each tile
+                const unsigned char* srow = v.sc + ((64 * (v.a0 + a) + 16 * j) / B - v.gfirst) * 128;
+#pragma unroll
+                for (int tt = 0; tt < TPW; ++tt) {
+                    const int r0 = 16 * (t0 + tt) + L.g8;
+                    const float s0 = fp4_block_scale<MODE>(srow[r0]) * gs;
+                    const float s1 = fp4_block_scale<MODE>(srow[r0 + 8]) * gs;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        acc[tt][nt][0] = fmaf(s0, c[tt][nt][0], acc[tt][nt][0]);
+                        acc[tt][nt][1] = fmaf(s0, c[tt][nt][1], acc[tt][nt][1]);
+                        acc[tt][nt][2] = fmaf(s1, c[tt][nt][2], acc[tt][nt][2]);
+                        acc[tt][nt][3] = fmaf(s1, c[tt][nt][3], acc[tt][nt][3]);
+                    }
                 }
             }
         }
@@ -1034,7 +1115,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                     uint32_t bytes = na * tb * 512;
                     if (!p.xres) bytes += C::aps * p.M * 128 + (p.s_inv ? na * 256 : 0);
                     if (GIDX) bytes += na * 256;
-                    else bytes += p.ngs * 256 * (p.zeros ? 2 : 1);
+                    else bytes += p.ngs * (MODE == kModeNvfp4 || MODE == kModeMxfp4 ? 128 : 256) * (p.zeros ? 2 : 1);
                     mbar_arrive_expect_tx(&full[r.s], bytes);
                     bulk_g2s_hint(st, p.qw + 128 * ((size_t)kTilesPerBand * p.KA * band + (size_t)a0 * tb),
                                   na * tb * 512, &full[r.s], policy);
@@ -1162,6 +1243,8 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                     v.kin = kg.x;
                     v.grow = kg.y;
                     if constexpr (GIDX) consume_gidx<NT, TPW>(v, p, L, band, t0, ab, ae, st + p.off_gi, acc);
+                    else if constexpr (MODE == kModeNvfp4 || MODE == kModeMxfp4)
+                        consume_fp4<NT, TPW, MODE>(v, L, t0, ab, ae, p.tscale ? __ldg(p.tscale) : 1.0f, acc);
                     else consume<NT, TPW, BF16, MODE>(v, L, t0, ab, ae, g, acc);
                 }
                 __syncwarp();

@@ -7,22 +7,26 @@
 // tensor cores and the next tiles are staged while the current ones are multiplied
 // ("Kernel Execution: Marlin vs. ExLlamaV2 INT4 GEMM Micro-Architecture", items 1-3).
 //
-// Persistent CTAs (one per SM) walk tiles of 256 output rows x 128 tokens of
+// Persistent CTAs (one per SM) walk tiles of 128 output rows x 256 tokens of
 // Y^T = What * X'^T (CTA t takes tiles t, t + gridDim.x, ...), 16 warps in four warpgroups:
 //   warp 0      TMA: activation tile (2-D tensor map, 128B swizzle) + packed weight tiles
-//               (1-D bulk copies) + zero-point rows into a 5-slot load ring;
+//               of one 128-row band (1-D bulk copy) + zero-point rows into a 4-slot load
+//               ring;
 //   warp 1      allocates tensor memory and issues tcgen05.mma (one elected lane): A = the
-//               dequantised weights of one 128-row half (K-major, 128B swizzle, shared
-//               memory), B = the activations, D = fp32 in tensor memory; two 128 x 128 x 16
-//               MMAs per 16-deep step, one per half;
+//               dequantised weights (K-major, 128B swizzle, shared memory), B = the
+//               activations, D = fp32 in tensor memory; one 128 x 256 x 16 MMA per 16-deep
+//               step;
 //   warps 2-7   unpack the packed tiles into exact integers q - z (fp16/bf16) in the
 //               swizzled A layout, into a 2-slot ring of their own (the load ring runs
 //               further ahead than the dequantised tiles need to);
 //   warps 8-15  epilogue: after each quantisation group the MMA warp hands over that
 //               group's fp32 partial tile (two tensor-memory buffers, ping-pong); each
-//               thread owns one output row of one half, multiplies the partial by the
-//               row's group scale and adds it to register accumulators; at the tile's end
-//               it stores Y through a staging buffer.
+//               thread owns one output row and one 128-token half, multiplies the partial
+//               by the row's group scale and adds it to register accumulators; at the
+//               tile's end it stores Y through a staging buffer.
+// Each dequantised 128 x 64 tile serves 256 tokens: per MAC the dequant work and the
+// shared-memory traffic (operand reads plus the dequantised and TMA writes) are lower
+// than with 256 rows x 128 tokens, which the earlier tiling used.
 // With act-order g_idx the scale is folded into fp16 weights instead and the whole K
 // accumulates in one tensor-memory buffer.
 #pragma once
@@ -30,11 +34,10 @@
 
 namespace w4p {
 
-constexpr int BN = 256;        // output rows per CTA: two 128-row halves (MMA M = 128 each)
-constexpr int BH = 128;        // rows per half
-constexpr int BM = 128;        // tokens per CTA (MMA N)
+constexpr int BN = 128;        // output rows per tile (MMA M)
+constexpr int BM = 256;        // tokens per tile (MMA N)
 constexpr int BK = 64;         // input channels per stage (one 128-byte swizzle row)
-constexpr int kLoadStages = 5;  // activations, codes, zero points: the copies run this far ahead
+constexpr int kLoadStages = 4;  // activations, codes, zero points: the copies run this far ahead
 constexpr int kDeqStages = 2;   // dequantised weight tiles (double-buffered)
 constexpr int kThreads = 512;  // producer, MMA, 6 dequant, 8 epilogue warps (4 warpgroups)
 constexpr int kDequantWarps = 6;
@@ -47,23 +50,22 @@ constexpr int kLaunchRegs = 128;
 constexpr int kRegsLow = 80;
 constexpr int kRegsHigh = 176;
 static_assert(2 * 128 * kRegsLow + 2 * 128 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
-constexpr int kTmemCols = 512; // two fp32 partial buffers x two halves x BM columns
-constexpr int kYChunk = 32;    // tokens per pass of the output staging buffer
+constexpr int kTmemCols = 512; // two fp32 partial buffers x BM columns
+constexpr int kYChunk = 32;    // tokens of each token half per pass of the output staging buffer
 
-constexpr int kAHalf = BH * BK * 2;    // 16 KB: one half's dequantised operand tile
-constexpr int kABytes = 2 * kAHalf;    // 32 KB
-constexpr int kBBytes = BM * BK * 2;   // 16 KB
-constexpr int kPBytes = BN * BK / 2;   // 8 KB packed codes (two 128-row bands)
+constexpr int kABytes = BN * BK * 2;   // 16 KB dequantised operand tile
+constexpr int kBBytes = BM * BK * 2;   // 32 KB activation tile
+constexpr int kPBytes = BN * BK / 2;   // 4 KB packed codes (one 128-row band)
 constexpr int kZBytes = 2 * BN * 2;    // zero-point rows of up to two groups
 constexpr int kStageBytes = kABytes + kBBytes + kPBytes + kZBytes;
 
 struct SmemLayout {
-    static constexpr int a = 0;                              // kDeqStages x 32 KB (1024-aligned)
-    static constexpr int b = a + kDeqStages * kABytes;       // kLoadStages x 16 KB
-    static constexpr int pk = b + kLoadStages * kBBytes;     // kLoadStages x 8 KB
-    static constexpr int zr = pk + kLoadStages * kPBytes;    // kLoadStages x 1 KB
-    static constexpr int y = zr + kLoadStages * kZBytes;     // output staging: kYChunk x BN fp32
-    static constexpr int bars = y + kYChunk * BN * 4;        // barriers
+    static constexpr int a = 0;                              // kDeqStages x 16 KB (1024-aligned)
+    static constexpr int b = a + kDeqStages * kABytes;       // kLoadStages x 32 KB
+    static constexpr int pk = b + kLoadStages * kBBytes;     // kLoadStages x 4 KB
+    static constexpr int zr = pk + kLoadStages * kPBytes;    // kLoadStages x 512 B
+    static constexpr int y = zr + kLoadStages * kZBytes;     // output staging: 2 x kYChunk x BN fp32
+    static constexpr int bars = y + 2 * kYChunk * BN * 4;    // barriers
     static constexpr int nbars = 2 * kLoadStages + 2 * kDeqStages + 4 + 1;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int flags = tmem_slot + 8;
@@ -149,11 +151,11 @@ W4_DEV uint64_t sw128_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor: fp32 accumulator, A/B fp16 (0) or bf16 (1), both K-major,
-// N = BM tokens, M = BH rows (one half; a single-CTA MMA is at most 128 rows).
+// N = BM tokens, M = BN rows (a single-CTA MMA is at most 128 rows and 256 columns).
 W4_DEV uint32_t mma_idesc(bool bf16) {
     const uint32_t fmt = bf16 ? 1u : 0u;
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(BM >> 3) << 17) |
-           ((uint32_t)(BH >> 4) << 24);
+           ((uint32_t)(BN >> 4) << 24);
 }
 
 // Per-warpgroup register limits (executed by all 128 threads of a warpgroup).  An increase
@@ -262,25 +264,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
                 const int rb = t % nbands;
                 const int n0 = rb * BN, m0 = (t / nbands) * BM;
-                int th[2];                                   // tiles of each half
-                for (int h = 0; h < 2; ++h) th[h] = max(0, min(BH / 16, p.tiles - (n0 + h * BH) / 16));
+                const int th = max(0, min(BN / 16, p.tiles - n0 / 16));   // 16-row tiles
                 const int zgroups = (!GIDX && p.zeros) ? (g == 32 ? 2 : 1) : 0;
-                const uint32_t bytes = kBBytes + (th[0] + th[1]) * (512 + zgroups * 32);
+                const uint32_t bytes = kBBytes + th * (512 + zgroups * 32);
                 for (int kt = 0; kt < KT; ++kt, ++gst) {
                     const int s = gst % kLoadStages, ph = (gst / kLoadStages) & 1;
                     if (gst >= kLoadStages && !wait_or_abort(&empty[s], ph ^ 1, abort_flag)) break;
                     mbar_arrive_expect_tx(&full[s], bytes);
-                    for (int h = 0; h < 2; ++h) {
-                        if (th[h] == 0) continue;
-                        const int band = 2 * rb + h;
-                        bulk_g2s(smem + L::pk + s * kPBytes + h * (kPBytes / 2),
-                                 p.qw + 128 * ((size_t)8 * p.KA * band + (size_t)kt * th[h]), th[h] * 512,
-                                 &full[s]);
-                        for (int zg = 0; zg < zgroups; ++zg)
-                            bulk_g2s(smem + L::zr + s * kZBytes + zg * BN * 2 + h * BH * 2,
-                                     p.zeros + (size_t)((kt * BK) / g + zg) * p.N + n0 + h * BH, th[h] * 32,
-                                     &full[s]);
-                    }
+                    bulk_g2s(smem + L::pk + s * kPBytes, p.qw + 128 * ((size_t)8 * p.KA * rb + (size_t)kt * th),
+                             th * 512, &full[s]);
+                    for (int zg = 0; zg < zgroups; ++zg)
+                        bulk_g2s(smem + L::zr + s * kZBytes + zg * BN * 2,
+                                 p.zeros + (size_t)((kt * BK) / g + zg) * p.N + n0, th * 32, &full[s]);
                     if (!waited) {
                         pdl_wait();   // activations may come from the preceding kernel
                         waited = true;
@@ -296,12 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         // the whole warp runs the loop (its values stay warp-uniform); one elected lane
-        // issues each MMA and commit.  Per 16-channel step: one 128x128x16 MMA per half,
-        // both against the same activation tile.
+        // issues each MMA and commit.  Per 16-channel step: one 128x256x16 MMA.
         const bool leader = elect_one();
         const uint32_t idesc = mma_idesc(BF16 && !GIDX);
-        // descriptors of slot 0 of each ring; slot s, half h and 16-channel step j are
-        // s * (tile bytes) + h * kAHalf + 32 j bytes further (>> 4 in the descriptors)
+        // descriptors of slot 0 of each ring; slot s and 16-channel step j are
+        // s * (tile bytes) + 32 j bytes further (>> 4 in the descriptors)
         const uint64_t a_desc0 = sw128_desc(smem_u32(smem + L::a));
         const uint64_t b_desc0 = sw128_desc(smem_u32(smem + L::b));
         // group boundaries: every spg stages (g a multiple of 64), twice per stage
@@ -339,14 +333,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                         }
                     }
-                    const uint32_t dcol = tmem_base + (uint32_t)((grp_i & 1) * 2 * BM);
+                    const uint32_t dcol = tmem_base + (uint32_t)((grp_i & 1) * BM);
                     if (leader) {
 #pragma unroll
                         for (int j = 0; j < 2; ++j)
-#pragma unroll
-                            for (int h = 0; h < 2; ++h)
-                                tc_mma(dcol + h * BM, ad + h * (kAHalf >> 4) + 4 * hk + 2 * j, bd + 4 * hk + 2 * j,
-                                       idesc, (starts && j == 0) ? 0u : 1u);
+                            tc_mma(dcol, ad + 4 * hk + 2 * j, bd + 4 * hk + 2 * j, idesc,
+                                   (starts && j == 0) ? 0u : 1u);
                     }
                     const bool ends = two_per_stage ? true : (hk == 1 && sig == spg - 1);
                     if (ends && leader) tc_commit(&pfull[grp_i & 1]);
@@ -365,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------------------ dequant warps
-        const int dq = warp - 2;                 // row tiles dq, dq + 6, dq + 12 of the 16
+        const int dq = warp - 2;                 // row tiles dq and dq + 6 of the 8
         const int gq = lane >> 2, c = 2 * (lane & 3);
         // stmatrix.x4 row addresses: lane l gives row (l & 7) of 8x8 matrix l >> 3, the
         // matrices being (rows 0-7 | 8-15) x (channels 0-7 | 8-15) of a 16x16 step, i.e.
@@ -388,14 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int ti = dq; ti < BN / 16; ti += kDequantWarps) {
                     if (ti >= tt_end) break;
-                    const int hh = ti >> 3, tt = ti & 7;          // half, tile within the half
-                    const uint32_t a_u32 = smem_u32(smem + L::a + ds * kABytes + hh * kAHalf);
-                    const unsigned char* pk = smem + L::pk + s * kPBytes + hh * (kPBytes / 2);
-                    const unsigned char* zs = smem + L::zr + s * kZBytes + hh * BH * 2;
+                    const int tt = ti;
+                    const uint32_t a_u32 = smem_u32(smem + L::a + ds * kABytes);
+                    const unsigned char* pk = smem + L::pk + s * kPBytes;
+                    const unsigned char* zs = smem + L::zr + s * kZBytes;
                     const uint4 wq = *reinterpret_cast<const uint4*>(pk + tt * 512 + lane * 16);
                     const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-                    const int r0 = 16 * tt + gq, r1 = r0 + 8;      // rows within the half
-                    const int nr0 = n0 + hh * BH + r0, nr1 = nr0 + 8;  // output rows
+                    const int r0 = 16 * tt + gq, r1 = r0 + 8;      // rows within the tile
+                    const int nr0 = n0 + r0, nr1 = nr0 + 8;            // output rows
                     const uint32_t row_addr = a_u32 + (uint32_t)((16 * tt + rr + 8 * (mi & 1)) * 128);
                     // zero-point constants of this stage's group(s) (two groups when g = 32)
                     ZeroConsts zc[2];
@@ -456,8 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         pdl_wait();   // before any store to Y
         const int e = warp - 8;
         const int quad = warp & 3;                 // tensor-memory lanes 32*quad..
-        const int h = e >> 2;                      // half
-        const int row = h * BH + 32 * quad + lane; // output row within the tile
+        const int h = e >> 2;                      // token half: columns 128 h ..
+        const int row = 32 * quad + lane;          // output row within the tile
         const int esz = p.out_dtype == 2 ? 4 : 2;
         unsigned char* yt = smem + L::y;
         int ge = 0;   // group counter across this CTA's tiles (partial buffer, phase)
@@ -466,9 +458,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n0 = (t % nbands) * BN, m0 = (t / nbands) * BM;
             const int n = n0 + row;
             const bool row_ok = n < p.N;
-            float acc[BM];
+            float acc[BM / 2];
 #pragma unroll
-            for (int i = 0; i < BM; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < BM / 2; ++i) acc[i] = 0.0f;
             for (int grp = 0; grp < ngroups && ok; ++grp, ++ge) {
                 const int pb = ge & 1;
                 float sc = 1.0f;
@@ -476,9 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = wait_or_abort(&pfull[pb], (ge >> 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(pb * 2 * BM + h * BM);
+                const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(pb * BM + h * (BM / 2));
 #pragma unroll
-                for (int ch = 0; ch < BM / 32; ++ch) {
+                for (int ch = 0; ch < BM / 64; ++ch) {
                     float v[32];
                     tmem_ld32(taddr + 32 * ch, v);
 #pragma unroll
@@ -487,17 +479,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&pempty[pb]);
             }
-            // Y tile through a staging buffer of kYChunk tokens: thread `row` writes column
-            // `row` of a [kYChunk tokens][BN rows] block, then the eight warps copy it out in
-            // 16-byte pieces along N.  The next tile's MMAs proceed meanwhile.
+            // Y tile through a staging buffer of kYChunk tokens of each token half: thread
+            // `row` of half h writes column `row` of rows h kYChunk .. of a [2 kYChunk
+            // tokens][BN rows] block, then the eight warps copy it out in 16-byte pieces
+            // along N.  The next tile's MMAs proceed meanwhile.
             const int cpr = BN * esz / 16;               // 16-byte pieces per token row
             const int ncols = min(BN, p.N - n0);         // a multiple of 16 (N % 16 == 0)
 #pragma unroll
-            for (int ck = 0; ck < BM / kYChunk; ++ck) {
+            for (int ck = 0; ck < BM / 2 / kYChunk; ++ck) {
                 if (ok) {
 #pragma unroll
                     for (int i = 0; i < kYChunk; ++i) {
-                        unsigned char* ep = yt + (i * BN + row) * esz;
+                        unsigned char* ep = yt + ((h * kYChunk + i) * BN + row) * esz;
                         const float v = acc[ck * kYChunk + i];
                         if (p.out_dtype == 2) *reinterpret_cast<float*>(ep) = v;
                         else if (p.out_dtype == 1) *reinterpret_cast<__nv_bfloat16*>(ep) = __float2bfloat16_rn(v);
@@ -506,9 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 named_bar_sync(1, 256);
                 if (ok) {
-                    for (int cc = 32 * e + lane; cc < kYChunk * cpr; cc += 256) {
+                    for (int cc = 32 * e + lane; cc < 2 * kYChunk * cpr; cc += 256) {
                         const int m = cc / cpr, pc = cc - m * cpr;
-                        const int mm = m0 + ck * kYChunk + m;
+                        const int mm = m0 + (m / kYChunk) * (BM / 2) + ck * kYChunk + m % kYChunk;
                         if (mm >= p.M || pc * 16 >= ncols * esz) continue;
                         const uint4 v = *reinterpret_cast<const uint4*>(yt + m * BN * esz + pc * 16);
                         *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(p.Y) +

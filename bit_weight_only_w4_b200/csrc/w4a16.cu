@@ -141,15 +141,17 @@ bool make_act_blocks_map(CUtensorMap* map, const void* X, bool bf16, int64_t M, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D map over fp16 group metadata [G,N] (N innermost): boxes of 128 columns x rows groups.
-bool make_meta_map(CUtensorMap* map, const void* base, int64_t G, int64_t N, int rows) {
+// 2-D map over group metadata [G,N] (N innermost), fp16 or (bytes) uint8: boxes of 128
+// columns x rows groups.
+bool make_meta_map(CUtensorMap* map, const void* base, int64_t G, int64_t N, int rows, bool bytes = false) {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)G};
-    const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * (bytes ? 1 : 2)};
     const cuuint32_t box[2] = {128u, (cuuint32_t)rows};
     const cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+    return enc(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+               const_cast<void*>(base), dims, strides,
                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -193,14 +195,17 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     const int span = 64 * C::aps;   // input channels per stage
     const int xrows = NT == 1 ? p.M : C::mpad;
     const bool staged_x = !p.xres;
-    p.ngs = GIDX ? 0 : (g == 32 ? span / 32 : std::min(p.G, (span + 2 * g - 65) / g));
+    // FP4: group_size is the scale block (16 or 32), the staged rows are bytes
+    constexpr bool FP4 = MODE == w4d::kModeNvfp4 || MODE == w4d::kModeMxfp4;
+    p.srow_bytes = FP4 ? 128 : 256;
+    p.ngs = GIDX ? 0 : FP4 ? span / g : (g == 32 ? span / 32 : std::min(p.G, (span + 2 * g - 65) / g));
     p.off_x = C::aps * w4d::kTilesPerBand * 512;
     p.off_xs = p.off_x + (staged_x ? up(C::aps * p.M * 128, 1024) : 0);
     p.off_sx = p.off_xs + (staged_x ? up(C::aps * xrows * 128, 128) : 0);
     p.off_si = p.off_sx + (staged_x && !GIDX ? C::sx_floats * 4 : 0);
     p.off_sc = p.off_si + (staged_x && p.s_inv ? C::aps * 256 : 0);
-    p.off_zr = p.off_sc + p.ngs * 256;
-    p.off_gi = p.off_zr + (p.zeros ? p.ngs * 256 : 0);
+    p.off_zr = p.off_sc + p.ngs * p.srow_bytes;
+    p.off_gi = p.off_zr + (p.zeros ? p.ngs * p.srow_bytes : 0);
     p.off_desc = p.off_gi + (GIDX ? C::aps * 256 : 0);
     p.stage_bytes = (p.off_desc + 48 + 1023) / 1024 * 1024;
     // as many stages as fit: the CTA fills the SM's shared memory, one CTA per SM
@@ -227,8 +232,8 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     map_sc = map_x;
     map_zr = map_x;
     if (!GIDX) {
-        if (!make_meta_map(&map_sc, p.scales, p.G, p.N, p.ngs)) return W4_ERR_CUDA;
-        if (p.zeros && !make_meta_map(&map_zr, p.zeros, p.G, p.N, p.ngs)) return W4_ERR_CUDA;
+        if (!make_meta_map(&map_sc, p.scales, p.G, p.N, p.ngs, FP4)) return W4_ERR_CUDA;
+        if (p.zeros && !make_meta_map(&map_zr, p.zeros, p.G, p.N, p.ngs, FP4)) return W4_ERR_CUDA;
     }
     // programmatic dependent launch: this kernel's prologue and weight loads may overlap
     // the tail of the preceding kernel on the stream
@@ -261,8 +266,10 @@ w4_status dispatch_mode(int mode, w4d::DecodeParams p, const void* X, unsigned c
                         cudaStream_t s) {
     if constexpr (!BF16 && !PERM) {
         if (mode == w4d::kModeGidx) return launch_decode<NT, false, w4d::kModeGidx, false>(p, X, ws, dev, s);
+        if (mode == w4d::kModeNvfp4) return launch_decode<NT, false, w4d::kModeNvfp4, false>(p, X, ws, dev, s);
+        if (mode == w4d::kModeMxfp4) return launch_decode<NT, false, w4d::kModeMxfp4, false>(p, X, ws, dev, s);
     } else {
-        if (mode == w4d::kModeGidx) return W4_ERR_UNSUPPORTED;
+        if (mode == w4d::kModeGidx || mode == w4d::kModeNvfp4 || mode == w4d::kModeMxfp4) return W4_ERR_UNSUPPORTED;
     }
     if (mode == w4d::kModeHalf) return launch_decode<NT, BF16, w4d::kModeHalf, PERM>(p, X, ws, dev, s);
     if (mode == w4d::kModeG32) return launch_decode<NT, BF16, w4d::kModeG32, PERM>(p, X, ws, dev, s);
@@ -933,6 +940,7 @@ w4_status chain_launch(const w4_chain_layer* layers, int l0, int n, int M, bool 
         p.rem = p.units % sms;
         const int g = p.group_size;
         p.ngs = g == 32 ? span / 32 : std::min(p.G, (span + 2 * g - 65) / g);
+        p.srow_bytes = 256;
         p.stages = stages;
         p.xres = 1;
         p.sstride = sstride;
@@ -1006,4 +1014,123 @@ extern "C" w4_status w4a16_gemm_chain(const w4_chain_layer* layers, int32_t n_la
         if (st != W4_OK) return st;
     }
     return W4_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Block-scaled FP4 weights (NVFP4, MXFP4): quantise/pack, and the GEMM with 16-bit
+// activations (the decode kernel's FP4 modes for M <= 64, the prefill kernel above).
+// ---------------------------------------------------------------------------------------
+namespace {
+
+int fp4_block(w4_fp4_format f) { return f == W4_FP4_NVFP4 ? 16 : 32; }
+
+w4_status check_fp4_shape(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0) return W4_ERR_INVALID_ARG;
+    if (N > INT_MAX / 2 || K > INT_MAX / 2) return W4_ERR_UNSUPPORTED;
+    if (N % 16 != 0 || K % 64 != 0 || N > kMaxBands * 128) return W4_ERR_UNSUPPORTED;
+    return W4_OK;
+}
+
+template <int FMT, bool BF16W>
+w4_status launch_fp4_pack(const w4f::Fp4Params& p, int dev, cudaStream_t s) {
+    static std::once_flag flags[kMaxDevices];
+    const int smem = (p.K / w4f::Fmt<FMT>::block) * w4f::kRows;
+    if (!ensure_smem(w4f::fp4_pack_kernel<FMT, BF16W>, 227 * 1024, flags, dev)) return W4_ERR_CUDA;
+    w4f::fp4_pack_kernel<FMT, BF16W><<<(unsigned)(p.N / 16), w4f::kThreads, smem, s>>>(p);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" w4_status w4_fp4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K,
+                                          w4_fp4_format format, uint32_t* qweight, uint8_t* block_scales,
+                                          float* tensor_scale, w4_stream_t stream) {
+    if (!W || !qweight || !block_scales) return W4_ERR_INVALID_ARG;
+    if (w_dtype != W4_F16 && w_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
+    if (format != W4_FP4_NVFP4 && format != W4_FP4_MXFP4) return W4_ERR_INVALID_ARG;
+    if ((format == W4_FP4_NVFP4) != (tensor_scale != nullptr)) return W4_ERR_INVALID_ARG;
+    if (!aligned(W, 2) || !aligned(qweight, 4) || !aligned(tensor_scale, 4)) return W4_ERR_INVALID_ARG;
+    w4_status st = check_fp4_shape(N, K);
+    if (st != W4_OK) return st;
+    if ((K / fp4_block(format)) * w4f::kRows > 227 * 1024) return W4_ERR_UNSUPPORTED;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    cudaStream_t strm = as_stream(stream);
+    w4f::Fp4Params p;
+    p.W = W;
+    p.qweight = qweight;
+    p.bscale = block_scales;
+    p.tscale = tensor_scale;
+    p.N = (int)N;
+    p.K = (int)K;
+    const bool bf16 = w_dtype == W4_BF16;
+    if (format == W4_FP4_NVFP4) {
+        // the tensor's amax (into *tensor_scale), the packing, then gs in its place
+        if (cudaMemsetAsync(tensor_scale, 0, sizeof(float), strm) != cudaSuccess) return W4_ERR_CUDA;
+        const size_t n = (size_t)N * (size_t)K;
+        const unsigned blocks = (unsigned)std::min<size_t>((n + 255) / 256, (size_t)sm_count(dev) * 8);
+        if (bf16) w4f::amax_kernel<true><<<blocks, 256, 0, strm>>>(W, n, tensor_scale);
+        else w4f::amax_kernel<false><<<blocks, 256, 0, strm>>>(W, n, tensor_scale);
+        if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+        st = bf16 ? launch_fp4_pack<w4f::kNvfp4, true>(p, dev, strm) : launch_fp4_pack<w4f::kNvfp4, false>(p, dev, strm);
+        if (st != W4_OK) return st;
+        w4f::finish_tscale_kernel<<<1, 1, 0, strm>>>(tensor_scale);
+        return launch_status();
+    }
+    return bf16 ? launch_fp4_pack<w4f::kMxfp4, true>(p, dev, strm) : launch_fp4_pack<w4f::kMxfp4, false>(p, dev, strm);
+}
+
+extern "C" size_t w4a16_fp4_workspace_bytes(int64_t M, int64_t N, int64_t K, w4_fp4_format format) {
+    if (format != W4_FP4_NVFP4 && format != W4_FP4_MXFP4) return 0;
+    if (M <= 0 || check_fp4_shape(N, K) != W4_OK) return 0;
+    const int dev = current_device();
+    const int sms = dev >= 0 ? sm_count(dev) : 0;
+    if (sms <= 0) return 0;
+    if (M <= kDecodeMaxM) return decode_workspace_bytes(M, sms);
+    return 0;   // the prefill kernel needs no workspace
+}
+
+extern "C" w4_status w4a16_fp4_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                                    const uint32_t* qweight, const uint8_t* block_scales,
+                                    const float* tensor_scale, w4_fp4_format format, void* Y,
+                                    w4_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                    w4_stream_t stream) {
+    if (M < 0) return W4_ERR_INVALID_ARG;
+    if (format != W4_FP4_NVFP4 && format != W4_FP4_MXFP4) return W4_ERR_INVALID_ARG;
+    if (act_dtype != W4_F16 && act_dtype != W4_BF16) return W4_ERR_INVALID_ARG;
+    if (out_dtype != W4_F16 && out_dtype != W4_BF16 && out_dtype != W4_F32) return W4_ERR_INVALID_ARG;
+    w4_status st = check_fp4_shape(N, K);
+    if (st != W4_OK) return st;
+    if (M == 0) return W4_OK;
+    if (act_dtype != W4_F16) return W4_ERR_UNSUPPORTED;   // E2M1 decodes exactly to fp16
+    if (!X || !qweight || !block_scales || !Y) return W4_ERR_INVALID_ARG;
+    if ((format == W4_FP4_NVFP4) != (tensor_scale != nullptr)) return W4_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(block_scales, 16) || !aligned(Y, 16) ||
+        !aligned(tensor_scale, 4) || !aligned(workspace, 256))
+        return W4_ERR_INVALID_ARG;
+    if (M > INT_MAX / 2 || (size_t)M * (size_t)K > (size_t)INT_MAX * 8) return W4_ERR_UNSUPPORTED;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    const int B = fp4_block(format);
+    cudaStream_t strm = as_stream(stream);
+    if (M > kDecodeMaxM) return W4_ERR_UNSUPPORTED;
+    const size_t need = w4a16_fp4_workspace_bytes(M, N, K, format);
+    if (need == 0) return W4_ERR_CUDA;
+    if (!workspace || workspace_bytes < need) return W4_ERR_INVALID_ARG;
+    w4d::DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.qw = qweight;
+    p.scales = reinterpret_cast<const __half*>(block_scales);
+    p.tscale = tensor_scale;
+    p.Y = Y;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.group_size = B;
+    p.G = (int)(K / B);
+    p.out_dtype = (int)out_dtype;
+    p.KA = (int)(K / 64);
+    p.tiles = (int)(N / 16);
+    const int mode = format == W4_FP4_NVFP4 ? w4d::kModeNvfp4 : w4d::kModeMxfp4;
+    return dispatch_decode<false>(mode, p, X, reinterpret_cast<unsigned char*>(workspace), dev, strm);
 }

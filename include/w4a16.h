@@ -292,6 +292,56 @@ w4_status w4a16_gemm_chain(const w4_chain_layer* layers, int32_t n_layers, int64
 size_t w4a16_chain_workspace_bytes(int64_t M);
 
 /*
+ * Block-scaled 4-bit floating-point weights (NVFP4, MXFP4), the Blackwell 4-bit format
+ * of "Production Quantization: AWQ, GPTQ, GGUF K-quants, FP8, MXFP4/NVFP4", section
+ * "MXFP4 / NVFP4" (4-bit floating-point values with a scale per block of weights): a
+ * comparator for the INT4 path on the same layer shapes, with 16-bit activations.
+ *   element  E2M1: sign, 2 exponent bits, 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5,
+ *            2, 3, 4, 6
+ *   NVFP4    blocks of 16 consecutive input channels, an E4M3 block scale sb, one fp32
+ *            tensor scale gs = amax|W| / (6 * 448) (1 for an all-zero W):
+ *            sb = E4M3(blockmax / 6 / gs), q = E2M1(w / (E4M3(sb) * gs))
+ *   MXFP4    blocks of 32, a power-of-two scale 2^e stored as the byte e + 127,
+ *            e = max(floor(log2 blockmax) - 2, -127), q = E2M1(w / 2^e)
+ * All in fp32; every conversion rounds to nearest, ties to even, and saturates finite
+ * values at the largest magnitude; an element's sign is its input's, also at zero.
+ */
+typedef enum { W4_FP4_NVFP4 = 0, W4_FP4_MXFP4 = 1 } w4_fp4_format;
+
+/*
+ * w4_fp4_quantize_pack -- quantise W to NVFP4 or MXFP4 and pack the codes.
+ *   W             device [N,K] row-major, fp16 (W4_F16) or bf16 (W4_BF16)
+ *   N, K          N % 16 == 0, K % 64 == 0
+ *   qweight       device uint32 [N*K/8] output: the E2M1 codes in the device layout of
+ *                 the INT4 codes above (code (n,k) where q[n][k] would be)
+ *   block_scales  device uint8 [K/B, N] output (B = 16 NVFP4, 32 MXFP4), block-row-major
+ *   tensor_scale  device fp32 [1] output for NVFP4 (gs); must be NULL for MXFP4
+ * Bit-exact (no fast-math).  Asynchronous on `stream`.
+ */
+w4_status w4_fp4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64_t K,
+                               w4_fp4_format format, uint32_t* qweight, uint8_t* block_scales,
+                               float* tensor_scale, w4_stream_t stream);
+
+/*
+ * w4a16_fp4_gemm -- Y[M,N] = X[M,K] @ What^T, What[n,k] = E2M1(q[n,k]) * scale(block of
+ * k, n) (* gs for NVFP4), fp32 accumulation.  fp16 activations only (every E2M1 value is
+ * exact in fp16; bf16 returns W4_ERR_UNSUPPORTED).  M <= 64 runs the bandwidth-bound
+ * decode kernel: each block's products are summed by the tensor cores and multiplied by
+ * the block's scale in fp32.
+ *   workspace  >= w4a16_fp4_workspace_bytes(M,N,K,format) bytes, 256-byte aligned,
+ *              zero-filled before its first use (as for w4a16_gemm)
+ */
+w4_status w4a16_fp4_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
+                         const uint32_t* qweight, const uint8_t* block_scales,
+                         const float* tensor_scale, w4_fp4_format format, void* Y,
+                         w4_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                         w4_stream_t stream);
+
+/* Bytes of workspace w4a16_fp4_gemm needs (0 on invalid sizes, and for M > 64, which
+ * needs none). */
+size_t w4a16_fp4_workspace_bytes(int64_t M, int64_t N, int64_t K, w4_fp4_format format);
+
+/*
  * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 32 (M <= 64 where the scratch fits)
  * without a caller-supplied workspace.  The pages have no counterpart to this call; it
  * exists for callers that cannot allocate device memory where they run the GEMM, such as

@@ -2,12 +2,15 @@
 against the CPU oracle run layer by layer.
 
 The oracle chain rounds every layer's output to the output type, as the GPU stores it,
-and feeds the next layer the same slice the GPU layer reads.  fp16 chains are held to the
-stated bound (relative L2 1e-3, max-abs 2e-2): the chains differ only where the GPU's fp32
-summation order moves a value across an fp16 rounding boundary (a 1-ulp difference on a
-small fraction of elements), and such differences pass through later layers at about
-their own relative size.  bf16 outputs are held to one bf16 ulp of the oracle plus the
-fp32 path's error bound.
+and feeds the next layer the same slice the GPU layer reads.  It also rounds each layer's
+X' = X s^-1 to the activation type before the product, as the kernels do: through a deep
+chain the per-layer X' rounding (about 1.4e-4 relative L2 a layer) otherwise accumulates
+like a random walk (about 1e-3 after 40 layers) and would hide what the chain test is
+for.  fp16 chains are then held to the stated bound (relative L2 1e-3, max-abs 2e-2): the
+chains differ only where the GPU's fp32 summation order moves a value across an fp16
+rounding boundary (a 1-ulp difference on a small fraction of elements), and such
+differences pass through later layers at about their own relative size.  bf16 outputs are
+held to one bf16 ulp of the oracle plus the fp32 path's error bound.
 """
 import numpy as np
 import pytest
@@ -22,6 +25,14 @@ pytestmark = pytest.mark.gpu
 
 def _round(y32, bf16):
     return oracle.f32_to_bf16(y32) if bf16 else oracle.f32_to_f16(y32)
+
+
+def _oracle_layer(Xb, s_inv, q, sc, zr, g, bf16):
+    """One layer of the oracle chain: X' = X s^-1 in fp32, rounded to the activation type
+    (as the kernels round it), then the dequantised weights and the fp32 product."""
+    Xp = oracle.awq_scale_acts(Xb, s_inv, bf16)
+    Xp = oracle.bf16_to_f32(oracle.f32_to_bf16(Xp)) if bf16 else oracle.f16_to_f32(oracle.f32_to_f16(Xp))
+    return oracle.gemm_f32(Xp, oracle.dequant(q, sc, zr, g))
 
 
 def _build(M, specs, seed, act="fp16", g=128):
@@ -42,9 +53,9 @@ def _build(M, specs, seed, act="fp16", g=128):
         q, sc, zr = oracle.quantize_weights(W, s, g)
         Y = torch.full((M, N), float("nan"), dtype=tdt, device="cuda")
         ys.append(Y)
-        Xd = X0d if src < 0 else ys[src][:, c0:c0 + K]
-        Xb = X0 if src < 0 else refbits[src][:, c0:c0 + K]
-        y = oracle.reference_y(np.ascontiguousarray(Xb), s_inv, q, sc, zr, g, x_is_bf16=bf16)
+        Xd = (X0d if src < 0 else ys[src])[:, c0:c0 + K]
+        Xb = (X0 if src < 0 else refbits[src])[:, c0:c0 + K]
+        y = _oracle_layer(np.ascontiguousarray(Xb), s_inv, q, sc, zr, g, bf16)
         ref32.append(y)
         refbits.append(_round(y, bf16))
         host.append({"Xbits": np.ascontiguousarray(Xb), "q": q, "sc": sc, "zr": zr, "s_inv": s_inv})
@@ -135,7 +146,7 @@ def test_chain_llama7b_block():
         q, sc, zr = oracle.quantize_weights(W_bits, li.s, li.group_size)
         src, c0 = workloads.CHAIN_SOURCE[j]
         Xb = X0 if src < 0 else refbits[src][:, c0:c0 + L.K]
-        y = oracle.reference_y(np.ascontiguousarray(Xb), s_inv, q, sc, zr, li.group_size)
+        y = _oracle_layer(np.ascontiguousarray(Xb), s_inv, q, sc, zr, li.group_size, False)
         refbits.append(oracle.f32_to_f16(y))
         Y = torch.full((M, L.N), float("nan"), dtype=torch.float16, device="cuda")
         Xd = dev_bits(X0, torch.float16) if src < 0 else ys[src][:, c0:c0 + L.K]
