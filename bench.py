@@ -747,6 +747,75 @@ def time_gptq_sweep(w4, torch, Ms=(1, 16, 1024), gs=(32, 64, 128, 4096)):
     return out
 
 
+def fp4_weight_bytes(N, K, fmt):
+    """Algorithmic bytes of FP4 weights: the codes (0.5 B/weight), one scale byte per block
+    (16 weights NVFP4, 32 MXFP4) and the NVFP4 fp32 tensor scale."""
+    B = 16 if fmt == "nvfp4" else 32
+    return N * K // 2 + N * K // B + (4 if fmt == "nvfp4" else 0)
+
+
+def time_fp4(w4, torch, fmts=("nvfp4", "mxfp4")):
+    """The block-scaled FP4 comparator: every 7B decode projection at M = 1 (GB/s of FP4
+    weight bytes, per launch over rotated copies larger than L2) and the two 8B prefill
+    projections at M = 4096 with fp16 activations (TFLOPS)."""
+    out = {}
+    wl = workloads.workload(DECODE_CFG)
+    for fmt in fmts:
+        rows = {}
+        for i, L in enumerate(wl.layers):
+            li = workloads.make_layer(wl, i, M=1)
+            W = dev_bits(li.W.view(np.uint16), torch.float16)
+            qw, bs, ts = w4.w4_fp4_quantize_pack(W, fmt)
+            by = fp4_weight_bytes(L.N, L.K, fmt)
+            n = max(2, math.ceil(4 * L2_BYTES / by))
+            copies = [(qw, bs)] + [(qw.clone(), bs.clone()) for _ in range(n - 1)]
+            X = dev_bits(li.X, torch.float16)
+            Y = torch.empty(1, L.N, dtype=torch.float16, device="cuda")
+            launches = max(n, 32)
+
+            def run(j, copies=copies, X=X, Y=Y, ts=ts):
+                q, b = copies[j % len(copies)]
+                w4.w4a16_fp4_gemm(X, q, b, ts, fmt, Y=Y)
+            for j in range(n):
+                run(j)
+            torch.cuda.synchronize()
+            g = capture(torch, lambda: [run(j) for j in range(launches)])
+            g.replay()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            us = a.elapsed_time(b) * 1e3 / launches
+            rows[f"{L.name} {L.K}x{L.N}"] = {"us": round(us, 3), "gbs": round(by / us / 1e3, 1)}
+            del g, copies
+        pw = workloads.workload(PREFILL_CFG)
+        pf = []
+        for i, L in enumerate(pw.layers):
+            M = 4096
+            W = (torch.randn(L.N, L.K, device="cuda", generator=torch.Generator(device="cuda").manual_seed(i))
+                 * workloads.W_STD).half()
+            qw, bs, ts = w4.w4_fp4_quantize_pack(W, fmt)
+            X = dev_bits(workloads.gen_acts(M, L.K, 0, PREFILL_CFG, i, "fp16"), torch.float16)
+            Y = torch.empty(M, L.N, dtype=torch.float16, device="cuda")
+            for _ in range(3):
+                w4.w4a16_fp4_gemm(X, qw, bs, ts, fmt, Y=Y)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(5):
+                w4.w4a16_fp4_gemm(X, qw, bs, ts, fmt, Y=Y)
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / 5
+            pf.append({"layer": f"{L.name} {L.K}x{L.N}", "ms": round(ms, 4),
+                       "tflops": round(workloads.gemm_flops(M, L.N, L.K) / ms / 1e9, 1)})
+        w4.w4_check_device_error()
+        out[fmt] = {"decode_m1": rows, "prefill_m4096_fp16": pf}
+    return out
+
+
 def our_arm(args, world, rank, local):
     import torch
     import bit_weight_only_w4_b200 as w4
@@ -803,6 +872,7 @@ def our_arm(args, world, rank, local):
         extras["prefill"] = time_prefill_sweep(w4, torch, peaks)
         extras["prefill_m4096"] = extras["prefill"]["4096"]
         extras["gptq_actorder_perm"] = time_gptq_sweep(w4, torch)
+        extras["fp4"] = time_fp4(w4, torch)
         extras["quantize_pack"] = time_quantize(w4, torch, projs)
         extras["awq_search"] = time_awq_search(w4, torch)
         # last: its larger workspace may replace the cached one the graphs above captured

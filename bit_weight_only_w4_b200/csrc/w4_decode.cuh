@@ -522,21 +522,8 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
     }
 }
 
-// FP4 weights: two E2M1 codes of one A-operand register become two exact fp16 values in
-// one hardware conversion (the byte holds the register's first column in its low
-// nibble); the MMA sums each scale block's products and the block's scale multiplies
-// that partial in fp32.  Nibbles i and i+4 of a device-layout word are the register's
-// two columns, so the bytes are (n0|n4), (n2|n6) from the word and (n1|n5), (n3|n7)
-// from the word shifted by 4.
-W4_DEV void unpack_fp4(uint32_t w, uint32_t (&a)[4]) {
-    const uint32_t zx = (w & 0x0F0Fu) | ((w >> 12) & 0xF0F0u);
-    const uint32_t zy = ((w >> 4) & 0x0F0Fu) | ((w >> 16) & 0xF0F0u);
-    a[0] = w4f::e2m1x2_to_h2(zx & 0xFFu);
-    a[1] = w4f::e2m1x2_to_h2(zy & 0xFFu);
-    a[2] = w4f::e2m1x2_to_h2((zx >> 8) & 0xFFu);
-    a[3] = w4f::e2m1x2_to_h2((zy >> 8) & 0xFFu);
-}
-
+// FP4 weights: the E2M1 codes become exact fp16 values (w4f::unpack_fp4); the MMA sums
+// each scale block's products and the block's scale multiplies that partial in fp32.
 // Scale of one staged block-scale byte: E4M3 (NVFP4) or 2^(byte - 127) (MXFP4; the
 // byte 0, 2^-127, reads as 0: such a block's weights are below 2^-124).
 template <int MODE>
@@ -570,7 +557,7 @@ W4_DEV void consume_fp4(const StageView& v, const Lane& L, int t0, int ab, int a
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt) {
                 uint32_t af[4];
-                unpack_fp4(word_j<TPW>(w[tt], j), af);
+                w4f::unpack_fp4(word_j<TPW>(w[tt], j), af);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if (first) mma_16816_z<false>(c[tt][nt], af, b0[nt], b1[nt]);

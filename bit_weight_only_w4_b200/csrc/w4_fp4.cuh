@@ -73,6 +73,21 @@ W4_DEV float e4m3_to_f32(uint32_t b) {
     return __low2float(u32_as_h2(e4m3x2_to_h2(b | (b << 8))));
 }
 
+// One device-layout word -> the four A-operand registers of a 16x16 MMA slice (a[0] =
+// row r0 cols c,c+1; a[1] = row r1 cols c,c+1; a[2] = row r0 cols c+8,c+9; a[3] = row r1
+// cols c+8,c+9), every element the exact fp16 value of its E2M1 code.  Nibbles i and
+// i+4 of the word are a register's two columns, so one conversion each takes the bytes
+// (n0|n4), (n2|n6) of the word and (n1|n5), (n3|n7) of the word shifted by 4 (the byte's
+// low nibble is the register's first column).
+W4_DEV void unpack_fp4(uint32_t w, uint32_t (&a)[4]) {
+    const uint32_t zx = (w & 0x0F0Fu) | ((w >> 12) & 0xF0F0u);
+    const uint32_t zy = ((w >> 4) & 0x0F0Fu) | ((w >> 16) & 0xF0F0u);
+    a[0] = e2m1x2_to_h2(zx & 0xFFu);
+    a[1] = e2m1x2_to_h2(zy & 0xFFu);
+    a[2] = e2m1x2_to_h2((zx >> 8) & 0xFFu);
+    a[3] = e2m1x2_to_h2((zy >> 8) & 0xFFu);
+}
+
 // 2^e for e in [-126, 127] (exact; fp32 bit pattern).
 W4_DEV float exp2i(int e) { return __int_as_float((e + 127) << 23); }
 

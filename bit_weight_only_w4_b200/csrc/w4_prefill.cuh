@@ -31,8 +31,17 @@
 // accumulates in one tensor-memory buffer.
 #pragma once
 #include "w4_common.cuh"
+#include "w4_fp4.cuh"
 
 namespace w4p {
+
+// Weight formats of the prefill kernel.
+enum : int {
+    kWInt4 = 0,    // INT4 codes, contiguous groups: per-group fp32 rescale of TMEM partials
+    kWGidx = 1,    // INT4 codes, act-order g_idx: the scale folded into each fp16 weight
+    kWNvfp4 = 2,   // NVFP4: E2M1 x E4M3 block scale, exact in fp16; tensor scale at the end
+    kWMxfp4 = 3,   // MXFP4: E2M1 x 2^e, exact in fp16 for e in [-13, 13]
+};
 
 constexpr int BN = 128;        // output rows per tile (MMA M)
 constexpr int BM = 256;        // tokens per tile (MMA N)
@@ -77,6 +86,8 @@ struct PrefillParams {
     const __half* scales;
     const __half* zeros;
     const int32_t* g_idx;
+    const uint8_t* bscale;   // FP4 block scales [K/B, N]
+    const float* tscale;     // NVFP4 tensor scale (device fp32) or null
     void* Y;
     int M, N, K, group_size, G, out_dtype;
     int KA;       // K / 64
@@ -195,9 +206,12 @@ W4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_fl
     return false;
 }
 
-template <bool BF16, bool GIDX>
+template <bool BF16, int WM>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const PrefillParams p) {
+    constexpr bool GIDX = WM == kWGidx;
+    constexpr bool FP4 = WM == kWNvfp4 || WM == kWMxfp4;
+    constexpr bool ONEBUF = GIDX || FP4;   // scale in the weights: one partial over the whole K
     extern __shared__ unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled operand tiles
     unsigned char* smem = align_smem_1024(smem_raw);
@@ -215,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = p.K / BK;              // stages along K per tile
     const int g = p.group_size;
-    const int ngroups = GIDX ? 1 : p.K / g;
+    const int ngroups = ONEBUF ? 1 : p.K / g;
     // persistent tiles: tile t covers tokens [m0, m0+BM) of m-block t / nbands and output
     // rows [n0, n0+BN) of row block t % nbands, so the CTAs running at one time share
     // their activation tiles (L2 reuse); a CTA takes tiles blockIdx.x, + gridDim.x, ...
@@ -265,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int rb = t % nbands;
                 const int n0 = rb * BN, m0 = (t / nbands) * BM;
                 const int th = max(0, min(BN / 16, p.tiles - n0 / 16));   // 16-row tiles
-                const int zgroups = (!GIDX && p.zeros) ? (g == 32 ? 2 : 1) : 0;
+                const int zgroups = (!ONEBUF && p.zeros) ? (g == 32 ? 2 : 1) : 0;
                 const uint32_t bytes = kBBytes + th * (512 + zgroups * 32);
                 for (int kt = 0; kt < KT; ++kt, ++gst) {
                     const int s = gst % kLoadStages, ph = (gst / kLoadStages) & 1;
@@ -300,8 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t b_desc0 = sw128_desc(smem_u32(smem + L::b));
         // group boundaries: every spg stages (g a multiple of 64), twice per stage
         // (g = 32) or once per tile (act-order: one partial sum over the whole K)
-        const int spg = GIDX ? KT : (g >= BK ? g / BK : 1);
-        const bool two_per_stage = !GIDX && g == 32;
+        const int spg = ONEBUF ? KT : (g >= BK ? g / BK : 1);
+        const bool two_per_stage = !ONEBUF && g == 32;
         int grp_i = -1;   // group counter across this CTA's tiles (partial buffer, phase)
         int gst = 0;
         bool ok = true;
@@ -391,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t row_addr = a_u32 + (uint32_t)((16 * tt + rr + 8 * (mi & 1)) * 128);
                     // zero-point constants of this stage's group(s) (two groups when g = 32)
                     ZeroConsts zc[2];
-                    if constexpr (!GIDX) {
+                    if constexpr (!ONEBUF) {
 #pragma unroll
                         for (int zg = 0; zg < 2; ++zg) {
                             const int zo = (g == 32 ? zg : 0) * BN * 2;
@@ -405,7 +419,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int kk = 16 * j + c;                 // column within the stage
                         const int kabs = kt * BK + kk;
                         uint32_t af[4];
-                        if constexpr (!GIDX) {
+                        if constexpr (FP4) {
+                            // E2M1 (exact fp16) times the block's scale (exact fp16 product)
+                            constexpr int B = WM == kWNvfp4 ? 16 : 32;
+                            const int blk = (kt * BK + 16 * j) / B;
+                            const uint32_t b0 = __ldg(p.bscale + (size_t)blk * p.N + nr0);
+                            const uint32_t b1 = __ldg(p.bscale + (size_t)blk * p.N + nr1);
+                            uint32_t s0, s1;
+                            if constexpr (WM == kWNvfp4) {
+                                s0 = w4f::e4m3x2_to_h2(b0 | (b0 << 8));
+                                s1 = w4f::e4m3x2_to_h2(b1 | (b1 << 8));
+                            } else {
+                                // 2^(b-127) as fp16; blocks outside [-13, 13] (other than the
+                                // all-but-zero byte 0) cannot be decoded exactly: reported
+                                const int e0 = (int)b0 - 127, e1 = (int)b1 - 127;
+                                if ((b0 != 0 && (e0 < -13 || e0 > 13)) || (b1 != 0 && (e1 < -13 || e1 > 13)))
+                                    atomicOr(&g_w4_error_word, W4_DEVERR_GIDX);
+                                const uint32_t h0 = (e0 < -14 || e0 > 15) ? 0u : (uint32_t)(e0 + 15) << 10;
+                                const uint32_t h1 = (e1 < -14 || e1 > 15) ? 0u : (uint32_t)(e1 + 15) << 10;
+                                s0 = h0 | (h0 << 16);
+                                s1 = h1 | (h1 << 16);
+                            }
+                            w4f::unpack_fp4(wv[j], af);
+                            af[0] = h2_as_u32(__hmul2(u32_as_h2(af[0]), u32_as_h2(s0)));
+                            af[1] = h2_as_u32(__hmul2(u32_as_h2(af[1]), u32_as_h2(s1)));
+                            af[2] = h2_as_u32(__hmul2(u32_as_h2(af[2]), u32_as_h2(s0)));
+                            af[3] = h2_as_u32(__hmul2(u32_as_h2(af[3]), u32_as_h2(s1)));
+                        } else if constexpr (!GIDX) {
                             unpack_word<BF16>(wv[j], zc[j >> 1], af);
                         } else {
                             int gk[4] = {__ldg(p.g_idx + kabs), __ldg(p.g_idx + kabs + 1),
@@ -464,7 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int grp = 0; grp < ngroups && ok; ++grp, ++ge) {
                 const int pb = ge & 1;
                 float sc = 1.0f;
-                if (!GIDX && row_ok) sc = __half2float(__ldg(p.scales + (size_t)grp * p.N + n));
+                if constexpr (FP4) sc = p.tscale ? __ldg(p.tscale) : 1.0f;
+                else if (!GIDX && row_ok) sc = __half2float(__ldg(p.scales + (size_t)grp * p.N + n));
                 ok = wait_or_abort(&pfull[pb], (ge >> 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();

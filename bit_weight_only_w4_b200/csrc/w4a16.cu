@@ -291,11 +291,11 @@ w4_status dispatch_decode(int mode, w4d::DecodeParams p, const void* X, unsigned
 }
 
 // ---------------------------------------------------------------- prefill launch plan
-template <bool BF16, bool GIDX>
+template <bool BF16, int WM>
 w4_status launch_prefill(const CUtensorMap& map, const w4p::PrefillParams& p, int dev,
                          cudaStream_t stream) {
     static std::once_flag flags[kMaxDevices];
-    auto k = w4p::prefill_kernel<BF16, GIDX>;
+    auto k = w4p::prefill_kernel<BF16, WM>;
     if (!ensure_smem(k, w4p::SmemLayout::bytes, flags, dev)) return W4_ERR_CUDA;
     // the kernel's per-warpgroup register split assumes this many registers a thread at
     // launch; any other build would make its register increase wait forever
@@ -556,9 +556,9 @@ static w4_status gemm_impl(const void* X, w4_dtype act_dtype, int64_t M, int64_t
     p.out_dtype = (int)out_dtype;
     p.KA = (int)(K / 64);
     p.tiles = (int)(N / 16);
-    if (bf16) return launch_prefill<true, false>(map, p, dev, strm);
-    return gidx ? launch_prefill<false, true>(map, p, dev, strm)
-                : launch_prefill<false, false>(map, p, dev, strm);
+    if (bf16) return launch_prefill<true, w4p::kWInt4>(map, p, dev, strm);
+    return gidx ? launch_prefill<false, w4p::kWGidx>(map, p, dev, strm)
+                : launch_prefill<false, w4p::kWInt4>(map, p, dev, strm);
 }
 
 size_t w4a16_workspace_bytes_perm(int64_t M, int64_t N, int64_t K, int32_t group_size) {
@@ -784,7 +784,25 @@ cudaError_t noalloc_rezero(int dev) {
     return e;
 }
 
+// Test aid: every split-K word of the scratch set to a flagged partial of 1.0.
+__global__ void plant_stale_kernel(unsigned long long* words, size_t n) {
+    const unsigned long long w = (1ull << 32) | (unsigned long long)__float_as_uint(1.0f);
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        words[i] = w;
+}
+
 }  // namespace
+
+extern "C" w4_status w4_selftest_noalloc_stale(w4_stream_t stream) {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    unsigned char* ws = reinterpret_cast<unsigned char*>(noalloc_scratch(dev));
+    if (!ws) return W4_ERR_CUDA;
+    const size_t n = (kNoAllocScratchBytes - kCounterBytes) / 8;
+    plant_stale_kernel<<<256, 256, 0, as_stream(stream)>>>(
+        reinterpret_cast<unsigned long long*>(ws + kCounterBytes), n);
+    return launch_status();
+}
 
 extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64_t M, int64_t N,
                                         int64_t K, const uint32_t* qweight, const void* scales,
@@ -1113,7 +1131,26 @@ extern "C" w4_status w4a16_fp4_gemm(const void* X, w4_dtype act_dtype, int64_t M
     if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
     const int B = fp4_block(format);
     cudaStream_t strm = as_stream(stream);
-    if (M > kDecodeMaxM) return W4_ERR_UNSUPPORTED;
+    if (M > kDecodeMaxM) {
+        CUtensorMap map;
+        if (!make_act_tensor_map(&map, X, false, M, K, w4p::BM)) return W4_ERR_CUDA;
+        w4p::PrefillParams pp;
+        std::memset(&pp, 0, sizeof(pp));
+        pp.qw = qweight;
+        pp.bscale = block_scales;
+        pp.tscale = tensor_scale;
+        pp.Y = Y;
+        pp.M = (int)M;
+        pp.N = (int)N;
+        pp.K = (int)K;
+        pp.group_size = B;
+        pp.G = (int)(K / B);
+        pp.out_dtype = (int)out_dtype;
+        pp.KA = (int)(K / 64);
+        pp.tiles = (int)(N / 16);
+        return format == W4_FP4_NVFP4 ? launch_prefill<false, w4p::kWNvfp4>(map, pp, dev, strm)
+                                      : launch_prefill<false, w4p::kWMxfp4>(map, pp, dev, strm);
+    }
     const size_t need = w4a16_fp4_workspace_bytes(M, N, K, format);
     if (need == 0) return W4_ERR_CUDA;
     if (!workspace || workspace_bytes < need) return W4_ERR_INVALID_ARG;

@@ -327,7 +327,11 @@ w4_status w4_fp4_quantize_pack(const void* W, w4_dtype w_dtype, int64_t N, int64
  * k, n) (* gs for NVFP4), fp32 accumulation.  fp16 activations only (every E2M1 value is
  * exact in fp16; bf16 returns W4_ERR_UNSUPPORTED).  M <= 64 runs the bandwidth-bound
  * decode kernel: each block's products are summed by the tensor cores and multiplied by
- * the block's scale in fp32.
+ * the block's scale (times gs) in fp32.  Larger M runs the tcgen05 prefill kernel on
+ * weights decoded to fp16 with their block scale (E2M1 x E4M3 and E2M1 x 2^e are exact in
+ * fp16 for e in [-13, 13]), the whole K accumulating in tensor memory and gs applied at
+ * the end; an MXFP4 block whose e lies outside [-13, 13] (other than the byte 0, whose
+ * block reads as zero) is reported as W4_ERR_DEVICE_ARG by w4_check_device_error().
  *   workspace  >= w4a16_fp4_workspace_bytes(M,N,K,format) bytes, 256-byte aligned,
  *              zero-filled before its first use (as for w4a16_gemm)
  */
@@ -379,7 +383,8 @@ w4_status w4_unpack_canonical(const uint32_t* qweight, int64_t N, int64_t K,
 
 /* Synchronises the current device, then reports and clears the device-side error word:
  * W4_ERR_TIMEOUT if a kernel gave up a bounded wait, W4_ERR_DEVICE_ARG if a kernel met
- * an out-of-range g_idx entry, W4_ERR_CUDA if the device reports a CUDA error, W4_OK.
+ * an out-of-range g_idx or permutation entry or an MXFP4 block scale the prefill kernel
+ * cannot decode exactly, W4_ERR_CUDA if the device reports a CUDA error, W4_OK.
  * On W4_ERR_TIMEOUT it also zeroes the current device's w4a16_gemm_noalloc scratch again
  * (a timed-out kernel may have left split-K flags in it); workspaces passed to
  * w4a16_gemm belong to the caller, who zeroes them again. */
@@ -393,6 +398,12 @@ w4_status w4_set_wait_limit_ns(uint64_t ns);
  * nothing completes; the bounded wait expires after the configured limit and sets the
  * device error word (so w4_check_device_error() then returns W4_ERR_TIMEOUT). */
 w4_status w4_selftest_expired_wait(w4_stream_t stream);
+
+/* Test aid for w4a16_gemm_noalloc's recovery: sets every split-K word of the current
+ * device's allocation-free scratch to a flagged stale partial (what a kernel that gave
+ * up a wait can leave behind).  A later w4a16_gemm_noalloc then adds those stale values
+ * into Y, until w4_check_device_error() reports a timeout and zeroes the scratch. */
+w4_status w4_selftest_noalloc_stale(w4_stream_t stream);
 
 /* Static string naming a status. */
 const char* w4_status_string(w4_status status);

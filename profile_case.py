@@ -1,7 +1,8 @@
 """Run one W4A16 GEMM case repeatedly, for a profiler to capture (ncu, CUDA events).
 
-    python -m bit_weight_only_w4_b200.profile_case decode  [--layer 2] [--m 1] [--iters 12]
-    python -m bit_weight_only_w4_b200.profile_case prefill [--layer 0] [--m 4096] [--iters 6]
+    python profile_case.py decode  [--layer 2] [--m 1] [--iters 12]
+    python profile_case.py prefill [--layer 0] [--m 4096] [--iters 6]
+    python profile_case.py chain   [--m 1] [--blocks 4] [--iters 3]
 
 decode:  one projection of the Llama-7B-shaped stack (layers 0..3 = qkv 4096x12288,
          o 4096x4096, gate_up 4096x22016, down 11008x4096), fp16 activations with s_inv,
@@ -9,6 +10,9 @@ decode:  one projection of the Llama-7B-shaped stack (layers 0..3 = qkv 4096x122
          hold the codes between launches.
 prefill: one 8B-shaped layer (0 = up 4096x14336, 1 = down 14336x4096), bf16
          activations already scaled, asymmetric INT4 g128.
+chain:   the decode step's projections as one layer sequence (w4a16_gemm_chain): --blocks
+         blocks of qkv -> o -> gate_up -> down, each fed from the previous output, one
+         weight copy per block (4 blocks = 430 MB of packed weights, above L2).
 
 Inputs are the seeded synthetic workloads of bit_weight_only_w4_b200.workloads, quantised
 on the GPU by w4_quantize_pack.  Nothing is checked here (the tests do that); the case only
@@ -25,7 +29,8 @@ def _bits(torch, a, dt):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("kind", choices=["decode", "prefill"])
+    ap.add_argument("kind", choices=["decode", "prefill", "chain"])
+    ap.add_argument("--blocks", type=int, default=4)
     ap.add_argument("--layer", type=int, default=None)
     ap.add_argument("--m", type=int, default=None)
     ap.add_argument("--iters", type=int, default=None)
@@ -49,6 +54,18 @@ def main(argv=None):
         for i in range(iters):
             q, s, z = copies[i % len(copies)]
             w4.w4a16_gemm(X, q, s, z, 128, s_inv=s_inv, Y=Y)
+    elif args.kind == "chain":
+        import os
+        import sys
+        sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+        import bench
+        layer = "all"
+        M = 1 if args.m is None else args.m
+        iters = 3 if args.iters is None else args.iters
+        _, projs, _ = bench.prepare_weights(w4, torch, n_layers=args.blocks)
+        layers, _, _ = bench.chain_layers(w4, torch, projs, M, n_blocks=args.blocks)
+        for _ in range(iters):
+            w4.w4a16_gemm_chain(layers)
     else:
         layer = 0 if args.layer is None else args.layer
         M = 4096 if args.m is None else args.m

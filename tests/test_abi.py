@@ -257,6 +257,33 @@ def test_chain_rejects_bad_arguments(L):
     assert L.w4a16_chain_workspace_bytes(0) == 0 and L.w4a16_chain_workspace_bytes(9) == 0
 
 
+def test_fp4_entry_points_reject_bad_arguments(L):
+    """The FP4 quantiser and GEMM check formats, shapes and pointers before any CUDA call."""
+    v = ctypes.c_void_p
+    q = lambda **kw: L.w4_fp4_quantize_pack(  # noqa: E731
+        v(kw.get("W", 256)), kw.get("wdt", 0), kw.get("N", 256), kw.get("K", 256), kw.get("fmt", 0),
+        v(kw.get("qw", 256)), v(kw.get("bs", 256)),
+        None if kw.get("ts", 256) is None else v(kw.get("ts", 256)), None)
+    assert q(fmt=2) == w4.W4_ERR_INVALID_ARG                  # no such format
+    assert q(fmt=1) == w4.W4_ERR_INVALID_ARG                  # MXFP4 has no tensor scale
+    assert q(fmt=0, ts=None) == w4.W4_ERR_INVALID_ARG         # NVFP4 needs one
+    assert q(wdt=2) == w4.W4_ERR_INVALID_ARG                  # fp32 weights
+    assert q(N=8) == w4.W4_ERR_UNSUPPORTED                    # N % 16
+    assert q(K=96) == w4.W4_ERR_UNSUPPORTED                   # K % 64
+    assert q(W=0) == w4.W4_ERR_INVALID_ARG
+    g = lambda **kw: L.w4a16_fp4_gemm(  # noqa: E731
+        v(kw.get("X", 256)), kw.get("act", 0), kw.get("M", 1), kw.get("N", 256), kw.get("K", 256),
+        v(256), v(kw.get("bs", 256)), None if kw.get("ts", 256) is None else v(kw.get("ts", 256)),
+        kw.get("fmt", 0), v(256), kw.get("out", 0), v(256), 1 << 30, None)
+    assert g(act=1) == w4.W4_ERR_UNSUPPORTED                  # bf16 activations
+    assert g(act=2) == w4.W4_ERR_INVALID_ARG
+    assert g(fmt=1) == w4.W4_ERR_INVALID_ARG                  # MXFP4 with a tensor scale
+    assert g(ts=None) == w4.W4_ERR_INVALID_ARG                # NVFP4 without
+    assert g(X=264) == w4.W4_ERR_INVALID_ARG                  # misaligned
+    assert g(M=0) == w4.W4_OK
+    assert L.w4a16_fp4_workspace_bytes(1, 8, 256, 0) == 0
+
+
 def test_library_builds_without_warnings(L):
     """nvcc's log of the in-tree build holds no warning (an unused function, a narrowing
     conversion, a missing return...).  ptxas reports no spill in the one-token-tile decode

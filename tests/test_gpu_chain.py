@@ -88,11 +88,16 @@ def test_chain_small_matches_oracle_chain(M):
 
 
 def test_chain_longer_than_one_launch_in_a_graph():
-    """40 layers: two launches (32 + 8); the output of layer 31 crosses the launch
-    boundary.  Captured in a CUDA graph and replayed."""
+    """40 layers: two launches (32 + 8).  Layers 31 -> 32 -> 33 read their predecessor
+    across the launch boundary (as do 1 and 2 at the start); the others read the block
+    input, so no dependency path is longer than four layers (each layer adds about 1.5e-4
+    of relative error against the oracle -- the fp32 fold of the biased codes and the fp16
+    output -- and a 40-deep path would add up to the stated bound by itself).  Captured
+    in a CUDA graph and replayed."""
     skip_without_gpu()
     import torch
-    specs = [(256, 256, -1, 0)] + [(256, 256, j, 0) for j in range(39)]
+    chained = {1, 2, 31, 32, 33}
+    specs = [(256, 256, -1, 0)] + [(256, 256, j - 1 if j in chained else -1, 0) for j in range(1, 40)]
     M = 2
     layers, ref32, _ = _build(M, specs, seed=7)
     _run(layers)                               # eager once

@@ -126,6 +126,14 @@ def test_fp4_gemm_ragged_shapes(fmt, N, K):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M,N,K", [(65, 256, 1024), (200, 384, 2048), (512, 144, 320)])
+def test_fp4_gemm_prefill(fmt, M, N, K):
+    """M > 64: the tcgen05 kernel on weights decoded with their block scale."""
+    skip_without_gpu()
+    _gemm_case(M, N, K, fmt)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
 def test_fp4_gemm_fp32_output(fmt):
     skip_without_gpu()
     _gemm_case(4, 512, 2048, fmt, out="fp32")
@@ -157,6 +165,35 @@ def test_fp4_llama7b_layers_m1(fmt, layer):
         What = oracle.mxfp4_dequant(codes, es)
     Y_ref = oracle.gemm_f32(oracle.f16_to_f32(li.X), What.astype(np.float32))
     check_y(to_f64(Y)[:, ns], Y_ref, "fp16")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("layer", [0, 1])
+def test_fp4_llama8b_prefill_m4096(fmt, layer):
+    """The 8B-shaped prefill projections at M = 4096 with fp16 activations (the FP4 path
+    takes fp16), oracle on sampled output rows and columns."""
+    skip_without_gpu()
+    import torch
+    wl = workloads.workload(4)
+    L = wl.layers[layer]
+    M = 4096
+    W_bits = workloads.gen_weights(L.N, L.K, 0, 4, layer).view(np.uint16)
+    X_bits = workloads.gen_acts(M, L.K, 0, 4, layer, "fp16")
+    qw, bsd, tsd = w4.w4_fp4_quantize_pack(dev_bits(W_bits, torch.float16), fmt)
+    Y = w4.w4a16_fp4_gemm(dev_bits(X_bits, torch.float16), qw, bsd, tsd, fmt, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    rng = np.random.default_rng(layer + 40)
+    ms = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, 24)]))
+    ns = np.unique(np.concatenate([[0, L.N - 1], rng.integers(0, L.N, 128)]))
+    if fmt == "nvfp4":
+        codes, bs, gs = oracle.nvfp4_quantize(W_bits)
+        What = oracle.nvfp4_dequant(codes[ns], bs[ns], gs)
+    else:
+        codes, es = oracle.mxfp4_quantize(W_bits[ns])
+        What = oracle.mxfp4_dequant(codes, es)
+    Y_ref = oracle.gemm_f32(oracle.f16_to_f32(X_bits), What.astype(np.float32), rows=ms)
+    check_y(to_f64(Y)[np.ix_(ms, ns)], Y_ref, "fp32")
 
 
 def test_fp4_gemm_refuses_bf16_activations():
