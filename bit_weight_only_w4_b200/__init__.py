@@ -65,8 +65,8 @@ def lib():
         L.w4_check_device_error.restype = st
         L.w4_set_wait_limit_ns.argtypes = [u64]
         L.w4_set_wait_limit_ns.restype = st
-        L.w4_selftest_noalloc_stale.argtypes = [vp]
-        L.w4_selftest_noalloc_stale.restype = st
+        L.w4_selftest_noalloc_scratch.argtypes = [i32, ctypes.POINTER(u64)]
+        L.w4_selftest_noalloc_scratch.restype = st
         L.w4_selftest_expired_wait.argtypes = [vp]
         L.w4_selftest_expired_wait.restype = st
         L.w4_status_string.argtypes = [st]

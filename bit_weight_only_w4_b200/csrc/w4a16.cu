@@ -784,24 +784,47 @@ cudaError_t noalloc_rezero(int dev) {
     return e;
 }
 
-// Test aid: every split-K word of the scratch set to a flagged partial of 1.0.
+// Test aid: every split-K word of the scratch set to a flagged partial of 1.0, or the
+// nonzero words counted.
+__device__ unsigned long long g_w4_selftest_count;
+
 __global__ void plant_stale_kernel(unsigned long long* words, size_t n) {
     const unsigned long long w = (1ull << 32) | (unsigned long long)__float_as_uint(1.0f);
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
         words[i] = w;
 }
 
+__global__ void count_nonzero_kernel(const unsigned long long* words, size_t n) {
+    unsigned long long c = 0;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        c += words[i] != 0ull;
+    if (c) atomicAdd(&g_w4_selftest_count, c);
+}
+
 }  // namespace
 
-extern "C" w4_status w4_selftest_noalloc_stale(w4_stream_t stream) {
+extern "C" w4_status w4_selftest_noalloc_scratch(int32_t plant, uint64_t* nonzero_words) {
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    if (!plant && !nonzero_words) return W4_ERR_INVALID_ARG;
     unsigned char* ws = reinterpret_cast<unsigned char*>(noalloc_scratch(dev));
     if (!ws) return W4_ERR_CUDA;
+    unsigned long long* words = reinterpret_cast<unsigned long long*>(ws + kCounterBytes);
     const size_t n = (kNoAllocScratchBytes - kCounterBytes) / 8;
-    plant_stale_kernel<<<256, 256, 0, as_stream(stream)>>>(
-        reinterpret_cast<unsigned long long*>(ws + kCounterBytes), n);
-    return launch_status();
+    if (plant) {
+        plant_stale_kernel<<<256, 256>>>(words, n);
+        if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return W4_ERR_CUDA;
+        if (nonzero_words) *nonzero_words = n;
+        return W4_OK;
+    }
+    const unsigned long long zero = 0;
+    if (cudaMemcpyToSymbol(g_w4_selftest_count, &zero, sizeof(zero)) != cudaSuccess) return W4_ERR_CUDA;
+    count_nonzero_kernel<<<256, 256>>>(words, n);
+    unsigned long long c = 0;
+    if (cudaGetLastError() != cudaSuccess || cudaMemcpyFromSymbol(&c, g_w4_selftest_count, sizeof(c)) != cudaSuccess)
+        return W4_ERR_CUDA;
+    *nonzero_words = c;
+    return W4_OK;
 }
 
 extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64_t M, int64_t N,

@@ -399,11 +399,12 @@ w4_status w4_set_wait_limit_ns(uint64_t ns);
  * device error word (so w4_check_device_error() then returns W4_ERR_TIMEOUT). */
 w4_status w4_selftest_expired_wait(w4_stream_t stream);
 
-/* Test aid for w4a16_gemm_noalloc's recovery: sets every split-K word of the current
- * device's allocation-free scratch to a flagged stale partial (what a kernel that gave
- * up a wait can leave behind).  A later w4a16_gemm_noalloc then adds those stale values
- * into Y, until w4_check_device_error() reports a timeout and zeroes the scratch. */
-w4_status w4_selftest_noalloc_stale(w4_stream_t stream);
+/* Test aid for w4a16_gemm_noalloc's recovery, on the current device (synchronous).
+ * plant != 0: sets every split-K word of the allocation-free scratch to a flagged stale
+ * partial (what a kernel that gave up a wait can leave behind); *nonzero_words, if not
+ * NULL, receives the number of words written.  plant == 0: counts the scratch's nonzero
+ * split-K words into *nonzero_words (0 once w4_check_device_error() has zeroed it). */
+w4_status w4_selftest_noalloc_scratch(int32_t plant, uint64_t* nonzero_words);
 
 /* Static string naming a status. */
 const char* w4_status_string(w4_status status);

@@ -69,9 +69,9 @@ def test_our_arm_prints_every_contract_key(monkeypatch, capsys):
     step_bytes = bench.N_LAYERS * 4_000_000
     monkeypatch.setattr(bench, "prepare_weights", lambda w4, torch: (wl, projs, step_bytes))
     clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
-    monkeypatch.setattr(bench, "time_chain", lambda *a, **k: (100.0, clk, 10 * 4))
+    monkeypatch.setattr(bench, "time_chain_per_launch", lambda *a, **k: (100.0, clk))
     monkeypatch.setattr(bench, "time_chain_e2e", lambda *a, **k: (200.0, 32768, 98304))
-    monkeypatch.setattr(bench, "time_chain_per_launch", lambda *a, **k: 150.0)
+    monkeypatch.setattr(bench, "time_chain", lambda *a, **k: (150.0, None, 10 * 4))
     monkeypatch.setattr(bench, "time_decode", lambda *a, **k: {
         "total_ms": 40.0, "launches": 3 * bench.N_LAYERS * len(projs), "clocks": None,
         "per_layer": {"qkv": 10.0}})
@@ -102,6 +102,6 @@ def test_our_arm_prints_every_contract_key(monkeypatch, capsys):
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == 0.04 * cb["cores"]
     assert cb["single_thread"]["cores"] == 1 and "cpu_model" in cb and cb["nproc"] >= 1
-    assert line["gpu_launches"] == 10 * 4
-    assert line["step_per_launch"]["ms_per_step"] == 15.0
+    assert line["gpu_launches"] == 10 * bench.N_LAYERS * 4
+    assert line["step_layer_sequence"]["ms_per_step"] == 15.0
     assert "workload" in line["config"]

@@ -85,25 +85,25 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     w4.w4_check_device_error()
 
 
+def _scratch(plant):
+    n = ctypes.c_uint64(0)
+    assert w4.lib().w4_selftest_noalloc_scratch(int(plant), ctypes.byref(n)) == w4.W4_OK
+    return n.value
+
+
 def test_noalloc_recovers_after_a_timed_out_call():
     """A kernel that gives up a bounded wait can leave flagged split-K partials in the
-    shared scratch, which a later call would add into Y.  The test plants such stale words
-    (a test aid writes them; nothing faults), shows that a call then goes wrong, plants
-    them again, lets a bounded wait expire (the watchdog's self-test kernel), and checks
-    that w4_check_device_error reports the timeout, zeroes the scratch, and that the next
-    two calls match the oracle."""
+    shared scratch, which a later call could add into Y.  The test plants such stale words
+    (a test aid writes them; nothing faults), lets a bounded wait expire (the watchdog's
+    self-test kernel), and checks that w4_check_device_error reports the timeout and
+    leaves no nonzero word in the scratch, and that the next two calls match the oracle."""
     skip_without_gpu()
-    import torch
     M, N, K, g = 1, 4096, 4096, 128
     d, Y_ref = _layer(M, N, K, g)
     _run_noalloc(d, M, N, g)                       # scratch set up, device clean
-    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    L = w4.lib()
-    assert L.w4_selftest_noalloc_stale(stream) == w4.W4_OK
-    Y = _run_noalloc(d, M, N, g)
-    err = np.abs(Y - Y_ref).max()
-    assert err > 0.5, f"stale partials were not picked up (max err {err})"
-    assert L.w4_selftest_noalloc_stale(stream) == w4.W4_OK
+    assert _scratch(plant=False) == 0              # every call leaves it zeroed
+    planted = _scratch(plant=True)
+    assert planted > 0 and _scratch(plant=False) == planted
     w4.w4_set_wait_limit_ns(2_000_000)
     try:
         w4.w4_selftest_expired_wait()
@@ -112,5 +112,6 @@ def test_noalloc_recovers_after_a_timed_out_call():
         assert e.value.status == w4.W4_ERR_TIMEOUT
     finally:
         w4.w4_set_wait_limit_ns(2_000_000_000)
+    assert _scratch(plant=False) == 0
     for _ in range(2):
         check_y(_run_noalloc(d, M, N, g), Y_ref, "fp16")
