@@ -60,8 +60,12 @@ template <int NT>
 struct Cfg {
     static constexpr int tpw = NT <= 2 ? 2 : 1;          // row tiles per MMA warp
     static constexpr int aps = NT == 1 ? 8 : 4;          // atoms (64-channel blocks) per stage
-    static constexpr int xw = NT == 1 ? 1 : NT <= 4 ? 3 : 4;   // activation warps
-    static constexpr int mma_warps = NT <= 4 ? 16 : 8;
+    // no activation warps: X' and its sums arrive prepared (resident, or copied per stage
+    // from the copy prep_acts_kernel wrote); every warp but the producer is an MMA warp
+    static constexpr int xw = 0;
+    // 17 warps with one or two token tiles; 9 with more, so that their larger
+    // accumulator sets fit the registers (9 warps allow 168 a thread)
+    static constexpr int mma_warps = NT <= 2 ? 16 : 8;
     static constexpr int groups = mma_warps / 8;         // stage-parity groups
     static constexpr int stage_warps = mma_warps / groups;   // MMA warps sharing a stage
     static constexpr int tsets = 8 / tpw;                // row-tile sets of a band
@@ -107,6 +111,9 @@ struct DecodeParams {
     int off_x, off_xs, off_sx, off_si, off_sc, off_zr, off_gi, off_desc, stage_bytes;
     int ldx;                  // row stride of X in elements (read by the layer-sequence kernel)
     int srow_bytes;           // bytes of one staged scale row: 256 (fp16 x 128), 128 (FP4 bytes)
+    const float* sg32;        // staged X': sums of X' over 32 / 64 / 128 channels,
+    const float* sg64;        // [segment][8 NT] fp32 (tokens >= M zero), written by
+    const float* sg128;       // prep_acts_kernel
     const float* tscale;      // NVFP4 tensor scale (device fp32), else null
 };
 
@@ -638,84 +645,54 @@ W4_DEV void consume_gidx(const StageView& v, const DecodeParams& p, const Lane& 
     }
 }
 
-// ---------------------------------------------------------------- activation warps
-// Per stage: X' = X * s_inv rounded to the activation type (a plain copy without s_inv)
-// into the stage's X' buffer, which the MMA warps read, and the sums of X' over 32, 64 and
-// 128 consecutive channels per token.  The stage's channels form 8-channel chunks (column
-// block c/8, 16-byte chunk c%8); each warp pass covers 32 consecutive chunks of one token.
-template <int NT, bool BF16, bool GIDX>
-W4_DEV void prep_stage(unsigned char* st, const DecodeParams& p, int na, int xw, int lane) {
-    using C = Cfg<NT>;
-    constexpr int CPT = 8 * C::aps;    // chunks per token
-    const unsigned char* xb = st + p.off_x;
-    unsigned char* xs = st + p.off_xs;
-    float* sx = reinterpret_cast<float*>(st + p.off_sx);
-    const float* si = reinterpret_cast<const float*>(st + p.off_si);
-    // two passes (token-row chunks base and base + 32 * xw) per iteration, their loads
-    // issued together
-    for (int base = 32 * xw; base < p.M * CPT; base += 64 * C::xw) {
-        int mm[2], cc[2];
-        bool act[2], ld[2];
-        uint4 v[2];
-        float sv[2][8];
+// ---------------------------------------------------------------- prepared activations
+// X' = X * s_inv rounded to the activation type (a plain copy without s_inv) and its sums
+// over every 32, 64 and 128 channels, once per GEMM, for the decode kernel's staged
+// activations: X' [M, K] with the 16-byte chunks of every 128-byte block permuted by the
+// row (chunk c of row m at c ^ (m & 7), the bank-conflict-free order the MMA warps read),
+// so that one tensor copy per stage lands it in shared memory as [row][block][128 B];
+// sums [segment][mpad], rows M..mpad-1 zero.  Thread t takes 8-channel chunk t % (K/8)
+// of token row t / (K/8): consecutive lanes hold consecutive chunks of one row, so the
+// sums are warp shuffles.
+template <bool BF16>
+__global__ void prep_acts_kernel(const void* __restrict__ X, const float* __restrict__ s_inv, int M, int K,
+                                 int mpad, void* __restrict__ Xp, float* __restrict__ s32,
+                                 float* __restrict__ s64, float* __restrict__ s128) {
+    const int cpt = K / 8;
+    const size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    const bool valid = t < (size_t)mpad * cpt;
+    const int m = valid ? (int)(t / cpt) : 0, c = valid ? (int)(t % cpt) : 0;
+    float s = 0.0f;
+    if (valid && m < M) {
+        uint4 v = reinterpret_cast<const uint4*>(X)[(size_t)m * cpt + c];
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        if (s_inv) {
+            const float4 a = __ldg(reinterpret_cast<const float4*>(s_inv) + 2 * c);
+            const float4 b = __ldg(reinterpret_cast<const float4*>(s_inv) + 2 * c + 1);
+            const float sv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int b = base + 32 * C::xw * u;
-            act[u] = b < p.M * CPT;
-            mm[u] = b / CPT;
-            cc[u] = b % CPT + lane;
-            ld[u] = act[u] && cc[u] < 8 * na;
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) sv[u][i] = 1.0f;
-            if (ld[u]) {
-                // the tensor box holds M rows per column block, 128B-swizzled by line index
-                const int line = (cc[u] >> 3) * p.M + mm[u];
-                v[u] = ld_u128(xb + line * 128 + (((cc[u] & 7) ^ (line & 7)) << 4));
-                if (p.s_inv) {
-                    const float4 s0 = *reinterpret_cast<const float4*>(si + 8 * cc[u]);
-                    const float4 s1 = *reinterpret_cast<const float4*>(si + 8 * cc[u] + 4);
-                    sv[u][0] = s0.x; sv[u][1] = s0.y; sv[u][2] = s0.z; sv[u][3] = s0.w;
-                    sv[u][4] = s1.x; sv[u][5] = s1.y; sv[u][6] = s1.z; sv[u][7] = s1.w;
-                }
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = unpack2<BF16>(w[i]);
+                w[i] = pack2<BF16>(__fmul_rn(f.x, sv[2 * i]), __fmul_rn(f.y, sv[2 * i + 1]));
             }
         }
+        const int blk = c >> 3, ch = c & 7;
+        reinterpret_cast<uint4*>(Xp)[(size_t)m * cpt + 8 * blk + (ch ^ (m & 7))] = make_uint4(w[0], w[1], w[2], w[3]);
+        float2 f[4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (!act[u]) break;
-            const int m = mm[u], c = cc[u];
-            const int blk = c >> 3, ch = c & 7;
-            float s = 0.0f;
-            if (ld[u]) {
-                uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                if (p.s_inv) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 f = unpack2<BF16>(w[i]);
-                        w[i] = pack2<BF16>(__fmul_rn(f.x, sv[u][2 * i]), __fmul_rn(f.y, sv[u][2 * i + 1]));
-                    }
-                }
-                // X': [token row][column block][128 B], lines swizzled by token row
-                *reinterpret_cast<uint4*>(xs + m * (C::aps * 128) + blk * 128 + ((ch ^ (m & 7)) << 4)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-                if constexpr (!GIDX) {
-                    float2 f[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) f[i] = unpack2<BF16>(w[i]);
-                    s = ((f[0].x + f[0].y) + (f[1].x + f[1].y)) + ((f[2].x + f[2].y) + (f[3].x + f[3].y));
-                }
-            }
-            if constexpr (!GIDX) {
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                if ((lane & 3) == 0) sx[(C::sx32 + (c >> 2)) * C::mpad + m] = s;
-                s += __shfl_xor_sync(0xffffffffu, s, 4);
-                if ((lane & 7) == 0) sx[(C::sx64 + (c >> 3)) * C::mpad + m] = s;
-                s += __shfl_xor_sync(0xffffffffu, s, 8);
-                if ((lane & 15) == 0) sx[(C::sx128 + (c >> 4)) * C::mpad + m] = s;
-            }
-        }
+        for (int i = 0; i < 4; ++i) f[i] = unpack2<BF16>(w[i]);
+        s = ((f[0].x + f[0].y) + (f[1].x + f[1].y)) + ((f[2].x + f[2].y) + (f[3].x + f[3].y));
     }
+    // groups of 4 / 8 / 16 consecutive chunks are aligned to 32 / 64 / 128 channels (K is a
+    // multiple of 64; the 128-channel sums are only read when K is a multiple of 128)
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    if (valid && (lane & 3) == 0) s32[(c >> 2) * mpad + m] = s;
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    if (valid && (lane & 7) == 0) s64[(c >> 3) * mpad + m] = s;
+    s += __shfl_xor_sync(0xffffffffu, s, 8);
+    if (valid && (lane & 15) == 0 && (c >> 4) < K / 128) s128[(c >> 4) * mpad + m] = s;
 }
 
 // Resident activations (one token tile, small M*K): X' = X * s_inv for the whole of K and
@@ -983,6 +960,28 @@ W4_DEV int total_stages(const DecodeParams& p, const PartIter& it, int u0, int u
     return n;
 }
 
+// Staged activations of a stage: the prepared X' box ([8*NT rows][aps blocks][128 B],
+// rows >= M and blocks beyond K zero-filled) and, unless act-order folds the scales into
+// the weights, the sums over its 32-, 64- and 128-channel segments ([segment][8*NT]).
+template <int NT, bool GIDX>
+W4_DEV uint32_t staged_act_bytes(int na) {
+    using C = Cfg<NT>;
+    return C::aps * C::mpad * 128 + (GIDX ? 0 : (2 * na + na + (na + 1) / 2) * C::mpad * 4);
+}
+
+template <int NT, bool GIDX>
+W4_DEV void load_staged_acts(const DecodeParams& p, unsigned char* st, const CUtensorMap* tmap_x, int a0, int na,
+                             uint64_t* bar) {
+    using C = Cfg<NT>;
+    tma_load_3d(st + p.off_x, tmap_x, 0, a0, 0, bar);
+    if constexpr (!GIDX) {
+        unsigned char* sx = st + p.off_sx;
+        bulk_g2s(sx + C::sx32 * C::mpad * 4, p.sg32 + (size_t)(2 * a0) * C::mpad, 2 * na * C::mpad * 4, bar);
+        bulk_g2s(sx + C::sx64 * C::mpad * 4, p.sg64 + (size_t)a0 * C::mpad, na * C::mpad * 4, bar);
+        bulk_g2s(sx + C::sx128 * C::mpad * 4, p.sg128 + (size_t)(a0 / 2) * C::mpad, (na + 1) / 2 * C::mpad * 4, bar);
+    }
+}
+
 // Ring position: slot and phase parity of consecutive stages.
 struct Ring {
     int s = 0, ph = 0;
@@ -1006,8 +1005,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
     unsigned char* smem = align_smem_1024(smem_raw);
     unsigned char* xchg = smem + p.off_xchg;
     uint64_t* full = reinterpret_cast<uint64_t*>(xchg + C::xchg_bytes);
-    uint64_t* xready = full + kMaxStages;
-    uint64_t* empty = xready + kMaxStages;
+    uint64_t* empty = full + kMaxStages;
     volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1018,21 +1016,17 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&xready[s], 32 * C::xw);
             mbar_init(&empty[s], C::stage_warps);
         }
         *s_abort = 0;
         fence_mbar_init();
     }
-    // activation sums and X' rows of tokens >= M are never written: start from zero
+    // resident activation sums of tokens >= M are never written: start from zero (staged
+    // X' and sums arrive with rows >= M zero)
     if (p.xres) {
         const int words = (p.K / 32 + p.K / 64 + p.K / 128) * p.sstride;
         for (int i = threadIdx.x; i < words; i += C::threads)
             reinterpret_cast<float*>(smem + p.off_res_s)[i] = 0.0f;
-    } else if (p.M < C::mpad) {
-        const int words = (p.off_si - p.off_xs) / 4;   // X' and sums of one stage
-        for (int i = threadIdx.x; i < S * words; i += C::threads)
-            reinterpret_cast<uint32_t*>(smem + (i / words) * p.stage_bytes + p.off_xs)[i % words] = 0u;
     }
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmap_x);
@@ -1053,10 +1047,11 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
         // ------------------------------------------------------------ producer
         // lane 0 arms the stage's barrier and issues one copy per operand: the codes
         // (a contiguous run of the band), the scale and zero-point rows (2-D boxes) or the
-        // g_idx slice, the activations (3-D box: 4 column blocks x 8*NT token rows, rows
-        // >= M and blocks beyond K zero-filled) and the s_inv slice.  The read-only weight
-        // operands of the first stages go out before pdl_wait(), the activations (possibly
-        // produced by the preceding kernel) after it.
+        // g_idx slice and, with staged activations, the prepared X' (3-D box: 8*NT token
+        // rows x the stage's column blocks, rows >= M and blocks beyond K zero-filled) and
+        // its three slices of sums.  The read-only weight operands of the first stages go
+        // out before pdl_wait(), the activations (written by the preparation kernel just
+        // before) after it.
         const uint64_t policy = policy_evict_first();
         const int total = total_stages<UPS>(p, it, u0, u1);
         const int pro = min(S, total);
@@ -1100,7 +1095,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                     desc[1] = make_int4(kg[0], kg[1], kg[2], kg[3]);
                     desc[2] = make_int4(kg[4], kg[5], kg[6], kg[7]);
                     uint32_t bytes = na * tb * 512;
-                    if (!p.xres) bytes += C::aps * p.M * 128 + (p.s_inv ? na * 256 : 0);
+                    if (!p.xres) bytes += staged_act_bytes<NT, GIDX>(na);
                     if (GIDX) bytes += na * 256;
                     else bytes += p.ngs * (MODE == kModeNvfp4 || MODE == kModeMxfp4 ? 128 : 256) * (p.zeros ? 2 : 1);
                     mbar_arrive_expect_tx(&full[r.s], bytes);
@@ -1112,10 +1107,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                         tma_load_2d(st + p.off_sc, &tmap_sc, band * kBandRows, g_first, &full[r.s]);
                         if (p.zeros) tma_load_2d(st + p.off_zr, &tmap_zr, band * kBandRows, g_first, &full[r.s]);
                     }
-                    if (i >= S && !p.xres) {
-                        tma_load_3d(st + p.off_x, &tmap_x, 0, 0, a0, &full[r.s]);
-                        if (p.s_inv) bulk_g2s(st + p.off_si, p.s_inv + 64 * a0, na * 256, &full[r.s]);
-                    }
+                    if (i >= S && !p.xres) load_staged_acts<NT, GIDX>(p, st, &tmap_x, a0, na, &full[r.s]);
                 }
                 if (i == pro - 1 && !p.xres) {
                     // the activations of the first stages, once the preceding grid is done
@@ -1128,10 +1120,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                             int aj, nj;
                             stage_atoms<UPS>(p, bj, qs, qe, sj, aj, nj);
                             unsigned char* sk = smem + k * p.stage_bytes;
-                            if (lane == 0) {
-                                tma_load_3d(sk + p.off_x, &tmap_x, 0, 0, aj, &full[k]);
-                                if (p.s_inv) bulk_g2s(sk + p.off_si, p.s_inv + 64 * aj, nj * 256, &full[k]);
-                            }
+                            if (lane == 0) load_staged_acts<NT, GIDX>(p, sk, &tmap_x, aj, nj, &full[k]);
                         }
                     }
                 }
@@ -1153,27 +1142,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                             warp - 1, C::warps - 1, lane);
         named_bar_sync(3, C::threads - 32);
     }
-    if (warp <= C::xw) {
-        // ------------------------------------------------------------ activation warps
-        if (p.xres) return;
-        const int xw = warp - 1;
-        bool aborted = false;
-        Ring r;
-        for (int pi = 0; pi < it.count(); ++pi) {
-            const int band = it.band(pi);
-            const int ps = max(u0, band * p.KU), pe = min(u1, (band + 1) * p.KU);
-            for (int stg = 0; UPS * stg < pe - ps; ++stg, r.next(S)) {
-                int a0, na;
-                stage_atoms<UPS>(p, band, ps, pe, stg, a0, na);
-                if (!aborted) {
-                    aborted = *s_abort || !mbar_wait(&full[r.s], r.ph);
-                    if (aborted) *s_abort = 1;
-                }
-                if (!aborted) prep_stage<NT, BF16, GIDX>(smem + r.s * p.stage_bytes, p, na, xw, lane);
-                mbar_arrive(&xready[r.s]);
-            }
-        }
-    } else {
+    {
         // ------------------------------------------------------------ MMA warps
         pdl_wait();   // before any store to Y or the workspace
         constexpr int TPW = C::tpw;
@@ -1182,7 +1151,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
         const int kp = ws / C::tsets;                  // K slice of the stage
         const int t0 = TPW * (ws % C::tsets);          // first row tile
         const int set = grp * C::kparts + kp;          // partial-sum set at a flush
-        const int xrows = NT == 1 ? p.M : C::mpad;
+        const int xrows = p.xres ? p.M : C::mpad;   // staged X' rows >= M are zero
         const int sstride = p.xres ? p.sstride : C::mpad;
         const Lane L = make_lane(lane, xrows, sstride, p.xres ? p.K / 64 * 128 : C::aps * 128);
         float acc[TPW][NT][4];
@@ -1197,7 +1166,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
             for (int stg = 0; UPS * stg < pe - ps; ++stg, ++i, r.next(S)) {
                 if ((i % C::groups) != grp) continue;   // the other group's stage
                 if (!aborted) {
-                    aborted = *s_abort || !mbar_wait(p.xres ? &full[r.s] : &xready[r.s], r.ph);
+                    aborted = *s_abort || !mbar_wait(&full[r.s], r.ph);
                     if (aborted) *s_abort = 1;
                 }
                 unsigned char* st = smem + r.s * p.stage_bytes;
@@ -1217,7 +1186,7 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
                         v.sx64 = rs + (p.K / 32 + a0) * sstride * 4;
                         v.sx128 = rs + (p.K / 32 + p.K / 64 + a0 / 2) * sstride * 4;
                     } else {
-                        v.x = st + p.off_xs;
+                        v.x = st + p.off_x;
                         v.sx32 = st + p.off_sx + C::sx32 * C::mpad * 4;
                         v.sx64 = st + p.off_sx + C::sx64 * C::mpad * 4;
                         v.sx128 = st + p.off_sx + C::sx128 * C::mpad * 4;

@@ -86,8 +86,39 @@ constexpr size_t kCounterBytes = (size_t)kMaxBands * 4;   // 32 KB
 size_t decode_slot_bytes(int NT, int sms) { return (size_t)sms * w4d::kTilesPerBand * NT * 4 * 32 * 8; }
 size_t slot_region_bytes(int sms) { return decode_slot_bytes(8, sms); }
 
-size_t decode_workspace_bytes(int64_t M, int sms) {
-    return kCounterBytes + decode_slot_bytes(decode_tiles_for(M), sms);
+// Behind the zero region and the split-K slots of the largest token-tile count the
+// workspace serves (8 for a caller's workspace, whatever the call's M; the no-allocation
+// scratch serves at most 4): the decode kernel's prepared activations (X' and its sums;
+// prep_acts_kernel), or the prefill kernel's scaled activations.  Calls of different M
+// sharing one workspace thus never find another call's activations where their split-K
+// flags are.
+size_t pre_offset(int max_tiles, int sms) { return kCounterBytes + decode_slot_bytes(max_tiles, sms); }
+
+// Prepared activations of the decode kernel: X' [M, K] (act type), then the sums over 32,
+// 64 and 128 channels, [K/32 | K/64 | ceil(K/128)][8 NT] fp32.
+struct PreLayout {
+    size_t x, s32, s64, s128, bytes;
+};
+PreLayout pre_layout(int64_t M, int64_t K) {
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    const size_t mpad = 8 * (size_t)decode_tiles_for(M);
+    PreLayout L;
+    L.x = 0;
+    L.s32 = up((size_t)M * (size_t)K * 2);
+    L.s64 = L.s32 + up((size_t)(K / 32) * mpad * 4);
+    L.s128 = L.s64 + up((size_t)(K / 64) * mpad * 4);
+    L.bytes = L.s128 + up((size_t)((K + 127) / 128) * mpad * 4);
+    return L;
+}
+
+size_t decode_workspace_bytes(int64_t M, int64_t K, int sms, int max_tiles = 8) {
+    return pre_offset(max_tiles, sms) + pre_layout(M, K).bytes;
+}
+
+// Act-order GEMM in permuted order with the gather kernel: the gathered activations go
+// behind what the GEMM on them uses (the decode kernel prepares its X' from them).
+size_t perm_gather_offset(int64_t M, int64_t K, int sms) {
+    return M <= kDecodeMaxM ? decode_workspace_bytes(M, K, sms) : pre_offset(8, sms);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -124,20 +155,21 @@ bool make_act_tensor_map(CUtensorMap* map, const void* X, bool bf16, int64_t M, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D view of activations [M,K] as (64 channels, M rows, K/64 column blocks): one box of
-// 4 column blocks x box_rows rows lands as [block][row][64], each row a 128-byte swizzled
-// line; rows >= M and blocks beyond K/64 are zero-filled.
+// 3-D view of prepared activations X' [M,K] as (64 channels, K/64 column blocks, M rows):
+// one box of `blocks` column blocks x box_rows rows lands as [row][block][64] (X' is
+// stored with its chunks already permuted, so no swizzle here); rows >= M and blocks
+// beyond K/64 are zero-filled.
 bool make_act_blocks_map(CUtensorMap* map, const void* X, bool bf16, int64_t M, int64_t K,
                          int box_rows, int blocks) {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return false;
-    const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
-    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
-    const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, (cuuint32_t)blocks};
+    const cuuint64_t dims[3] = {64, (cuuint64_t)(K / 64), (cuuint64_t)M};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)K * 2};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)blocks, (cuuint32_t)box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                const_cast<void*>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -165,7 +197,7 @@ bool decode_x_resident(int64_t M, int64_t K) {
 }
 
 template <int NT, bool BF16, int MODE, bool PERM>
-w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
+w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, size_t pre_off, int dev,
                         cudaStream_t stream) {
     using C = w4d::Cfg<NT>;
     constexpr bool GIDX = MODE == w4d::kModeGidx;
@@ -189,21 +221,20 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     if (PERM != (p.perm != nullptr) || (PERM && !p.xres))   // the gather is part of the resident X'
         return W4_ERR_UNSUPPORTED;
     p.sstride = p.xres ? sstride_res : C::mpad;
-    // stage layout: codes | activation box (M rows) | X' | activation sums | s_inv |
-    // scale rows | zero-point rows | g_idx   (no activation parts when X' is resident)
+    // stage layout: codes | X' box (8*NT rows) | activation sums | scale rows | zero-point
+    // rows | g_idx | descriptor   (no activation parts when X' is resident)
     const int g = p.group_size;
     const int span = 64 * C::aps;   // input channels per stage
-    const int xrows = NT == 1 ? p.M : C::mpad;
     const bool staged_x = !p.xres;
     // FP4: group_size is the scale block (16 or 32), the staged rows are bytes
     constexpr bool FP4 = MODE == w4d::kModeNvfp4 || MODE == w4d::kModeMxfp4;
     p.srow_bytes = FP4 ? 128 : 256;
     p.ngs = GIDX ? 0 : FP4 ? span / g : (g == 32 ? span / 32 : std::min(p.G, (span + 2 * g - 65) / g));
     p.off_x = C::aps * w4d::kTilesPerBand * 512;
-    p.off_xs = p.off_x + (staged_x ? up(C::aps * p.M * 128, 1024) : 0);
-    p.off_sx = p.off_xs + (staged_x ? up(C::aps * xrows * 128, 128) : 0);
+    p.off_xs = p.off_x;
+    p.off_sx = p.off_x + (staged_x ? C::aps * C::mpad * 128 : 0);
     p.off_si = p.off_sx + (staged_x && !GIDX ? C::sx_floats * 4 : 0);
-    p.off_sc = p.off_si + (staged_x && p.s_inv ? C::aps * 256 : 0);
+    p.off_sc = p.off_si;
     p.off_zr = p.off_sc + p.ngs * p.srow_bytes;
     p.off_gi = p.off_zr + (p.zeros ? p.ngs * p.srow_bytes : 0);
     p.off_desc = p.off_gi + (GIDX ? C::aps * 256 : 0);
@@ -228,7 +259,23 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, i
     p.rem = p.units % P;
     p.slots = reinterpret_cast<unsigned long long*>(ws + kCounterBytes);
     CUtensorMap map_x, map_sc, map_zr;
-    if (!make_act_blocks_map(&map_x, X, BF16, p.M, p.K, p.M, C::aps)) return W4_ERR_CUDA;
+    std::memset(&map_x, 0, sizeof(map_x));
+    if (staged_x) {
+        // X' and its sums, prepared once for every CTA (the decode kernel waits for this
+        // kernel before it reads them)
+        const PreLayout L = pre_layout(p.M, p.K);
+        unsigned char* pre = ws + pre_off;
+        p.sg32 = reinterpret_cast<const float*>(pre + L.s32);
+        p.sg64 = reinterpret_cast<const float*>(pre + L.s64);
+        p.sg128 = reinterpret_cast<const float*>(pre + L.s128);
+        const size_t threads = (size_t)C::mpad * (size_t)(p.K / 8);
+        const unsigned blocks = (unsigned)((threads + 255) / 256);
+        w4d::prep_acts_kernel<BF16><<<blocks, 256, 0, stream>>>(
+            X, p.s_inv, p.M, p.K, C::mpad, pre + L.x, const_cast<float*>(p.sg32), const_cast<float*>(p.sg64),
+            const_cast<float*>(p.sg128));
+        if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+        if (!make_act_blocks_map(&map_x, pre + L.x, BF16, p.M, p.K, C::mpad, C::aps)) return W4_ERR_CUDA;
+    }
     map_sc = map_x;
     map_zr = map_x;
     if (!GIDX) {
@@ -262,31 +309,31 @@ int decode_mode(int64_t K, int32_t g, bool gidx) {
 }
 
 template <int NT, bool BF16, bool PERM>
-w4_status dispatch_mode(int mode, w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
+w4_status dispatch_mode(int mode, w4d::DecodeParams p, const void* X, unsigned char* ws, size_t pre_off, int dev,
                         cudaStream_t s) {
     if constexpr (!BF16 && !PERM) {
-        if (mode == w4d::kModeGidx) return launch_decode<NT, false, w4d::kModeGidx, false>(p, X, ws, dev, s);
-        if (mode == w4d::kModeNvfp4) return launch_decode<NT, false, w4d::kModeNvfp4, false>(p, X, ws, dev, s);
-        if (mode == w4d::kModeMxfp4) return launch_decode<NT, false, w4d::kModeMxfp4, false>(p, X, ws, dev, s);
+        if (mode == w4d::kModeGidx) return launch_decode<NT, false, w4d::kModeGidx, false>(p, X, ws, pre_off, dev, s);
+        if (mode == w4d::kModeNvfp4) return launch_decode<NT, false, w4d::kModeNvfp4, false>(p, X, ws, pre_off, dev, s);
+        if (mode == w4d::kModeMxfp4) return launch_decode<NT, false, w4d::kModeMxfp4, false>(p, X, ws, pre_off, dev, s);
     } else {
         if (mode == w4d::kModeGidx || mode == w4d::kModeNvfp4 || mode == w4d::kModeMxfp4) return W4_ERR_UNSUPPORTED;
     }
-    if (mode == w4d::kModeHalf) return launch_decode<NT, BF16, w4d::kModeHalf, PERM>(p, X, ws, dev, s);
-    if (mode == w4d::kModeG32) return launch_decode<NT, BF16, w4d::kModeG32, PERM>(p, X, ws, dev, s);
-    return launch_decode<NT, BF16, w4d::kModeAtom, PERM>(p, X, ws, dev, s);
+    if (mode == w4d::kModeHalf) return launch_decode<NT, BF16, w4d::kModeHalf, PERM>(p, X, ws, pre_off, dev, s);
+    if (mode == w4d::kModeG32) return launch_decode<NT, BF16, w4d::kModeG32, PERM>(p, X, ws, pre_off, dev, s);
+    return launch_decode<NT, BF16, w4d::kModeAtom, PERM>(p, X, ws, pre_off, dev, s);
 }
 
 template <bool BF16>
-w4_status dispatch_decode(int mode, w4d::DecodeParams p, const void* X, unsigned char* ws, int dev,
+w4_status dispatch_decode(int mode, w4d::DecodeParams p, const void* X, unsigned char* ws, size_t pre_off, int dev,
                           cudaStream_t s) {
     // act-order columns gathered while the resident X' is prepared: one token tile only
-    if (p.perm) return decode_tiles_for(p.M) == 1 ? dispatch_mode<1, BF16, true>(mode, p, X, ws, dev, s)
+    if (p.perm) return decode_tiles_for(p.M) == 1 ? dispatch_mode<1, BF16, true>(mode, p, X, ws, pre_off, dev, s)
                                                   : W4_ERR_UNSUPPORTED;
     switch (decode_tiles_for(p.M)) {
-        case 1: return dispatch_mode<1, BF16, false>(mode, p, X, ws, dev, s);
-        case 2: return dispatch_mode<2, BF16, false>(mode, p, X, ws, dev, s);
-        case 4: return dispatch_mode<4, BF16, false>(mode, p, X, ws, dev, s);
-        default: return dispatch_mode<8, BF16, false>(mode, p, X, ws, dev, s);
+        case 1: return dispatch_mode<1, BF16, false>(mode, p, X, ws, pre_off, dev, s);
+        case 2: return dispatch_mode<2, BF16, false>(mode, p, X, ws, pre_off, dev, s);
+        case 4: return dispatch_mode<4, BF16, false>(mode, p, X, ws, pre_off, dev, s);
+        default: return dispatch_mode<8, BF16, false>(mode, p, X, ws, pre_off, dev, s);
     }
 }
 
@@ -456,7 +503,7 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size
     const int dev = current_device();
     const int sms = dev >= 0 ? sm_count(dev) : 0;
     if (sms <= 0) return 0;
-    if (M <= kDecodeMaxM) return decode_workspace_bytes(M, sms);
+    if (M <= kDecodeMaxM) return decode_workspace_bytes(M, K, sms);
     // prefill: scaled activations, behind the zero region and the decode slot region
     return kCounterBytes + slot_region_bytes(sms) + (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
 }
@@ -525,8 +572,9 @@ static w4_status gemm_impl(const void* X, w4_dtype act_dtype, int64_t M, int64_t
         p.tiles = (int)(N / 16);
         unsigned char* ws = reinterpret_cast<unsigned char*>(workspace);
         const int mode = decode_mode(K, group_size, gidx);
-        if (bf16) return dispatch_decode<true>(mode, p, X, ws, dev, strm);
-        return dispatch_decode<false>(mode, p, X, ws, dev, strm);
+        const size_t pre_off = pre_offset(8, sm_count(dev));
+        if (bf16) return dispatch_decode<true>(mode, p, X, ws, pre_off, dev, strm);
+        return dispatch_decode<false>(mode, p, X, ws, pre_off, dev, strm);
     }
 
     const void* Xeff = X;
@@ -567,9 +615,8 @@ size_t w4a16_workspace_bytes_perm(int64_t M, int64_t N, int64_t K, int32_t group
     const int dev = current_device();
     const int sms = dev >= 0 ? sm_count(dev) : 0;
     if (sms <= 0) return 0;
-    // the gathered activations sit where the prefill path keeps its scaled activations:
-    // behind the zero region and the decode slot region, which the GEMM itself uses
-    return kCounterBytes + slot_region_bytes(sms) + (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
+    // the gathered activations sit behind everything the GEMM itself uses
+    return perm_gather_offset(M, K, sms) + (size_t)(((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
 }
 
 w4_status w4a16_gemm_perm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N, int64_t K,
@@ -595,7 +642,7 @@ w4_status w4a16_gemm_perm(const void* X, w4_dtype act_dtype, int64_t M, int64_t 
         return gemm_impl(X, act_dtype, M, N, K, qweight, scales, zeros, nullptr, perm, group_size, s_inv, Y,
                          out_dtype, workspace, workspace_bytes, stream);
     cudaStream_t strm = as_stream(stream);
-    void* xp = reinterpret_cast<unsigned char*>(workspace) + kCounterBytes + slot_region_bytes(sm_count(dev));
+    void* xp = reinterpret_cast<unsigned char*>(workspace) + perm_gather_offset(M, K, sm_count(dev));
     const size_t chunks = (size_t)M * (size_t)K / 8;
     const unsigned blocks = (unsigned)std::min<size_t>((chunks + 255) / 256, (size_t)65535 * 8);
     if (act_dtype == W4_BF16) w4a::gather_acts_kernel<true><<<blocks, 256, 0, strm>>>(X, perm, s_inv, xp, (int)M, (int)K);
@@ -750,6 +797,7 @@ extern "C" w4_status w4_selftest_expired_wait(w4_stream_t stream) {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;   // 8 MiB
+constexpr int kNoAllocMaxTiles = 4;                          // token tiles: M <= 32
 __device__ __align__(256) unsigned char g_w4_noalloc_scratch[kNoAllocScratchBytes];
 
 struct NoAllocScratch {
@@ -810,7 +858,9 @@ extern "C" w4_status w4_selftest_noalloc_scratch(int32_t plant, uint64_t* nonzer
     unsigned char* ws = reinterpret_cast<unsigned char*>(noalloc_scratch(dev));
     if (!ws) return W4_ERR_CUDA;
     unsigned long long* words = reinterpret_cast<unsigned long long*>(ws + kCounterBytes);
-    const size_t n = (kNoAllocScratchBytes - kCounterBytes) / 8;
+    const int sms = sm_count(dev);
+    if (sms <= 0) return W4_ERR_CUDA;
+    const size_t n = decode_slot_bytes(kNoAllocMaxTiles, sms) / 8;   // the split-K slot region
     if (plant) {
         plant_stale_kernel<<<256, 256>>>(words, n);
         if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return W4_ERR_CUDA;
@@ -850,7 +900,9 @@ extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64
     if (dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
     const int sms = sm_count(dev);
     if (sms <= 0) return W4_ERR_CUDA;
-    if (decode_workspace_bytes(M, sms) > kNoAllocScratchBytes) return W4_ERR_UNSUPPORTED;
+    if (decode_tiles_for(M) > kNoAllocMaxTiles ||
+        decode_workspace_bytes(M, K, sms, kNoAllocMaxTiles) > kNoAllocScratchBytes)
+        return W4_ERR_UNSUPPORTED;
     unsigned char* ws = reinterpret_cast<unsigned char*>(noalloc_scratch(dev));
     if (!ws) return W4_ERR_CUDA;
 
@@ -872,8 +924,9 @@ extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64
     p.tiles = (int)(N / 16);
     cudaStream_t strm = as_stream(stream);
     const int mode = decode_mode(K, group_size, gidx);
-    if (bf16) return dispatch_decode<true>(mode, p, X, ws, dev, strm);
-    return dispatch_decode<false>(mode, p, X, ws, dev, strm);
+    const size_t pre_off = pre_offset(kNoAllocMaxTiles, sms);
+    if (bf16) return dispatch_decode<true>(mode, p, X, ws, pre_off, dev, strm);
+    return dispatch_decode<false>(mode, p, X, ws, pre_off, dev, strm);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1127,7 +1180,7 @@ extern "C" size_t w4a16_fp4_workspace_bytes(int64_t M, int64_t N, int64_t K, w4_
     const int dev = current_device();
     const int sms = dev >= 0 ? sm_count(dev) : 0;
     if (sms <= 0) return 0;
-    if (M <= kDecodeMaxM) return decode_workspace_bytes(M, sms);
+    if (M <= kDecodeMaxM) return decode_workspace_bytes(M, K, sms);
     return 0;   // the prefill kernel needs no workspace
 }
 
@@ -1192,5 +1245,6 @@ extern "C" w4_status w4a16_fp4_gemm(const void* X, w4_dtype act_dtype, int64_t M
     p.KA = (int)(K / 64);
     p.tiles = (int)(N / 16);
     const int mode = format == W4_FP4_NVFP4 ? w4d::kModeNvfp4 : w4d::kModeMxfp4;
-    return dispatch_decode<false>(mode, p, X, reinterpret_cast<unsigned char*>(workspace), dev, strm);
+    return dispatch_decode<false>(mode, p, X, reinterpret_cast<unsigned char*>(workspace),
+                                  pre_offset(8, sm_count(dev)), dev, strm);
 }

@@ -346,8 +346,8 @@ w4_status w4a16_fp4_gemm(const void* X, w4_dtype act_dtype, int64_t M, int64_t N
 size_t w4a16_fp4_workspace_bytes(int64_t M, int64_t N, int64_t K, w4_fp4_format format);
 
 /*
- * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 32 (M <= 64 where the scratch fits)
- * without a caller-supplied workspace.  The pages have no counterpart to this call; it
+ * w4a16_gemm_noalloc -- w4a16_gemm for 1 <= M <= 32 without a caller-supplied
+ * workspace.  The pages have no counterpart to this call; it
  * exists for callers that cannot allocate device memory where they run the GEMM, such as
  * plug-ins of inference runtimes that forbid allocation after their set-up phase, or C
  * callers without a caching allocator, for whom cudaMalloc/cudaFree per call would
@@ -355,8 +355,10 @@ size_t w4a16_fp4_workspace_bytes(int64_t M, int64_t N, int64_t K, w4_fp4_format 
  *
  * Arguments, layouts and results are those of w4a16_gemm minus the workspace.  The
  * scratch is one fixed 8 MiB array in device memory that every GPU loading this library
- * holds until the process exits.  Calls whose scratch would exceed it (M above 32 on a
- * 148-SM B200; any M > 64) return W4_ERR_UNSUPPORTED; use w4a16_gemm for them.  The
+ * holds until the process exits: the split-K slots of up to four token tiles, then the
+ * prepared activations (M*K*2 bytes plus their sums, K up to about 48000 at M = 32 on a
+ * 148-SM B200).  Calls beyond it (M > 32, or a larger M*K) return W4_ERR_UNSUPPORTED;
+ * use w4a16_gemm for them.  The
  * first call on a device sets up that device (looks up the array's address, zeroes the
  * array and synchronises the device); make that first call before any stream
  * capture.  If the set-up fails the call returns W4_ERR_CUDA and the next call tries it

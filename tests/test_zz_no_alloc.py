@@ -67,8 +67,9 @@ def test_noalloc_matches_oracle_twice(M, N, K):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    """M = 33 needs eight token tiles of split-K slots (about 9.7 MB on 148 SMs): more
-    than the fixed scratch, so the scratch-size check (not the M <= 64 limit) refuses it."""
+    """M = 33 needs eight token tiles of split-K slots (about 9.7 MB on 148 SMs), more
+    than the fixed scratch holds, so the scratch refuses it (the workspace entry point,
+    whose decode kernel goes to M = 64, runs it)."""
     skip_without_gpu()
     import torch
     K, N, g = 1024, 256, 128
