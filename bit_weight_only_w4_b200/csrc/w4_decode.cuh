@@ -296,6 +296,35 @@ struct StageView {
     int kin, grow;                // first consumed atom: offset in its group, staged group row
 };
 
+// Four 8x8 16-bit matrices from shared memory: lane l gives the address of row l % 8 of
+// matrix l / 8, and register i receives matrix i in the MMA fragment order (thread t:
+// row t / 4, elements 2 (t % 4) and 2 (t % 4) + 1).
+W4_DEV void ldmatrix_x4(uint32_t saddr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(saddr));
+}
+
+// B fragments of 16-deep step j for every token tile of a staged X' ([token row][block]
+// [128 B], rows Cfg::aps * 128 bytes apart, chunks permuted by row): one ldmatrix.x4 per
+// pair of token tiles gives b0, b1 of both (the matrices (tile, k 0-7), (tile, k 8-15)).
+template <int NT>
+W4_DEV void load_b_frags(const unsigned char* xa, int lane, int j, uint32_t (&b0)[NT], uint32_t (&b1)[NT]) {
+    static_assert(NT % 2 == 0, "pairs of token tiles");
+    constexpr int RS = Cfg<NT>::aps * 128;
+    const int m = lane >> 3, rr = lane & 7;
+    const uint32_t base = smem_u32(xa) + (uint32_t)((8 * (m >> 1) + rr) * RS + ((((2 * j + (m & 1)) ^ rr) & 7) << 4));
+#pragma unroll
+    for (int pp = 0; pp < NT / 2; ++pp) {
+        uint32_t r[4];
+        ldmatrix_x4(base + (uint32_t)(pp * 16 * RS), r);
+        b0[2 * pp] = r[0];
+        b1[2 * pp] = r[1];
+        b0[2 * pp + 1] = r[2];
+        b1[2 * pp + 1] = r[3];
+    }
+}
+
 // D(16x8, fp32) = A(16x16) * B(16x8), no accumulator input.
 template <bool BF16>
 W4_DEV void mma_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -316,13 +345,14 @@ W4_DEV void mma_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint
 
 // One 16-deep step of TPW row tiles against NT token tiles; FIRST starts the partial sums.
 template <int NT, int TPW, bool BF16, bool FIRST>
-W4_DEV void mma_step(const uint32_t (&wj)[TPW], const unsigned char* xa, int xl, int xh,
+W4_DEV void mma_step(const uint32_t (&wj)[TPW], const unsigned char* xa, int xl, int xh, int lane, int j,
                      float (&c)[TPW][NT][4]) {
     uint32_t b0[NT], b1[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        b0[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + xl);
-        b1[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + xh);
+    if constexpr (NT >= 2) {
+        load_b_frags<NT>(xa, lane, j, b0, b1);
+    } else {
+        b0[0] = ld_u32(xa + xl);
+        b1[0] = ld_u32(xa + xh);
     }
 #pragma unroll
     for (int tt = 0; tt < TPW; ++tt) {
@@ -391,7 +421,6 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
         // token tile the odd 16-deep steps accumulate into a second register set so
         // consecutive MMAs of a tile do not wait on each other.
         constexpr int CH = NT == 1 ? 2 : 1;
-        constexpr int NTOFF = 8 * Cfg<NT>::aps * 128;   // token tiles of the staged X'
         const unsigned char* xb = v.x + ab * 128;
         const unsigned char* xq[8];
 #pragma unroll
@@ -435,10 +464,11 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
                 for (int j = 0; j < 4; ++j) {
                     const int xo = (2 * pr + aa) * 128;
                     uint32_t b0[NT], b1[NT];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        b0[nt] = ld_u32(xq[2 * j] + xo + nt * NTOFF);
-                        b1[nt] = ld_u32(xq[2 * j + 1] + xo + nt * NTOFF);
+                    if constexpr (NT >= 2) {
+                        load_b_frags<NT>(xb + xo, L.lane, j, b0, b1);
+                    } else {
+                        b0[0] = ld_u32(xq[2 * j] + xo);
+                        b1[0] = ld_u32(xq[2 * j + 1] + xo);
                     }
                     const int st = 4 * aa + j;
 #pragma unroll
@@ -500,7 +530,7 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
                 uint32_t wj[TPW];
 #pragma unroll
                 for (int tt = 0; tt < TPW; ++tt) wj[tt] = word_j<TPW>(w[tt], j);
-                mma_step<NT, TPW, BF16, false>(wj, xa, L.xlo[j], L.xhi[j], c);
+                mma_step<NT, TPW, BF16, false>(wj, xa, L.xlo[j], L.xhi[j], L.lane, j, c);
                 if constexpr (MODE == kModeG32) {
                     if (j & 1) {
                         float2 S32[NT];
@@ -555,10 +585,11 @@ W4_DEV void consume_fp4(const StageView& v, const Lane& L, int t0, int ab, int a
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             uint32_t b0[NT], b1[NT];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                b0[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + L.xlo[j]);
-                b1[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + L.xhi[j]);
+            if constexpr (NT >= 2) {
+                load_b_frags<NT>(xa, L.lane, j, b0, b1);
+            } else {
+                b0[0] = ld_u32(xa + L.xlo[j]);
+                b1[0] = ld_u32(xa + L.xhi[j]);
             }
             const bool first = B == 16 || (j & 1) == 0;
 #pragma unroll
@@ -613,10 +644,11 @@ W4_DEV void consume_gidx(const StageView& v, const DecodeParams& p, const Lane& 
                     gk[e] = 0;
                 }
             uint32_t b0[NT], b1[NT];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                b0[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + L.xlo[j]);
-                b1[nt] = ld_u32(xa + nt * (8 * Cfg<NT>::aps * 128) + L.xhi[j]);
+            if constexpr (NT >= 2) {
+                load_b_frags<NT>(xa, L.lane, j, b0, b1);
+            } else {
+                b0[0] = ld_u32(xa + L.xlo[j]);
+                b1[0] = ld_u32(xa + L.xhi[j]);
             }
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt) {
@@ -813,31 +845,47 @@ W4_DEV int share_slot(int x, int M) {
 }
 
 // MMA thread mt of nthr: for each entry x = mt, mt + nthr, ... of the band, xc[slot] = the
-// sum of the shares CTAs [c_first, cta) published, in CTA order; the loads of up to eight
-// contributors of an entry go out together.  False on a timed-out wait.
+// sum of the shares CTAs [c_first, cta) published, in CTA order.  A thread takes 4 of its
+// entries at a time (2 with one token tile) and loads them from 2 contributors at a time,
+// so up to 8 loads are in flight: with many tokens a band holds thousands of entries
+// (8 tiles x 16 rows x M), and one entry at a time cost one round trip to L2 each.  False
+// on a timed-out wait.
 template <int NT>
 W4_DEV bool sum_shares(const DecodeParams& p, float* xc, int band, int c_first, int cta, int mt, int nthr) {
     constexpr int kSlot = kTilesPerBand * NT * 4 * 32;
+    constexpr int E = NT == 1 ? 2 : 4, CB = 2;   // entries, contributors per round
     const int n_ent = band_tiles(p, band) * 16 * p.M;
-    for (int x = mt; x < n_ent; x += nthr) {
-        const int j = share_slot<NT>(x, p.M);
-        float tot = 0.0f;
-        for (int c0 = c_first; c0 < cta; c0 += 8) {
-            unsigned long long v[8];
+    for (int x0 = mt; x0 < n_ent; x0 += E * nthr) {
+        int j[E];
+        float tot[E];
 #pragma unroll
-            for (int b = 0; b < 8; ++b)
-                v[b] = c0 + b < cta ? slot_get(p.slots + (size_t)(c0 + b) * kSlot + j) : 0ull;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                if (c0 + b >= cta) break;
-                unsigned long long* a = p.slots + (size_t)(c0 + b) * kSlot + j;
-                float val = __uint_as_float((uint32_t)v[b]);
-                if ((v[b] >> 32) == 0 && !slot_wait(a, val)) return false;
-                tot += val;
-                slot_clear(a);
-            }
+        for (int e = 0; e < E; ++e) {
+            const int x = x0 + e * nthr;
+            j[e] = x < n_ent ? share_slot<NT>(x, p.M) : -1;
+            tot[e] = 0.0f;
         }
-        xc[j] = tot;
+        for (int c0 = c_first; c0 < cta; c0 += CB) {
+            unsigned long long v[E][CB];
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+#pragma unroll
+                for (int b = 0; b < CB; ++b)
+                    v[e][b] = (j[e] >= 0 && c0 + b < cta) ? slot_get(p.slots + (size_t)(c0 + b) * kSlot + j[e]) : 0ull;
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+#pragma unroll
+                for (int b = 0; b < CB; ++b) {
+                    if (j[e] < 0 || c0 + b >= cta) continue;
+                    unsigned long long* a = p.slots + (size_t)(c0 + b) * kSlot + j[e];
+                    float val = __uint_as_float((uint32_t)v[e][b]);
+                    if ((v[e][b] >> 32) == 0 && !slot_wait(a, val)) return false;
+                    tot[e] += val;
+                    slot_clear(a);
+                }
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            if (j[e] >= 0) xc[j[e]] = tot[e];
     }
     return true;
 }

@@ -3,6 +3,7 @@
     python profile_case.py decode  [--layer 2] [--m 1] [--iters 12]
     python profile_case.py prefill [--layer 0] [--m 4096] [--iters 6]
     python profile_case.py chain   [--m 1] [--blocks 4] [--iters 3]
+    python profile_case.py fp4     [--layer 2] [--m 1] [--iters 12] [--fmt nvfp4]
 
 decode:  one projection of the Llama-7B-shaped stack (layers 0..3 = qkv 4096x12288,
          o 4096x4096, gate_up 4096x22016, down 11008x4096), fp16 activations with s_inv,
@@ -13,6 +14,8 @@ prefill: one 8B-shaped layer (0 = up 4096x14336, 1 = down 14336x4096), bf16
 chain:   the decode step's projections as one layer sequence (w4a16_gemm_chain): --blocks
          blocks of qkv -> o -> gate_up -> down, each fed from the previous output, one
          weight copy per block (4 blocks = 430 MB of packed weights, above L2).
+fp4:     one 7B projection with NVFP4 or MXFP4 weights (w4a16_fp4_gemm), fp16
+         activations, eight rotated weight copies.
 
 Inputs are the seeded synthetic workloads of bit_weight_only_w4_b200.workloads, quantised
 on the GPU by w4_quantize_pack.  Nothing is checked here (the tests do that); the case only
@@ -29,7 +32,8 @@ def _bits(torch, a, dt):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("kind", choices=["decode", "prefill", "chain"])
+    ap.add_argument("kind", choices=["decode", "prefill", "chain", "fp4"])
+    ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--blocks", type=int, default=4)
     ap.add_argument("--layer", type=int, default=None)
     ap.add_argument("--m", type=int, default=None)
@@ -54,6 +58,18 @@ def main(argv=None):
         for i in range(iters):
             q, s, z = copies[i % len(copies)]
             w4.w4a16_gemm(X, q, s, z, 128, s_inv=s_inv, Y=Y)
+    elif args.kind == "fp4":
+        layer = 2 if args.layer is None else args.layer
+        M = 1 if args.m is None else args.m
+        iters = 12 if args.iters is None else args.iters
+        li = workloads.make_layer(workloads.workload(2), layer, M=M)
+        qw, bs, ts = w4.w4_fp4_quantize_pack(_bits(torch, li.W.view(np.uint16), torch.float16), args.fmt)
+        copies = [(qw, bs)] + [(qw.clone(), bs.clone()) for _ in range(7)]
+        X = _bits(torch, li.X, torch.float16)
+        Y = torch.empty(M, li.N, dtype=torch.float16, device="cuda")
+        for i in range(iters):
+            q, b = copies[i % len(copies)]
+            w4.w4a16_fp4_gemm(X, q, b, ts, args.fmt, Y=Y)
     elif args.kind == "chain":
         import os
         import sys
