@@ -690,6 +690,11 @@ template <bool BF16>
 __global__ void prep_acts_kernel(const void* __restrict__ X, const float* __restrict__ s_inv, int M, int K,
                                  int mpad, void* __restrict__ Xp, float* __restrict__ s32,
                                  float* __restrict__ s64, float* __restrict__ s128) {
+    // launched with programmatic dependent launch: the decode kernel after it may start
+    // its prologue and weight copies at once (it waits for this grid before reading X');
+    // X itself may come from the kernel before
+    pdl_launch_dependents();
+    pdl_wait();
     const int cpt = K / 8;
     const size_t t = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
     const int lane = threadIdx.x & 31;
@@ -845,15 +850,16 @@ W4_DEV int share_slot(int x, int M) {
 }
 
 // MMA thread mt of nthr: for each entry x = mt, mt + nthr, ... of the band, xc[slot] = the
-// sum of the shares CTAs [c_first, cta) published, in CTA order.  A thread takes 4 of its
-// entries at a time (2 with one token tile) and loads them from 2 contributors at a time,
-// so up to 8 loads are in flight: with many tokens a band holds thousands of entries
-// (8 tiles x 16 rows x M), and one entry at a time cost one round trip to L2 each.  False
-// on a timed-out wait.
+// sum of the shares CTAs [c_first, cta) published, in CTA order.  With several token
+// tiles a thread takes 4 of its entries at a time from 2 contributors at a time; with
+// one, one entry from up to 8 contributors: up to 8 loads are in flight either way.
+// False on a timed-out wait.
 template <int NT>
 W4_DEV bool sum_shares(const DecodeParams& p, float* xc, int band, int c_first, int cta, int mt, int nthr) {
     constexpr int kSlot = kTilesPerBand * NT * 4 * 32;
-    constexpr int E = NT == 1 ? 2 : 4, CB = 2;   // entries, contributors per round
+    // up to 8 loads in flight: with one token tile a band has few entries and often 4-8
+    // contributors; with more tiles, thousands of entries
+    constexpr int E = NT == 1 ? 1 : 4, CB = NT == 1 ? 8 : 2;   // entries, contributors per round
     const int n_ent = band_tiles(p, band) * 16 * p.M;
     for (int x0 = mt; x0 < n_ent; x0 += E * nthr) {
         int j[E];

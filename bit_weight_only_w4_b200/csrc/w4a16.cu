@@ -269,11 +269,19 @@ w4_status launch_decode(w4d::DecodeParams p, const void* X, unsigned char* ws, s
         p.sg64 = reinterpret_cast<const float*>(pre + L.s64);
         p.sg128 = reinterpret_cast<const float*>(pre + L.s128);
         const size_t threads = (size_t)C::mpad * (size_t)(p.K / 8);
-        const unsigned blocks = (unsigned)((threads + 255) / 256);
-        w4d::prep_acts_kernel<BF16><<<blocks, 256, 0, stream>>>(
-            X, p.s_inv, p.M, p.K, C::mpad, pre + L.x, const_cast<float*>(p.sg32), const_cast<float*>(p.sg64),
-            const_cast<float*>(p.sg128));
-        if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+        cudaLaunchConfig_t pc = {};
+        pc.gridDim = dim3((unsigned)((threads + 255) / 256));
+        pc.blockDim = dim3(256);
+        pc.stream = stream;
+        cudaLaunchAttribute pa[1];
+        pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pa[0].val.programmaticStreamSerializationAllowed = 1;
+        pc.attrs = pa;
+        pc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&pc, w4d::prep_acts_kernel<BF16>, X, p.s_inv, p.M, p.K, (int)C::mpad,
+                               (void*)(pre + L.x), const_cast<float*>(p.sg32), const_cast<float*>(p.sg64),
+                               const_cast<float*>(p.sg128)) != cudaSuccess)
+            return W4_ERR_CUDA;
         if (!make_act_blocks_map(&map_x, pre + L.x, BF16, p.M, p.K, C::mpad, C::aps)) return W4_ERR_CUDA;
     }
     map_sc = map_x;
