@@ -73,14 +73,21 @@ def _run(layers, workspace=None):
     return [to_f64(d["Y"]) for d in layers]
 
 
+# every layer reads its predecessor's output at a 128-aligned column: each takes its X'
+# from the exchange buffer its predecessor's stores wrote
 SMALL = [(512, 1536, -1, 0), (512, 512, 0, 0), (512, 1024, 1, 0), (768, 512, 2, 256),
+         (512, 768, 3, 0)]
+# layer 1 reads layer 0 at column 64 and layer 2 reads layer 0 (not its predecessor): both
+# prepare X' from Y in the kernel; layers 3 and 4 take it from the exchange buffer
+MIXED = [(512, 1536, -1, 0), (512, 512, 0, 64), (512, 1024, 0, 512), (768, 512, 2, 256),
          (512, 768, 3, 0)]
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 8])
-def test_chain_small_matches_oracle_chain(M):
+@pytest.mark.parametrize("M,specs", [(1, "small"), (2, "small"), (3, "small"), (8, "small"),
+                                     (1, "mixed"), (8, "mixed")])
+def test_chain_small_matches_oracle_chain(M, specs):
     skip_without_gpu()
-    layers, ref32, _ = _build(M, SMALL, seed=M)
+    layers, ref32, _ = _build(M, SMALL if specs == "small" else MIXED, seed=M)
     for _ in range(2):                         # twice: the counter is left at zero
         ys = _run(layers)
         for y, r in zip(ys, ref32):
@@ -118,14 +125,16 @@ def test_chain_longer_than_one_launch_in_a_graph():
             check_y(to_f64(d["Y"]), r, "fp16")
 
 
-def test_chain_matches_separate_gemm_calls():
+@pytest.mark.parametrize("act,specs,M", [("fp16", "small", 3), ("fp16", "mixed", 3), ("bf16", "small", 2),
+                                         ("bf16", "mixed", 1)])
+def test_chain_matches_separate_gemm_calls(act, specs, M):
     """Each layer of the chain computes exactly what w4a16_gemm computes for the same
     input: fed the chain's own intermediate outputs, the separate calls agree bit for bit
-    (same kernel arithmetic, same deterministic split-K order)."""
+    (same kernel arithmetic, same deterministic split-K order; an X' taken from the
+    exchange buffer equals the one prepared from the stored output)."""
     skip_without_gpu()
     import torch
-    M = 3
-    layers, _, _ = _build(M, SMALL, seed=99)
+    layers, _, _ = _build(M, SMALL if specs == "small" else MIXED, seed=99, act=act)
     ys = _run(layers)
     for j, d in enumerate(layers):
         X = d["X"].contiguous()
