@@ -180,11 +180,6 @@ W4_DEV void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// The same between generic-proxy accesses to global memory and bulk copies (async proxy).
-W4_DEV void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // ---------------------------------------------------------------- warp-level MMA
 // D(16x8, fp32) += A(16x16, row) * B(16x8, col); operands fp16 or bf16.
 template <bool BF16>

@@ -943,10 +943,7 @@ extern "C" w4_status w4a16_gemm_noalloc(const void* X, w4_dtype act_dtype, int64
 // ---------------------------------------------------------------------------------------
 namespace {
 
-// [zero region][split-K slots of the single-GEMM kernel][two X' exchange buffers]: the
-// exchange buffers sit where a w4a16_gemm workspace keeps prepared activations, so one
-// workspace serves both (the zero region and the slots are left zero by every launch).
-size_t chain_workspace_bytes(int sms) { return pre_offset(8, sms) + 2 * (size_t)w4c::kXbufBytes; }
+size_t chain_workspace_bytes(int sms) { return kCounterBytes + decode_slot_bytes(1, sms); }
 
 // The layer-sequence kernel keeps every layer's X' and sums resident; up to 120 KB of them
 // still leave the weight ring at least three stages (checked again per launch).
@@ -969,7 +966,7 @@ w4_status launch_chain(w4c::ChainParams& cp, int smem, int grid, int dev, cudaSt
     if (!attr_ok) return W4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(w4c::kThreads);
+    cfg.blockDim = dim3(w4d::Cfg<1>::threads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -984,7 +981,6 @@ w4_status launch_chain(w4c::ChainParams& cp, int smem, int grid, int dev, cudaSt
 // One launch over layers [l0, l0 + n) of the list (n <= kMaxLayers).
 w4_status chain_launch(const w4_chain_layer* layers, int l0, int n, int M, bool bf16, int out_dtype, int mode,
                        unsigned char* ws, int dev, int sms, cudaStream_t stream) {
-    // (out_dtype: 0 fp16, 1 bf16, 2 fp32)
     using C = w4d::Cfg<1>;
     auto up = [](int v, int a) { return (v + a - 1) / a * a; };
     constexpr int kMaxSmem = 227 * 1024;
@@ -1008,7 +1004,7 @@ w4_status chain_launch(const w4_chain_layer* layers, int l0, int n, int M, bool 
     const int off_zr = off_sc + ngs_max * 256;
     const int off_desc = off_zr + (any_zeros ? ngs_max * 256 : 0);
     const int stage_bytes = up(off_desc + 48, 1024);
-    const int fixed = res_x + res_s + C::xchg_bytes + w4c::kExtraSmem + (2 * w4d::kMaxStages + 3) * 8 + 16 + 1024;
+    const int fixed = res_x + res_s + C::xchg_bytes + 3 * w4d::kMaxStages * 8 + 16 + 1024;
     const int stages = std::min(w4d::kMaxStages, (kMaxSmem - fixed) / stage_bytes);
     if (stages < 3) return W4_ERR_UNSUPPORTED;
     const int smem = stages * stage_bytes + fixed;
@@ -1020,21 +1016,6 @@ w4_status chain_launch(const w4_chain_layer* layers, int l0, int n, int M, bool 
     std::memset(&cp, 0, sizeof(cp));
     cp.n_layers = n;
     cp.counter = reinterpret_cast<unsigned int*>(ws);   // word 0 of the zero region
-    cp.xbuf[0] = ws + pre_offset(8, sms);
-    cp.xbuf[1] = cp.xbuf[0] + w4c::kXbufBytes;
-    // layer j+1 takes its X' from layer j's stores when X_{j+1} is a 128-aligned column
-    // slice of Y_j written in the activation type
-    const bool act_out = out_dtype == (bf16 ? 1 : 0);
-    for (int j = 0; j + 1 < n; ++j) {
-        const w4_chain_layer& P = layers[l0 + j];
-        const w4_chain_layer& Q = layers[l0 + j + 1];
-        const auto y = reinterpret_cast<uintptr_t>(P.Y), x = reinterpret_cast<uintptr_t>(Q.X);
-        if (!act_out || x < y || (x - y) % 256 != 0) continue;
-        const int64_t col0 = (int64_t)((x - y) / 2);
-        if (col0 + Q.K > P.N || Q.K % 128 != 0 || (M > 1 && Q.ldx != P.N)) continue;
-        cp.feed[j] = 1;
-        cp.col0[j] = (int)col0;
-    }
     for (int j = 0; j < n; ++j) {
         const w4_chain_layer& Lc = layers[l0 + j];
         w4d::DecodeParams& p = cp.L[j];

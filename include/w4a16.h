@@ -250,10 +250,6 @@ size_t w4_awq_search_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t gr
  * X_{l+1} may point into the output of any earlier layer of the list (a slice of a row:
  * X + offset with row stride ldx).  Each X_l row holds K_l values of act_dtype; Y_l is
  * written in out_dtype, so a layer that feeds a later one wants out_dtype == act_dtype.
- * When X_{l+1} is the slice of Y_l starting at a column that is a multiple of 128 (rows
- * N_l apart), with K_{l+1} % 128 == 0 and out_dtype == act_dtype, the CTAs that store Y_l
- * also write layer l+1's scaled activations X' = X s^-1 and their channel sums to the
- * workspace, and layer l+1 copies them from there; the result is the same bit for bit.
  *
  *   layers     HOST array of n_layers descriptors (read during the call only):
  *                X       device [M, K] activations, rows ldx elements apart
@@ -267,11 +263,9 @@ size_t w4_awq_search_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t gr
  *   every layer must use the same group handling: group sizes all multiples of 128 with
  *              K % 128 == 0, or all 32, or all other multiples of 64
  *   workspace  device, >= w4a16_chain_workspace_bytes(M) bytes, 256-byte aligned,
- *              ZERO-FILLED BEFORE ITS FIRST USE; each launch leaves the parts that must
- *              be zero zero again (the layer counter and split-K slots; the X' exchange
- *              buffers behind them need no particular content); a w4a16_gemm workspace
- *              of at least this size may be shared with it on one stream; after
- *              W4_ERR_TIMEOUT zero it again
+ *              ZERO-FILLED BEFORE ITS FIRST USE; each launch leaves it zero again (a
+ *              w4a16_gemm workspace of at least this size may be shared with it on one
+ *              stream); after W4_ERR_TIMEOUT zero it again
  * All CTAs of a launch (one per SM) must be resident together, which holds when no
  * other work occupies the GPU's SMs; the waits between layers are bounded and report
  * W4_ERR_TIMEOUT through w4_check_device_error() if that is ever violated.

@@ -73,12 +73,12 @@ def _run(layers, workspace=None):
     return [to_f64(d["Y"]) for d in layers]
 
 
-# every layer reads its predecessor's output at a 128-aligned column: each takes its X'
-# from the exchange buffer its predecessor's stores wrote
+# every layer reads its predecessor's output (at columns 0 and 256)
 SMALL = [(512, 1536, -1, 0), (512, 512, 0, 0), (512, 1024, 1, 0), (768, 512, 2, 256),
          (512, 768, 3, 0)]
-# layer 1 reads layer 0 at column 64 and layer 2 reads layer 0 (not its predecessor): both
-# prepare X' from Y in the kernel; layers 3 and 4 take it from the exchange buffer
+# layer 1 reads layer 0 at column 64 (a slice that starts inside a 16-byte chunk of the
+# row) and layer 2 reads layer 0 (not its predecessor); layers 3 and 4 read their
+# predecessors
 MIXED = [(512, 1536, -1, 0), (512, 512, 0, 64), (512, 1024, 0, 512), (768, 512, 2, 256),
          (512, 768, 3, 0)]
 
@@ -130,8 +130,7 @@ def test_chain_longer_than_one_launch_in_a_graph():
 def test_chain_matches_separate_gemm_calls(act, specs, M):
     """Each layer of the chain computes exactly what w4a16_gemm computes for the same
     input: fed the chain's own intermediate outputs, the separate calls agree bit for bit
-    (same kernel arithmetic, same deterministic split-K order; an X' taken from the
-    exchange buffer equals the one prepared from the stored output)."""
+    (same kernel arithmetic, same deterministic split-K order)."""
     skip_without_gpu()
     import torch
     layers, _, _ = _build(M, SMALL if specs == "small" else MIXED, seed=99, act=act)
