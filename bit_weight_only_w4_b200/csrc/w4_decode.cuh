@@ -59,7 +59,7 @@ enum : int {
 template <int NT>
 struct Cfg {
     static constexpr int tpw = NT <= 2 ? 2 : 1;          // row tiles per MMA warp
-    static constexpr int aps = NT == 1 ? 8 : 4;          // atoms (64-channel blocks) per stage
+    static constexpr int aps = NT <= 4 ? 8 : 4;          // atoms (64-channel blocks) per stage
     // no activation warps: X' and its sums arrive prepared (resident, or copied per stage
     // from the copy prep_acts_kernel wrote); every warp but the producer is an MMA warp
     static constexpr int xw = 0;
@@ -416,11 +416,12 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
                     float (&acc)[TPW][NT][4]) {
     const unsigned char* wl = v.codes + t0 * 512 + L.lane * 16;
     if constexpr (MODE == kModeHalf) {
-        // atoms come in pairs, each pair inside one group (at most two pairs per call).
+        // atoms come in pairs, each pair inside one group (at most apk / 2 pairs per call).
         // Every address below is a per-call pointer plus a compile-time offset.  With one
         // token tile the odd 16-deep steps accumulate into a second register set so
         // consecutive MMAs of a tile do not wait on each other.
         constexpr int CH = NT == 1 ? 2 : 1;
+        constexpr int NPR = Cfg<NT>::apk / 2;
         const unsigned char* xb = v.x + ab * 128;
         const unsigned char* xq[8];
 #pragma unroll
@@ -429,10 +430,10 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
             xq[2 * j + 1] = xb + L.xhi[j];
         }
         const int wstride = v.tb * 512;
-        const unsigned char* wp[4];
+        const unsigned char* wp[2 * NPR];
         wp[0] = v.codes + ab * wstride + t0 * 512 + L.lane * 16;
 #pragma unroll
-        for (int k = 1; k < 4; ++k) wp[k] = wp[k - 1] + wstride;
+        for (int k = 1; k < 2 * NPR; ++k) wp[k] = wp[k - 1] + wstride;
         const unsigned char* scp = v.sc + (16 * t0 + L.g8) * 2;
         const unsigned char* zrp = v.zr + (16 * t0 + L.g8) * 2;
         const unsigned char* sxp = v.sx128 + ((ab >> 1) * v.sstride + L.st) * 4;
@@ -440,7 +441,7 @@ W4_DEV void consume(const StageView& v, const Lane& L, int t0, int ab, int ae, i
         int kin = v.kin;
         int grow = v.grow;
 #pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
+        for (int pr = 0; pr < NPR; ++pr) {
             if (ab + 2 * pr >= ae) break;
             uint4 w[2][TPW];
 #pragma unroll
