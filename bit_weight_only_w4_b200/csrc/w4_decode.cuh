@@ -59,7 +59,7 @@ enum : int {
 template <int NT>
 struct Cfg {
     static constexpr int tpw = NT <= 2 ? 2 : 1;          // row tiles per MMA warp
-    static constexpr int aps = NT <= 4 ? 8 : 4;          // atoms (64-channel blocks) per stage
+    static constexpr int aps = 8;                        // atoms (64-channel blocks) per stage: 32 KB of codes
     // no activation warps: X' and its sums arrive prepared (resident, or copied per stage
     // from the copy prep_acts_kernel wrote); every warp but the producer is an MMA warp
     static constexpr int xw = 0;
