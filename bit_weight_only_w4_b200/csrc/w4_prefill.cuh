@@ -95,6 +95,16 @@ struct PrefillParams {
 };
 
 // ---------------------------------------------------------------- tcgen05 wrappers
+// d = a * b + d on two fp32 lanes at once (sm_100 packed fp32 FMA; each lane rounds as
+// fmaf does).
+W4_DEV void fma2(float& d0, float& d1, float a, float b0, float b1) {
+    asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+        "mov.b64 pa, {%2, %2};\n\tmov.b64 pb, {%3, %4};\n\tmov.b64 pd, {%0, %1};\n\t"
+        "fma.rn.f32x2 pd, pa, pb, pd;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a), "f"(b0), "f"(b1));
+}
+
 W4_DEV void tmem_alloc(uint32_t* slot, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(slot)),
@@ -515,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float v[32];
                     tmem_ld32(taddr + 32 * ch, v);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[32 * ch + i] = fmaf(sc, v[i], acc[32 * ch + i]);
+                    for (int i = 0; i < 32; i += 2) fma2(acc[32 * ch + i], acc[32 * ch + i + 1], sc, v[i], v[i + 1]);
                 }
                 tc_fence_before();
                 mbar_arrive(&pempty[pb]);
