@@ -202,8 +202,10 @@ __global__ void __launch_bounds__(w4d::Cfg<1>::threads, 1)
             }
             named_bar_sync(3, kConsumers);
         }
+        int ca0, ca1, cb0, cb1;
+        prep_ranges(p, unit_begin(p, cta), unit_begin(p, cta + 1), ca0, ca1, cb0, cb1);
         prep_resident<BF16, false, true>(p, p.X, smem + p.off_res, reinterpret_cast<float*>(smem + p.off_res_s),
-                                         warp - 1, C::warps - 1, lane);
+                                         warp - 1, C::warps - 1, lane, ca0, ca1, cb0, cb1);
         named_bar_sync(3, kConsumers);
         if (!mma) continue;
         const int u0 = unit_begin(p, cta), u1 = unit_begin(p, cta + 1);

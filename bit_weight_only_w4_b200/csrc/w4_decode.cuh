@@ -739,11 +739,36 @@ __global__ void prep_acts_kernel(const void* __restrict__ X, const float* __rest
 // 64-channel block; sums are [segment][sstride].  Consecutive lanes take consecutive
 // 8-channel chunks, so the sums are warp shuffles; a lane takes its chunk for every token
 // (M <= 8 here), loading the chunk's s_inv once and all M activation chunks together.
+// The 8-channel chunks of X' that the units [u0, u1) read: the whole row when the range
+// holds a band's worth of units, else the K units of the range (one run, or two when
+// the range crosses into the next band), rounded out to 16 chunks and clipped to K.
+W4_DEV void prep_ranges(const DecodeParams& p, int u0, int u1, int& ca0, int& ca1, int& cb0, int& cb1) {
+    const int cpt = p.K / 8;
+    ca0 = ca1 = cb0 = cb1 = 0;
+    if (u0 >= u1) return;
+    if (u1 - u0 >= p.KU) {
+        ca1 = cpt;
+        return;
+    }
+    const int lo = u0 % p.KU, hi = (u1 - 1) % p.KU;
+    if (lo <= hi) {
+        ca0 = 16 * lo;
+        ca1 = min(16 * (hi + 1), cpt);
+    } else {
+        ca0 = 16 * lo;
+        ca1 = cpt;
+        cb1 = min(16 * (hi + 1), cpt);
+    }
+}
+
 // COHERENT: X was written earlier in the same launch by other CTAs (the layer-sequence
 // kernel), so it is read through L2 (ld.global.cg), with rows p.ldx elements apart.
+// Only the chunks [ca0, ca1) and [cb0, cb1) are prepared: the input channels of the CTA's
+// own units (multiples of 16 chunks, i.e. of 128 channels, so that the 32-, 64- and
+// 128-channel sums of a warp's lanes never straddle the two ranges).
 template <bool BF16, bool PERM, bool COHERENT = false>
 W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* xr, float* sr, int w,
-                          int nw, int lane) {
+                          int nw, int lane, int ca0, int ca1, int cb0, int cb1) {
     const int cpt = p.K / 8;                       // chunks per token
     const int rpt = COHERENT ? p.ldx / 8 : cpt;    // chunks between consecutive token rows
     const int ss = p.sstride;
@@ -751,9 +776,12 @@ W4_DEV void prep_resident(const DecodeParams& p, const void* X, unsigned char* x
     float* s64 = s32 + (p.K / 32) * ss;
     float* s128 = s64 + (p.K / 64) * ss;
     const uint4* x4 = reinterpret_cast<const uint4*>(X);
-    for (int base = 32 * w; base < cpt; base += 32 * nw) {
-        const int c = base + lane;
-        const bool valid = c < cpt;
+    // lanes walk the first range, then (from the next multiple of 16 lanes) the second
+    const int na = ca1 - ca0, nb0 = (na + 15) / 16 * 16, nv = nb0 + (cb1 - cb0);
+    for (int base = 32 * w; base < nv; base += 32 * nw) {
+        const int vi = base + lane;
+        const bool valid = vi < na || (vi >= nb0 && vi < nv);
+        const int c = vi < na ? ca0 + vi : cb0 + (vi - nb0);
         float sv[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) sv[i] = 1.0f;
@@ -1190,12 +1218,16 @@ __global__ void __launch_bounds__(Cfg<NT>::threads, 1)
         }
         __syncwarp();
     } else {
+    if constexpr (NT == 1) {   // (the host sets xres for one token tile only)
     if (p.xres) {
         // ------------------------------------------------------------ resident X'
         pdl_wait();   // X may come from the preceding kernel
+        int ca0, ca1, cb0, cb1;
+        prep_ranges(p, u0, u1, ca0, ca1, cb0, cb1);
         prep_resident<BF16, PERM>(p, p.X, smem + p.off_res, reinterpret_cast<float*>(smem + p.off_res_s),
-                            warp - 1, C::warps - 1, lane);
+                                  warp - 1, C::warps - 1, lane, ca0, ca1, cb0, cb1);
         named_bar_sync(3, C::threads - 32);
+    }
     }
     {
         // ------------------------------------------------------------ MMA warps
