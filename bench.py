@@ -885,7 +885,7 @@ def our_arm(args, world, rank, local):
     # dram read + write 48.58 MB against 47.91 MB of codes, scales and zero points); the
     # step's average launch is scaled by its algorithmic bytes (traffic grows with the
     # codes streamed).  Set to None whenever the kernel changes until it is re-captured.
-    TRAFFIC_RATIO = 48.579840 / 47.906816
+    TRAFFIC_RATIO = 48.580608 / 47.906816
     traffic = (TRAFFIC_RATIO * step_bytes / (launches / args.steps)) if TRAFFIC_RATIO else None
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
