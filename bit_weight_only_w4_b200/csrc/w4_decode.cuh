@@ -15,19 +15,21 @@
 //   unit      = 2 column blocks (128 input channels) of one band; all units of the layer
 //               are split into equal contiguous ranges, one per CTA (stream-K), so every
 //               SM streams the same number of bytes whatever N and K are;
-//   stage     = up to 4 units of one band with one token tile (2 with more): the codes
-//               (one bulk copy) and the group rows of scales and zero points (2-D boxes);
-//               staged activations add a 3-D TMA box of column blocks x 8*NT token rows
-//               (128B swizzle, rows >= M zero-filled) and the s_inv slice;
-//   CTA       = 1 producer warp (lane 0 issues a stage's copies), XW activation warps and
-//               16 MMA warps in two groups that take alternate stages (8 in one group at
-//               8 token tiles); one CTA per SM, its ring filling the SM's shared memory,
-//               so every SM holds exactly one CTA of a GEMM even when the next GEMM's CTAs
-//               start early under programmatic dependent launch;
+//   stage     = up to 4 units of one band (32 KB of codes, one bulk copy) and the group
+//               rows of scales and zero points (2-D boxes); staged activations add a 3-D
+//               TMA box of the stage's column blocks x 8*NT token rows of the prepared X'
+//               (rows >= M zero-filled) and three bulk copies of its sums;
+//   CTA       = 1 producer warp (lane 0 issues a stage's copies) and 16 MMA warps in two
+//               groups that take alternate stages (8 in one group with 4 or 8 token
+//               tiles); one CTA per SM, its ring filling the SM's shared memory, so every
+//               SM holds exactly one CTA of a GEMM even when the next GEMM's CTAs start
+//               early under programmatic dependent launch;
 //   activations= with one token tile and a small M*K, X' = X * s_inv and its sums over 32,
-//               64 and 128 channels are prepared once per CTA and stay resident (with
-//               act-order weights packed in permuted order, gathered through perm);
-//               otherwise the activation warps prepare each stage's X' and sums;
+//               64 and 128 channels are prepared by every CTA for the input channels of
+//               its own units and stay resident (with act-order weights packed in
+//               permuted order, gathered through perm); otherwise prep_acts_kernel
+//               prepares them once per GEMM in the workspace, and each stage copies its
+//               slice;
 //   zero point= the MMA multiplies the biased codes o + m*q (o + m*q is what the AND/OR
 //               unpack yields; no subtraction per weight) and the per-group fold removes
 //               the bias and the zero point with the activation sums S = sum_k X'[m,k] of
