@@ -63,6 +63,17 @@ def test_decode_ragged_shapes(N, K):
     case(5, N, K, 64)
 
 
+@pytest.mark.parametrize("M,N,K,g", [(1, 16384, 320, 64), (2, 8192, 576, 64), (8, 12288, 960, 32),
+                                     (3, 4096, 1152, 128)])
+def test_decode_ranges_crossing_bands(M, N, K, g):
+    """More units than CTAs with few units a band, so most CTAs' ranges cross into the
+    next band: each CTA prepares X' for two runs of input channels, with K a multiple of
+    64 but not of 128 in the first three cases (the second run then starts on a half
+    unit of lanes)."""
+    skip_without_gpu()
+    case(M, N, K, g)
+
+
 @pytest.mark.parametrize("g", [32, 64, 128, 256, 1024])
 @pytest.mark.parametrize("sym", [False, True])
 def test_decode_group_sizes(g, sym):
